@@ -1,0 +1,7 @@
+"""CPU fp64 oracle of the chunked H2O attention step.
+
+Test infrastructure only: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline legs of ``bench.py``; never by the product path.
+"""
+from .h2o_oracle import (OracleCache, Placement, attention_one_cache,  # noqa: F401
+                         evict_one_head, gap_at_boundary, kv_head_of, visible_mask)
