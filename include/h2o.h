@@ -1,0 +1,192 @@
+/*
+ * h2o.h -- C ABI of the chunked H2O sparse-attention step on one B200.
+ *
+ * The operation (from "Learning how to Forget: Fine-tuning for Long-Context
+ * Sparse Attention", arXiv 2608.19920):
+ *   - §1 Introduction: keys and values live in a fixed-size KV cache of C
+ *     slots; when the cache is full, a policy evicts slots.  H2O (heavy-hitter
+ *     oracle) is the policy the paper optimises, with dedicated SDPA kernels.
+ *   - §1, second contribution: the SDPA kernel also returns the attention
+ *     weight each key received, summed over queries (and heads).
+ *   - §2 Related work: the summed attention weights are H2O's score input.
+ *   - Summary page, glossary "H2O": cache entries are scored by how often and
+ *     how strongly they were attended; the less important ones are evicted.
+ *
+ * One step, for each independent cache b and KV head g, with G = H_q / H_kv
+ * query heads per KV head, n valid slots and a chunk of n_q tokens at
+ * positions t0 .. t0+n_q-1:
+ *   1. O = softmax(scale * Q K^T) V, where query i of head h (KV head h / G)
+ *      sees the n valid cache slots and chunk keys j <= i.
+ *   2. colsum[b,g,key] = sum over the G heads and the n_q queries of the
+ *      softmax probability that key received.
+ *   3. score[s] += colsum (fp32) for every valid slot s; new token i gets
+ *      candidate score colsum of chunk key i.
+ *   4. If n + n_q <= C the new tokens fill slots n .. n+n_q-1.  Otherwise keep
+ *      every candidate at position >= t0 + n_q - W (recent window) and the
+ *      highest-scoring others up to C entries; ties go to the lower candidate
+ *      index (slot s -> s, new token i -> C + i).  The kept new tokens, in
+ *      ascending order, move into the freed and empty slots in ascending
+ *      order; kept entries stay in place.
+ *   5. n <- min(C, n + n_q); t0 <- t0 + n_q.
+ *
+ * Layouts (row-major, contiguous, every base pointer 16-byte aligned; the
+ * workspace 256-byte aligned):
+ *   q, out            [batch, n_q, H_q, head_dim]      element type = dtype
+ *   k_new, v_new      [batch, n_q, H_kv, head_dim]     element type = dtype
+ *   cache k, v        [batch, H_kv, capacity, head_dim] element type = dtype
+ *   scores            [batch, H_kv, capacity]          float32
+ *   pos               [batch, H_kv, capacity]          int32, -1 = empty slot
+ *   state             [4] int32: n, t0, device error bits, reserved
+ *   colsum (in/out)   [batch, H_kv, capacity + n_q]    float32; entry s < n is
+ *                     cache slot s, entries n .. capacity-1 are 0, entry
+ *                     capacity + j is chunk key j.
+ *
+ * Conventions:
+ *   - Every call is asynchronous on the given CUDA stream (NULL = legacy
+ *     default stream).  Argument errors are returned synchronously, before
+ *     anything is launched.  Errors detected on the device (a bounded wait
+ *     that expired, an inconsistent eviction plan) are latched in state[2]
+ *     and returned by h2o_cache_check().
+ *   - All memory is owned by the caller; the library allocates nothing on
+ *     the device.  h2o_cache_destroy() frees only the host handle.
+ *   - All caches of a handle advance together (one n_q per call).  A handle
+ *     must not be used from two host threads at once.
+ *   - Supported: head_dim 64 or 128; dtype BF16 (tensor-core path) or F32
+ *     (fp32 FMA path); H_q a multiple of H_kv; 0 <= recent_window <=
+ *     capacity; capacity + max_chunk <= 50176 (the selection keeps one fp32
+ *     key per candidate in shared memory).
+ */
+#ifndef H2O_H_
+#define H2O_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define H2O_API __attribute__((visibility("default")))
+#else
+#define H2O_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  H2O_OK = 0,
+  H2O_ERR_INVALID_ARG = 1, /* null pointer, n_q out of range, bad handle     */
+  H2O_ERR_SHAPE = 2,       /* unsupported sizes, buffer too small            */
+  H2O_ERR_DTYPE = 3,       /* unknown dtype                                  */
+  H2O_ERR_ALIGN = 4,       /* pointer not 16-byte (workspace: 256-byte) aligned */
+  H2O_ERR_CUDA = 5,        /* a CUDA runtime call failed                     */
+  H2O_ERR_TIMEOUT = 6,     /* a kernel's bounded wait expired (device bit 1) */
+  H2O_ERR_STATE = 7        /* inconsistent eviction plan (device bit 2)      */
+} h2o_status;
+
+typedef enum { H2O_BF16 = 0, H2O_F32 = 1 } h2o_dtype;
+
+typedef struct {
+  int32_t batch;          /* independent caches (layers x sequences), >= 1   */
+  int32_t n_q_heads;      /* H_q                                             */
+  int32_t n_kv_heads;     /* H_kv, divides H_q                               */
+  int32_t head_dim;       /* 64 or 128                                       */
+  int32_t capacity;       /* C, slots per (cache, KV head)                   */
+  int32_t max_chunk;      /* largest n_q accepted by the step calls          */
+  int32_t recent_window;  /* W, 0 <= W <= C                                  */
+  h2o_dtype dtype;        /* element type of q, k, v, out and the cache      */
+  float softmax_scale;    /* <= 0 selects 1/sqrt(head_dim)                   */
+} h2o_config;
+
+/* Byte sizes of the caller-owned device buffers for a configuration. */
+typedef struct {
+  size_t k_bytes, v_bytes;  /* cache K and V                                 */
+  size_t scores_bytes;      /* float32 scores                                */
+  size_t pos_bytes;         /* int32 positions                               */
+  size_t state_bytes;       /* 4 x int32                                     */
+  size_t workspace_bytes;   /* row statistics, summed weights, eviction plan,
+                               and staging for h2o_chunk_step_host           */
+} h2o_sizes;
+
+/* Caller-owned device buffers (sizes from h2o_required_bytes). */
+typedef struct {
+  void* k;
+  void* v;
+  float* scores;
+  int32_t* pos;
+  int32_t* state;
+  void* workspace;
+  size_t workspace_bytes;
+} h2o_buffers;
+
+typedef struct h2o_cache h2o_cache;
+
+/* Validates cfg and fills *out.  Host only; touches no device. */
+H2O_API h2o_status h2o_required_bytes(const h2o_config* cfg, h2o_sizes* out);
+
+/* Creates a handle over caller-owned buffers and, on `stream`, clears the
+ * cache to the empty state (K, V, scores = 0; pos = -1; n = t0 = 0; no
+ * error).  The buffers must stay valid until h2o_cache_destroy. */
+H2O_API h2o_status h2o_cache_create(const h2o_config* cfg, const h2o_buffers* bufs,
+                            void* stream, h2o_cache** out);
+
+/* The whole step (attention with summed weights, score update, selection,
+ * placement) for all caches.  q, k_new, v_new, out: device pointers in the
+ * layouts above with 1 <= n_q <= max_chunk (n_q = 0 is a no-op).
+ * colsum_out (device, may be NULL) receives the summed weights in the colsum
+ * layout.  Advances n and t0. */
+H2O_API h2o_status h2o_chunk_step(h2o_cache* c, const void* q, const void* k_new,
+                          const void* v_new, int32_t n_q, void* out,
+                          float* colsum_out, void* stream);
+
+/* Same step with HOST buffers (pinned memory recommended): the inputs are
+ * copied into the workspace's staging area, the step runs, and out (and
+ * colsum_out, may be NULL) are copied back, all on `stream`.  The host
+ * buffers must stay untouched until the stream reaches this point. */
+H2O_API h2o_status h2o_chunk_step_host(h2o_cache* c, const void* q_host,
+                               const void* k_new_host, const void* v_new_host,
+                               int32_t n_q, void* out_host,
+                               float* colsum_out_host, void* stream);
+
+/* Steps 1-2 only: out and colsum_out (both device; colsum_out may be NULL)
+ * for the current cache contents.  The cache state does not change. */
+H2O_API h2o_status h2o_attention(h2o_cache* c, const void* q, const void* k_new,
+                         const void* v_new, int32_t n_q, void* out,
+                         float* colsum_out, void* stream);
+
+/* Steps 3-5 only, with caller-supplied summed weights `colsum` (device,
+ * colsum layout for this n_q, float32).  Advances n and t0. */
+H2O_API h2o_status h2o_evict(h2o_cache* c, const float* colsum, const void* k_new,
+                     const void* v_new, int32_t n_q, void* stream);
+
+/* Copies the cache state out.  k, v, scores, pos may each be NULL or a
+ * device or host pointer (the copy kind is inferred); n_t0 (host, may be
+ * NULL) receives {n, t0}. */
+H2O_API h2o_status h2o_cache_read(const h2o_cache* c, void* k, void* v, float* scores,
+                          int32_t* pos, int32_t* n_t0, void* stream);
+
+/* Replaces the cache state (checkpoint restore).  Pointers as in
+ * h2o_cache_read (all four required); n_t0 (host) = {n, t0} with
+ * 0 <= n <= capacity and t0 >= n.  Clears the device error bits. */
+H2O_API h2o_status h2o_cache_write(h2o_cache* c, const void* k, const void* v,
+                           const float* scores, const int32_t* pos,
+                           const int32_t* n_t0, void* stream);
+
+/* Synchronises `stream` and returns the device error bits as a status:
+ * H2O_OK, H2O_ERR_TIMEOUT or H2O_ERR_STATE (or H2O_ERR_CUDA). */
+H2O_API h2o_status h2o_cache_check(h2o_cache* c, void* stream);
+
+/* Host-side view of the handle: n, t0 and the number of kernels launched
+ * through it so far (each may be NULL). */
+H2O_API h2o_status h2o_cache_info(const h2o_cache* c, int32_t* n, int32_t* t0,
+                          uint64_t* kernel_launches);
+
+/* Frees the host handle only. */
+H2O_API void h2o_cache_destroy(h2o_cache* c);
+
+H2O_API const char* h2o_status_string(h2o_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* H2O_H_ */

@@ -1,0 +1,37 @@
+// attn.h -- launchers of the attention kernels (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.h"
+
+namespace h2o {
+
+// TMA descriptors of one call (bf16 path).
+struct AttnMaps {
+  CUtensorMap q;   // [B, nq, Hq, d]     box (64, 1, 128, 1)
+  CUtensorMap kc;  // [B*Hkv, n, d]      box (64, 128, 1)   rows >= n read as zero
+  CUtensorMap vc;
+  CUtensorMap kn;  // [B, nq, Hkv, d]    box (64, 1, 128, 1) rows >= nq read as zero
+  CUtensorMap vn;
+};
+
+// Records that a kernel's shared-memory opt-in was set on the current device.
+bool smem_attr_done(const void* fn, int* slot_bits);
+
+// K1: attention forward + row statistics (tcgen05), head_dim 64 or 128.
+cudaError_t launch_attn_fwd_bf16(int head_dim, const AttnMaps& m, const AttnParams& p,
+                                 cudaStream_t st);
+// K2: summed attention weights per key (tcgen05), head_dim 64 or 128.
+cudaError_t launch_attn_colsum_bf16(int head_dim, const AttnMaps& m, const AttnParams& p,
+                                    cudaStream_t st);
+// fp32 path (FMA): K1 and K2 for float inputs.
+cudaError_t launch_attn_f32(int head_dim, const float* q, const float* kc, const float* vc,
+                            const float* kn, const float* vn, const AttnParams& p,
+                            cudaStream_t st);
+
+// K3 + K4: score update, selection, placement and K/V scatter.
+cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st);
+
+}  // namespace h2o

@@ -1,0 +1,259 @@
+// attn_colsum.cu -- summed attention weights per key on sm_100a tensor cores.
+//
+// colsum[b, g, key] = sum over the G query heads of KV head g and the chunk's
+// queries of softmax probability P[h, i, key] ("Learning how to Forget", §1:
+// the SDPA kernel returns summed attention weights, the H2O score input).
+// P is rebuilt from the logits and the row statistic lse2 written by the
+// forward kernel: P = 2^(x - lse2), x = scale*log2(e)*<q, k>.  Nothing of P
+// is stored.
+//
+// Key-stationary: one CTA per (cache, KV head, tile of 128 keys).  The MMA
+// computes S^T = K_tile Q_rows^T with the keys on the 128 TMEM lanes, so every
+// thread owns one key and sums its probabilities along its own TMEM row: the
+// column sum needs no cross-thread reduction.  Rows are processed in tiles of
+// 128 queries of one head; the sum order is fixed, so results are
+// deterministic (no atomics).
+//   warp 0      TMA producer: the key tile once, then Q tiles + their lse2
+//   warp 1      TMEM allocation; one thread issues the tcgen05.mma
+//   warps 2..9  two threads per key: columns 0..63 and 64..127 of each tile
+#include "attn.h"
+#include "sm100.cuh"
+
+namespace h2o {
+
+template <int D>
+struct ColLayout {
+  static constexpr int kRegions = D / 64;
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kQStages = 2;
+  static constexpr int kKOff = 0;
+  static constexpr int kQOff = kKOff + kTileBytes;
+  static constexpr int kLseOff = kQOff + kQStages * kTileBytes;  // 512 bytes per stage
+  static constexpr int kBarOff = kLseOff + kQStages * 512;
+  // k_full, q_full[S], q_empty[S], s_full[2], s_empty[2], drain
+  static constexpr int kNumBars = 1 + 2 * kQStages + 4 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kRedOff = kMiscOff + 16;
+  static constexpr int kBytes = kRedOff + 128 * 4;
+  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr int kTmemCols = 256;
+  static constexpr int kThreads = 320;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 2)
+    attn_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_kc,
+                       const __grid_constant__ CUtensorMap tm_kn, const AttnParams p) {
+  using L = ColLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int bg = blockIdx.y;
+  const int b = bg / p.Hkv;
+  const int g = bg % p.Hkv;
+  const int NCTC = cdiv(p.C, 128);  // key tiles covering the whole capacity
+  const int NQT = cdiv(p.nq, 128);
+  const bool is_chunk = static_cast<int>(blockIdx.x) >= NCTC;
+  const int kt = is_chunk ? blockIdx.x - NCTC : blockIdx.x;
+  const int j0 = kt * 128;
+  float* out = p.colsum + static_cast<size_t>(bg) * p.colsum_ld;
+
+  if (!is_chunk && j0 >= p.n) {
+    // slots beyond the valid ones received no weight
+    for (int j = j0 + threadIdx.x; j < min(j0 + 128, p.C); j += blockDim.x) out[j] = 0.f;
+    return;
+  }
+  const int qt_min = is_chunk ? kt : 0;  // a chunk key is seen by queries i >= key
+  const int span = NQT - qt_min;
+  const int R = p.G * span;
+
+  const uint32_t bar_k = sbase + L::kBarOff;
+  const uint32_t bar_q_full0 = bar_k + 8;
+  const uint32_t bar_q_empty0 = bar_q_full0 + 8 * L::kQStages;
+  const uint32_t bar_s_full0 = bar_q_empty0 + 8 * L::kQStages;
+  const uint32_t bar_s_empty0 = bar_s_full0 + 16;
+  const uint32_t bar_drain = bar_s_empty0 + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  float* red = reinterpret_cast<float*>(smem + L::kRedOff);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_k, 1);
+    for (int s = 0; s < L::kQStages; ++s) {
+      mbar_init(bar_q_full0 + 8 * s, 1);
+      mbar_init(bar_q_empty0 + 8 * s, 1 + 256);  // MMA commit + every summing thread
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_s_full0 + 8 * s, 1);
+      mbar_init(bar_s_empty0 + 8 * s, 256);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_k, L::kTileBytes);
+      for (int r = 0; r < L::kRegions; ++r) {
+        if (is_chunk)
+          tma_load_4d(sbase + L::kKOff + r * 16384, &tm_kn, bar_k, r * 64, g, j0, b);
+        else
+          tma_load_3d(sbase + L::kKOff + r * 16384, &tm_kc, bar_k, r * 64, j0, b * p.Hkv + g);
+      }
+      int issued = 0;
+      for (int u = 0; u < R; ++u) {
+        const int s = u % L::kQStages;
+        if (u >= L::kQStages &&
+            !mbar_wait(bar_q_empty0 + 8 * s, ((u / L::kQStages) + 1) & 1, p.err, abort_flag))
+          break;
+        const int h = g * p.G + u / span;
+        const int qt = qt_min + u % span;
+        const uint32_t bar = bar_q_full0 + 8 * s;
+        mbar_arrive_expect_tx(bar, L::kTileBytes + 512);
+        const uint32_t dst = sbase + L::kQOff + s * L::kTileBytes;
+        for (int r = 0; r < L::kRegions; ++r)
+          tma_load_4d(dst + r * 16384, &tm_q, bar, r * 64, h, qt * 128, b);
+        bulk_load(sbase + L::kLseOff + s * 512,
+                  p.lse2 + (static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + qt * 128, 512, bar);
+        issued = u + 1;
+      }
+      mbar_wait_drain(bar_k, 0, p.err);
+      for (int u = (issued > L::kQStages ? issued - L::kQStages : 0); u < issued; ++u)
+        mbar_wait_drain(bar_q_full0 + 8 * (u % L::kQStages), (u / L::kQStages) & 1, p.err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, false, false);
+      bool ok = mbar_wait(bar_k, 0, p.err, abort_flag);
+      for (int u = 0; u < R && ok; ++u) {
+        const int s = u % L::kQStages;
+        const int sb = u & 1;
+        ok = mbar_wait(bar_q_full0 + 8 * s, (u / L::kQStages) & 1, p.err, abort_flag);
+        if (ok && u >= 2) ok = mbar_wait(bar_s_empty0 + 8 * sb, ((u >> 1) + 1) & 1, p.err, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t qbase = sbase + L::kQOff + s * L::kTileBytes;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_bf16_ss(tmem + sb * 128, sw128_desc(sbase + L::kKOff + off, 16, 1024),
+                      sw128_desc(qbase + off, 16, 1024), kIdesc, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_s_full0 + 8 * sb);
+        mma_commit(bar_q_empty0 + 8 * s);
+      }
+      mma_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0, p.err);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;  // 0: columns 0..63, 1: columns 64..127
+    const int row = quad * 32 + lane;  // key j0 + row
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16) + half * 64;
+    const float c = p.scale_log2;
+    float acc = 0.f;
+    bool ok = true;
+    for (int u = 0; u < R; ++u) {
+      const int s = u % L::kQStages;
+      const int sb = u & 1;
+      ok = mbar_wait(bar_s_full0 + 8 * sb, (u >> 1) & 1, p.err, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      tmem_ld32(lane_base + sb * 128, v0);
+      tmem_ld32(lane_base + sb * 128 + 32, v1);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar_s_empty0 + 8 * sb);
+      // lse2 of this row tile (already landed: the MMA waited for it)
+      ok = mbar_wait(bar_q_full0 + 8 * s, (u / L::kQStages) & 1, p.err, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const float4* lse4 = reinterpret_cast<const float4*>(smem + L::kLseOff + s * 512) + half * 16;
+      const int qt = qt_min + u % span;
+      // on the diagonal tile query i0+col sees key j0+row iff row <= col
+      const int first_col = (is_chunk && qt == kt) ? row - half * 64 : 0;
+      float part = 0.f;
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 ls = lse4[q4];
+        const float l4[4] = {ls.x, ls.y, ls.z, ls.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int col = q4 * 4 + e;
+          const float pr = ex2_approx(__uint_as_float(v0[col]) * c - l4[e]);
+          part += (col >= first_col) ? pr : 0.f;
+        }
+      }
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 ls = lse4[8 + q4];
+        const float l4[4] = {ls.x, ls.y, ls.z, ls.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int col = 32 + q4 * 4 + e;
+          const float pr = ex2_approx(__uint_as_float(v1[q4 * 4 + e]) * c - l4[e]);
+          part += (col >= first_col) ? pr : 0.f;
+        }
+      }
+      acc += part;
+      mbar_arrive(bar_q_empty0 + 8 * s);
+    }
+    // combine the two column halves in a fixed order
+    if (half == 1) red[row] = acc;
+    named_bar_sync(1, 256);
+    if (half == 0 && ok) {
+      const float total = acc + red[row];
+      const int key = j0 + row;
+      if (is_chunk) {
+        if (key < p.nq) out[p.C + key] = total;
+      } else if (key < p.n) {
+        out[key] = total;
+      } else if (key < p.C) {
+        out[key] = 0.f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+template <int D>
+static cudaError_t launch_colsum(const AttnMaps& m, const AttnParams& p, cudaStream_t st) {
+  using L = ColLayout<D>;
+  static int attr_bits[2] = {0, 0};
+  if (!smem_attr_done(reinterpret_cast<const void*>(attn_colsum_kernel<D>), attr_bits)) {
+    cudaError_t e = cudaFuncSetAttribute(attn_colsum_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(cdiv(p.C, 128) + cdiv(p.nq, 128), p.B * p.Hkv);
+  attn_colsum_kernel<D><<<grid, L::kThreads, L::kAlloc, st>>>(m.q, m.kc, m.kn, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_colsum_bf16(int head_dim, const AttnMaps& m, const AttnParams& p,
+                                    cudaStream_t st) {
+  return head_dim == 128 ? launch_colsum<128>(m, p, st) : launch_colsum<64>(m, p, st);
+}
+
+}  // namespace h2o

@@ -1,0 +1,61 @@
+// common.h -- definitions shared by the host API and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+namespace h2o {
+
+// Device error bits, latched in state[2].
+constexpr int kDevErrTimeout = 1;  // a bounded mbarrier wait expired
+constexpr int kDevErrPlan = 2;     // freed-slot and kept-token counts disagree
+
+// Longest time a kernel thread waits on one mbarrier phase before it gives up.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+constexpr int kTileRows = 128;  // query rows per attention tile (TMEM lanes)
+constexpr int kTileKeys = 128;  // keys per attention tile
+
+// Largest capacity + max_chunk the selection kernel keeps in shared memory.
+constexpr int kMaxCandidates = 50176;
+
+__host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------- attention
+
+// Arguments of the tensor-core attention kernel and the column-sum kernel.
+struct AttnParams {
+  int B, Hq, Hkv, G;    // caches, query heads, KV heads, heads per group
+  int nq;               // chunk length of this call
+  int n;                // valid cache slots
+  int C;                // capacity
+  int nq_pad;           // row stride of the row statistics (multiple of 128)
+  float scale_log2;     // softmax scale * log2(e)
+  void* out;            // [B, nq, Hq, d]
+  float* lse2;          // [B, Hq, nq_pad], log2-domain log-sum-exp per row
+  float* colsum;        // [B, Hkv, colsum_ld]
+  int colsum_ld;        // row stride of colsum (>= C + nq)
+  int* err;             // device error word (state + 2)
+};
+
+// ---------------------------------------------------------------- eviction
+
+struct EvictParams {
+  int B, Hkv, C, d, esize;  // esize: bytes per element of K/V
+  int n, t0, nq, W;
+  const float* colsum;      // [B, Hkv, colsum_ld]
+  int colsum_ld;
+  float* scores;            // [B, Hkv, C]
+  int* pos;                 // [B, Hkv, C]
+  int* plan_slots;          // [B, Hkv, max_chunk]
+  int* plan_tokens;         // [B, Hkv, max_chunk]
+  int* plan_count;          // [B, Hkv]
+  int plan_ld;              // max_chunk
+  const void* k_new;        // [B, nq, Hkv, d]
+  const void* v_new;
+  void* k_cache;            // [B, Hkv, C, d]
+  void* v_cache;
+  int* state;               // [4]: n, t0, err, reserved
+};
+
+}  // namespace h2o

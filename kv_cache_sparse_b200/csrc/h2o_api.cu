@@ -1,0 +1,461 @@
+// h2o_api.cu -- host side of the C ABI declared in include/h2o.h.
+//
+// Validates arguments, lays out the caller's workspace, encodes the TMA
+// descriptors of each call and launches the four kernels of a step on the
+// caller's stream:
+//   K1 attention forward + row statistics   (attn_fwd.cu, tcgen05)
+//   K2 summed attention weights per key     (attn_colsum.cu, tcgen05)
+//   K3 score update + top-C selection       (evict.cu)
+//   K4 K/V scatter into the freed slots     (evict.cu)
+// Float32 caches use the fp32 kernels of attn_f32.cu for K1/K2.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "../../include/h2o.h"
+#include "attn.h"
+
+using namespace h2o;
+
+struct h2o_cache {
+  h2o_config cfg;
+  h2o_buffers buf;
+  int n = 0;
+  int t0 = 0;
+  uint64_t launches = 0;
+  // workspace carve-up
+  int nq_pad = 0;     // row stride of lse2
+  int colsum_ld = 0;  // row stride of colsum
+  float* lse2 = nullptr;
+  float* colsum = nullptr;
+  int* plan_slots = nullptr;
+  int* plan_tokens = nullptr;
+  int* plan_count = nullptr;
+  uint8_t* stage_q = nullptr;
+  uint8_t* stage_kn = nullptr;
+  uint8_t* stage_vn = nullptr;
+  uint8_t* stage_out = nullptr;
+};
+
+namespace {
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t esize_of(h2o_dtype t) { return t == H2O_BF16 ? 2 : 4; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Layout {
+  size_t lse, colsum, slots, tokens, count, sq, skn, svn, sout, total;
+  int nq_pad, colsum_ld;
+};
+
+Layout workspace_layout(const h2o_config& c) {
+  Layout L{};
+  const size_t e = esize_of(c.dtype);
+  const size_t BHkv = static_cast<size_t>(c.batch) * c.n_kv_heads;
+  L.nq_pad = static_cast<int>(round_up(c.max_chunk, 128));
+  L.colsum_ld = static_cast<int>(round_up(static_cast<size_t>(c.capacity) + c.max_chunk, 4));
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = round_up(off + bytes, 256);
+    return at;
+  };
+  L.lse = take(static_cast<size_t>(c.batch) * c.n_q_heads * L.nq_pad * 4);
+  L.colsum = take(BHkv * L.colsum_ld * 4);
+  L.slots = take(BHkv * c.max_chunk * 4);
+  L.tokens = take(BHkv * c.max_chunk * 4);
+  L.count = take(BHkv * 4);
+  const size_t rows = static_cast<size_t>(c.batch) * c.max_chunk * c.head_dim * e;
+  L.sq = take(rows * c.n_q_heads);
+  L.skn = take(rows * c.n_kv_heads);
+  L.svn = take(rows * c.n_kv_heads);
+  L.sout = take(rows * c.n_q_heads);
+  L.total = off;
+  return L;
+}
+
+h2o_status check_config(const h2o_config* c) {
+  if (!c) return H2O_ERR_INVALID_ARG;
+  if (c->dtype != H2O_BF16 && c->dtype != H2O_F32) return H2O_ERR_DTYPE;
+  if (c->batch < 1 || c->n_q_heads < 1 || c->n_kv_heads < 1 || c->capacity < 1 ||
+      c->max_chunk < 1)
+    return H2O_ERR_SHAPE;
+  if (c->n_q_heads % c->n_kv_heads != 0) return H2O_ERR_SHAPE;
+  if (c->head_dim != 64 && c->head_dim != 128) return H2O_ERR_SHAPE;
+  if (c->recent_window < 0 || c->recent_window > c->capacity) return H2O_ERR_SHAPE;
+  if (static_cast<long long>(c->capacity) + c->max_chunk > kMaxCandidates) return H2O_ERR_SHAPE;
+  if (static_cast<long long>(c->batch) * c->n_kv_heads > 65535) return H2O_ERR_SHAPE;
+  if (static_cast<long long>(c->batch) * c->n_q_heads * cdiv(c->max_chunk, 128) > (1ll << 31) - 1)
+    return H2O_ERR_SHAPE;
+  return H2O_OK;
+}
+
+// ---------------------------------------------------------------- TMA encoding
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor of `rank` dims (innermost first), 128-byte swizzled boxes
+bool encode_bf16(CUtensorMap* tm, const void* base, int rank, const cuuint64_t* dims,
+                 const cuuint64_t* strides, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [B, nq, H, d] chunk tensors: dims (d, H, nq, B), box (64, 1, 128, 1)
+bool encode_chunk(CUtensorMap* tm, const void* base, int B, int nq, int H, int d) {
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)nq, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2,
+                                 (cuuint64_t)nq * H * d * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  return encode_bf16(tm, base, 4, dims, strides, box);
+}
+
+// [B*Hkv, C, d] cache with only the first n rows visible: dims (d, n, B*Hkv)
+bool encode_cache(CUtensorMap* tm, const void* base, int BH, int n, int C, int d) {
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)(n > 0 ? n : 1), (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)C * d * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  return encode_bf16(tm, base, 3, dims, strides, box);
+}
+
+h2o_status cuda_status(cudaError_t e) { return e == cudaSuccess ? H2O_OK : H2O_ERR_CUDA; }
+
+h2o_status check_step_args(h2o_cache* c, const void* q, const void* kn, const void* vn, int nq,
+                           const void* out) {
+  if (!c) return H2O_ERR_INVALID_ARG;
+  if (nq < 0 || nq > c->cfg.max_chunk) return H2O_ERR_INVALID_ARG;
+  if (nq == 0) return H2O_OK;
+  if (!q || !kn || !vn || !out) return H2O_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kn, 16) || !aligned(vn, 16) || !aligned(out, 16))
+    return H2O_ERR_ALIGN;
+  return H2O_OK;
+}
+
+AttnParams attn_params(h2o_cache* c, int nq, void* out) {
+  const h2o_config& g = c->cfg;
+  AttnParams p;
+  p.B = g.batch;
+  p.Hq = g.n_q_heads;
+  p.Hkv = g.n_kv_heads;
+  p.G = g.n_q_heads / g.n_kv_heads;
+  p.nq = nq;
+  p.n = c->n;
+  p.C = g.capacity;
+  p.nq_pad = c->nq_pad;
+  const float scale = g.softmax_scale > 0.f ? g.softmax_scale : 1.f / sqrtf((float)g.head_dim);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = out;
+  p.lse2 = c->lse2;
+  p.colsum = c->colsum;
+  p.colsum_ld = c->colsum_ld;
+  p.err = c->buf.state + 2;
+  return p;
+}
+
+// K1 + K2 into the workspace (lse2, colsum) and `out`.
+h2o_status run_attention(h2o_cache* c, const void* q, const void* kn, const void* vn, int nq,
+                         void* out, cudaStream_t st) {
+  const h2o_config& g = c->cfg;
+  AttnParams p = attn_params(c, nq, out);
+  if (g.dtype == H2O_F32) {
+    cudaError_t e = launch_attn_f32(g.head_dim, static_cast<const float*>(q),
+                                    static_cast<const float*>(c->buf.k),
+                                    static_cast<const float*>(c->buf.v),
+                                    static_cast<const float*>(kn), static_cast<const float*>(vn),
+                                    p, st);
+    c->launches += (c->n < g.capacity) ? 3 : 2;
+    return cuda_status(e);
+  }
+  AttnMaps m;
+  const int BH = g.batch * g.n_kv_heads;
+  if (!encode_chunk(&m.q, q, g.batch, nq, g.n_q_heads, g.head_dim) ||
+      !encode_chunk(&m.kn, kn, g.batch, nq, g.n_kv_heads, g.head_dim) ||
+      !encode_chunk(&m.vn, vn, g.batch, nq, g.n_kv_heads, g.head_dim) ||
+      !encode_cache(&m.kc, c->buf.k, BH, c->n, g.capacity, g.head_dim) ||
+      !encode_cache(&m.vc, c->buf.v, BH, c->n, g.capacity, g.head_dim))
+    return H2O_ERR_CUDA;
+  cudaError_t e = launch_attn_fwd_bf16(g.head_dim, m, p, st);
+  if (e != cudaSuccess) return H2O_ERR_CUDA;
+  c->launches += 1;
+  e = launch_attn_colsum_bf16(g.head_dim, m, p, st);
+  if (e != cudaSuccess) return H2O_ERR_CUDA;
+  c->launches += 1;
+  return H2O_OK;
+}
+
+// K3 + K4 with summed weights `colsum` (row stride ld); advances n and t0.
+h2o_status run_evict(h2o_cache* c, const float* colsum, int ld, const void* kn, const void* vn,
+                     int nq, cudaStream_t st) {
+  const h2o_config& g = c->cfg;
+  EvictParams e;
+  e.B = g.batch;
+  e.Hkv = g.n_kv_heads;
+  e.C = g.capacity;
+  e.d = g.head_dim;
+  e.esize = static_cast<int>(esize_of(g.dtype));
+  e.n = c->n;
+  e.t0 = c->t0;
+  e.nq = nq;
+  e.W = g.recent_window;
+  e.colsum = colsum;
+  e.colsum_ld = ld;
+  e.scores = c->buf.scores;
+  e.pos = c->buf.pos;
+  e.plan_slots = c->plan_slots;
+  e.plan_tokens = c->plan_tokens;
+  e.plan_count = c->plan_count;
+  e.plan_ld = g.max_chunk;
+  e.k_new = kn;
+  e.v_new = vn;
+  e.k_cache = c->buf.k;
+  e.v_cache = c->buf.v;
+  e.state = c->buf.state;
+  cudaError_t err = launch_evict(e, g.max_chunk, st);
+  if (err != cudaSuccess) return H2O_ERR_CUDA;
+  c->launches += 2;
+  c->n = c->n + nq < g.capacity ? c->n + nq : g.capacity;
+  c->t0 += nq;
+  return H2O_OK;
+}
+
+h2o_status copy_colsum(h2o_cache* c, float* dst, int nq, cudaStream_t st) {
+  const size_t w = (static_cast<size_t>(c->cfg.capacity) + nq) * sizeof(float);
+  return cuda_status(cudaMemcpy2DAsync(dst, w, c->colsum, c->colsum_ld * sizeof(float), w,
+                                       static_cast<size_t>(c->cfg.batch) * c->cfg.n_kv_heads,
+                                       cudaMemcpyDefault, st));
+}
+
+}  // namespace
+
+namespace h2o {
+bool smem_attr_done(const void* fn, int* slot_bits) {
+  (void)fn;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const int w = dev / 32, bit = 1 << (dev % 32);
+  if (slot_bits[w] & bit) return true;
+  slot_bits[w] |= bit;
+  return false;
+}
+}  // namespace h2o
+
+extern "C" {
+
+h2o_status h2o_required_bytes(const h2o_config* cfg, h2o_sizes* out) {
+  h2o_status s = check_config(cfg);
+  if (s != H2O_OK) return s;
+  if (!out) return H2O_ERR_INVALID_ARG;
+  const size_t slots = static_cast<size_t>(cfg->batch) * cfg->n_kv_heads * cfg->capacity;
+  out->k_bytes = slots * cfg->head_dim * esize_of(cfg->dtype);
+  out->v_bytes = out->k_bytes;
+  out->scores_bytes = slots * 4;
+  out->pos_bytes = slots * 4;
+  out->state_bytes = 4 * sizeof(int32_t);
+  out->workspace_bytes = workspace_layout(*cfg).total;
+  return H2O_OK;
+}
+
+h2o_status h2o_cache_create(const h2o_config* cfg, const h2o_buffers* bufs, void* stream,
+                            h2o_cache** out) {
+  h2o_status s = check_config(cfg);
+  if (s != H2O_OK) return s;
+  if (!bufs || !out) return H2O_ERR_INVALID_ARG;
+  if (!bufs->k || !bufs->v || !bufs->scores || !bufs->pos || !bufs->state || !bufs->workspace)
+    return H2O_ERR_INVALID_ARG;
+  if (!aligned(bufs->k, 16) || !aligned(bufs->v, 16) || !aligned(bufs->scores, 16) ||
+      !aligned(bufs->pos, 16) || !aligned(bufs->state, 16) || !aligned(bufs->workspace, 256))
+    return H2O_ERR_ALIGN;
+  const Layout L = workspace_layout(*cfg);
+  if (bufs->workspace_bytes < L.total) return H2O_ERR_SHAPE;
+  if (cfg->dtype == H2O_BF16 && !encode_fn()) return H2O_ERR_CUDA;
+  h2o_cache* c = new (std::nothrow) h2o_cache();
+  if (!c) return H2O_ERR_INVALID_ARG;
+  c->cfg = *cfg;
+  c->buf = *bufs;
+  uint8_t* ws = static_cast<uint8_t*>(bufs->workspace);
+  c->nq_pad = L.nq_pad;
+  c->colsum_ld = L.colsum_ld;
+  c->lse2 = reinterpret_cast<float*>(ws + L.lse);
+  c->colsum = reinterpret_cast<float*>(ws + L.colsum);
+  c->plan_slots = reinterpret_cast<int*>(ws + L.slots);
+  c->plan_tokens = reinterpret_cast<int*>(ws + L.tokens);
+  c->plan_count = reinterpret_cast<int*>(ws + L.count);
+  c->stage_q = ws + L.sq;
+  c->stage_kn = ws + L.skn;
+  c->stage_vn = ws + L.svn;
+  c->stage_out = ws + L.sout;
+  h2o_sizes sz;
+  h2o_required_bytes(cfg, &sz);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(bufs->k, 0, sz.k_bytes, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(bufs->v, 0, sz.v_bytes, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(bufs->scores, 0, sz.scores_bytes, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(bufs->pos, 0xFF, sz.pos_bytes, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(bufs->state, 0, sz.state_bytes, st);
+  if (e != cudaSuccess) {
+    delete c;
+    return H2O_ERR_CUDA;
+  }
+  *out = c;
+  return H2O_OK;
+}
+
+h2o_status h2o_attention(h2o_cache* c, const void* q, const void* k_new, const void* v_new,
+                         int32_t n_q, void* out, float* colsum_out, void* stream) {
+  h2o_status s = check_step_args(c, q, k_new, v_new, n_q, out);
+  if (s != H2O_OK || n_q == 0) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = run_attention(c, q, k_new, v_new, n_q, out, st);
+  if (s == H2O_OK && colsum_out) s = copy_colsum(c, colsum_out, n_q, st);
+  return s;
+}
+
+h2o_status h2o_evict(h2o_cache* c, const float* colsum, const void* k_new, const void* v_new,
+                     int32_t n_q, void* stream) {
+  if (!c || n_q < 0 || n_q > c->cfg.max_chunk) return H2O_ERR_INVALID_ARG;
+  if (n_q == 0) return H2O_OK;
+  if (!colsum || !k_new || !v_new) return H2O_ERR_INVALID_ARG;
+  if (!aligned(colsum, 4) || !aligned(k_new, 16) || !aligned(v_new, 16)) return H2O_ERR_ALIGN;
+  return run_evict(c, colsum, c->cfg.capacity + n_q, k_new, v_new, n_q,
+                   static_cast<cudaStream_t>(stream));
+}
+
+h2o_status h2o_chunk_step(h2o_cache* c, const void* q, const void* k_new, const void* v_new,
+                          int32_t n_q, void* out, float* colsum_out, void* stream) {
+  h2o_status s = check_step_args(c, q, k_new, v_new, n_q, out);
+  if (s != H2O_OK || n_q == 0) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = run_attention(c, q, k_new, v_new, n_q, out, st);
+  if (s == H2O_OK && colsum_out) s = copy_colsum(c, colsum_out, n_q, st);
+  if (s == H2O_OK) s = run_evict(c, c->colsum, c->colsum_ld, k_new, v_new, n_q, st);
+  return s;
+}
+
+h2o_status h2o_chunk_step_host(h2o_cache* c, const void* q_host, const void* k_new_host,
+                               const void* v_new_host, int32_t n_q, void* out_host,
+                               float* colsum_out_host, void* stream) {
+  if (!c) return H2O_ERR_INVALID_ARG;
+  if (n_q < 0 || n_q > c->cfg.max_chunk) return H2O_ERR_INVALID_ARG;
+  if (n_q == 0) return H2O_OK;
+  if (!q_host || !k_new_host || !v_new_host || !out_host) return H2O_ERR_INVALID_ARG;
+  const h2o_config& g = c->cfg;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t rows = static_cast<size_t>(g.batch) * n_q * g.head_dim * esize_of(g.dtype);
+  const size_t bq = rows * g.n_q_heads, bkv = rows * g.n_kv_heads;
+  cudaError_t e = cudaMemcpyAsync(c->stage_q, q_host, bq, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->stage_kn, k_new_host, bkv, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->stage_vn, v_new_host, bkv, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return H2O_ERR_CUDA;
+  h2o_status s = h2o_chunk_step(c, c->stage_q, c->stage_kn, c->stage_vn, n_q, c->stage_out,
+                                colsum_out_host, stream);
+  if (s != H2O_OK) return s;
+  return cuda_status(cudaMemcpyAsync(out_host, c->stage_out, bq, cudaMemcpyDeviceToHost, st));
+}
+
+h2o_status h2o_cache_read(const h2o_cache* c, void* k, void* v, float* scores, int32_t* pos,
+                          int32_t* n_t0, void* stream) {
+  if (!c) return H2O_ERR_INVALID_ARG;
+  h2o_sizes sz;
+  h2o_required_bytes(&c->cfg, &sz);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (k) e = cudaMemcpyAsync(k, c->buf.k, sz.k_bytes, cudaMemcpyDefault, st);
+  if (e == cudaSuccess && v) e = cudaMemcpyAsync(v, c->buf.v, sz.v_bytes, cudaMemcpyDefault, st);
+  if (e == cudaSuccess && scores)
+    e = cudaMemcpyAsync(scores, c->buf.scores, sz.scores_bytes, cudaMemcpyDefault, st);
+  if (e == cudaSuccess && pos)
+    e = cudaMemcpyAsync(pos, c->buf.pos, sz.pos_bytes, cudaMemcpyDefault, st);
+  if (n_t0) {
+    n_t0[0] = c->n;
+    n_t0[1] = c->t0;
+  }
+  return cuda_status(e);
+}
+
+h2o_status h2o_cache_write(h2o_cache* c, const void* k, const void* v, const float* scores,
+                           const int32_t* pos, const int32_t* n_t0, void* stream) {
+  if (!c || !k || !v || !scores || !pos || !n_t0) return H2O_ERR_INVALID_ARG;
+  if (n_t0[0] < 0 || n_t0[0] > c->cfg.capacity || n_t0[1] < n_t0[0]) return H2O_ERR_INVALID_ARG;
+  h2o_sizes sz;
+  h2o_required_bytes(&c->cfg, &sz);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(c->buf.k, k, sz.k_bytes, cudaMemcpyDefault, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->buf.v, v, sz.v_bytes, cudaMemcpyDefault, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->buf.scores, scores, sz.scores_bytes, cudaMemcpyDefault, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->buf.pos, pos, sz.pos_bytes, cudaMemcpyDefault, st);
+  static int32_t fresh[4];
+  fresh[0] = n_t0[0];
+  fresh[1] = n_t0[1];
+  fresh[2] = 0;
+  fresh[3] = 0;
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->buf.state, fresh, sizeof(fresh), cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return H2O_ERR_CUDA;
+  c->n = n_t0[0];
+  c->t0 = n_t0[1];
+  return H2O_OK;
+}
+
+h2o_status h2o_cache_check(h2o_cache* c, void* stream) {
+  if (!c) return H2O_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return H2O_ERR_CUDA;
+  int32_t word = 0;
+  if (cudaMemcpy(&word, c->buf.state + 2, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return H2O_ERR_CUDA;
+  if (word & kDevErrTimeout) return H2O_ERR_TIMEOUT;
+  if (word & kDevErrPlan) return H2O_ERR_STATE;
+  return H2O_OK;
+}
+
+h2o_status h2o_cache_info(const h2o_cache* c, int32_t* n, int32_t* t0, uint64_t* launches) {
+  if (!c) return H2O_ERR_INVALID_ARG;
+  if (n) *n = c->n;
+  if (t0) *t0 = c->t0;
+  if (launches) *launches = c->launches;
+  return H2O_OK;
+}
+
+void h2o_cache_destroy(h2o_cache* c) { delete c; }
+
+const char* h2o_status_string(h2o_status s) {
+  switch (s) {
+    case H2O_OK: return "ok";
+    case H2O_ERR_INVALID_ARG: return "invalid argument";
+    case H2O_ERR_SHAPE: return "unsupported shape or buffer too small";
+    case H2O_ERR_DTYPE: return "unsupported dtype";
+    case H2O_ERR_ALIGN: return "misaligned pointer";
+    case H2O_ERR_CUDA: return "CUDA runtime error";
+    case H2O_ERR_TIMEOUT: return "device wait timed out";
+    case H2O_ERR_STATE: return "inconsistent eviction plan";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,74 @@
+"""Score update, selection, placement and scatter of the CUDA path
+(h2o_evict) fed the oracle's fp32 summed weights: always bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import gpu_helpers as gh
+from kv_cache_sparse_b200 import binding
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built(cuda_ok):
+    gh.ensure_built()
+
+
+CASES = [
+    # B, Hkv, d, C, n, nq, W, levels, dtype       what it covers
+    (1, 2, 128, 64, 64, 16, 0, None, torch.bfloat16),    # full cache, no window
+    (1, 2, 128, 64, 64, 16, 16, None, torch.bfloat16),   # window = chunk
+    (1, 2, 128, 64, 64, 16, 40, None, torch.bfloat16),   # window wider than the chunk
+    (2, 3, 64, 100, 80, 64, 8, None, torch.bfloat16),    # partially full: n < C < n + nq
+    (1, 2, 128, 256, 100, 64, 8, None, torch.bfloat16),  # fill phase: no eviction
+    (1, 4, 128, 512, 512, 128, 0, 4, torch.bfloat16),    # heavy ties (4 score levels)
+    (1, 4, 128, 512, 512, 128, 32, 1, torch.bfloat16),   # all scores equal
+    (1, 1, 128, 2048, 2048, 1, 0, None, torch.bfloat16),  # single new token
+    (1, 8, 128, 8192, 8192, 1024, 256, None, torch.bfloat16),  # full-size shape
+    (1, 2, 64, 256, 256, 64, 0, None, torch.float32),    # fp32 cache
+    (4, 2, 64, 33, 20, 20, 5, 3, torch.float32),         # tiny, odd sizes
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B{}_Hkv{}_d{}_C{}_n{}_nq{}_W{}_lv{}".format(*c[:8]))
+def test_evict_fed_oracle_weights_is_bit_exact(case):
+    B, Hkv, d, C, n, nq, W, levels, dt = case
+    rng = np.random.default_rng(C + n + nq + W)
+    shape = gh.shape_of(B, Hkv, Hkv, d, C, nq, W, dt)
+    gpu = binding.H2OCache(shape)
+    ref = gh.oracle_for(shape)
+    t0 = n + 3
+    K, V, sc, pos = gh.random_state(shape, n, t0, rng, score_levels=levels)
+    gh.install_state(gpu, ref, K, V, sc, pos, n, t0)
+    if levels:
+        cs = (rng.integers(0, levels, (B, Hkv, C + nq)) / levels).astype(np.float32)
+    else:
+        cs = (rng.random((B, Hkv, C + nq)) * 2).astype(np.float32)
+    cs[:, :, n:C] = 0
+    kn = torch.randn(B, nq, Hkv, d).to(dt)
+    vn = torch.randn(B, nq, Hkv, d).to(dt)
+    gpu.evict(torch.from_numpy(cs).cuda(), kn.cuda(), vn.cuda())
+    assert gpu.check() == 0
+    ref.evict(cs, gh.np64(kn), gh.np64(vn))
+    gh.assert_state_equal(gpu.read(), ref, dt, str(case))
+
+
+def test_evict_many_steps_bit_exact():
+    """A run of evictions on one cache (each fed the same weights on both
+    sides) stays bit-identical, through the fill phase into eviction."""
+    B, Hkv, d, C, nq, W = 2, 2, 128, 96, 40, 10
+    shape = gh.shape_of(B, Hkv, Hkv, d, C, nq, W)
+    gpu = binding.H2OCache(shape)
+    ref = gh.oracle_for(shape)
+    rng = np.random.default_rng(9)
+    for step in range(8):
+        m = int(rng.integers(1, nq + 1))
+        cs = (rng.random((B, Hkv, C + m)) * 3).astype(np.float32)
+        cs[:, :, ref.n:C] = 0
+        kn = torch.randn(B, m, Hkv, d).to(torch.bfloat16)
+        vn = torch.randn(B, m, Hkv, d).to(torch.bfloat16)
+        gpu.evict(torch.from_numpy(cs).cuda(), kn.cuda(), vn.cuda())
+        ref.evict(cs, gh.np64(kn), gh.np64(vn))
+        gh.assert_state_equal(gpu.read(), ref, torch.bfloat16, f"step {step}")
+    assert gpu.check() == 0
