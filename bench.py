@@ -1,0 +1,438 @@
+"""Benchmark of the chunked H2O attention step on B200.
+
+A step is one pass of the whole hot path -- attention forward, summed
+weights, score update + top-C selection, K/V scatter -- over one chunk of
+synthetic input, on a full cache (steady state).  The workload is the
+Qwen3-4B-shaped single cache (H_q 32, H_kv 8, d 128, bf16, C 8192,
+n_q 1024, W 256).  Inputs are drawn on the device before the timed region;
+L2 is flushed (256 MiB write) before every timed step, outside its events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  With N > 1 (launched by torchrun) every
+rank runs its own independent cache (weak scaling, no collective on the
+data path); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from kv_cache_sparse_b200.workloads import QWEN_C8K, device_chunk  # noqa: E402
+
+WL = QWEN_C8K
+METRIC = "chunk-tokens/s per H2O attention+evict step (1 B200); % bf16 TC peak; evict GB/s"
+UNIT = "chunk-tokens/s"
+KERNELS = ["attn_fwd_kernel", "attn_colsum_kernel", "h2o_select", "h2o_scatter"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attention_flops(wl, n, nq):
+    """Algorithmic FLOPs of one step's attention: QK^T and PV over the
+    visible (query, key) pairs, 2*d each, for every query head and cache."""
+    pairs = nq * n + nq * (nq + 1) // 2
+    return 4.0 * wl.head_dim * wl.n_q_heads * wl.batch * pairs
+
+
+def evict_bytes(wl, n, nq, kept_total):
+    """Algorithmic bytes of the score update + selection + scatter: read the
+    scores and summed weights, write the scores; per kept new token write its
+    position and score and read + write its K and V rows."""
+    units = wl.batch * wl.n_kv_heads
+    e = 2 if wl.dtype == "bf16" else 4
+    per_unit = 4 * n + 4 * (n + nq) + 4 * n
+    return units * per_unit + kept_total * (8 + 4 * wl.head_dim * e)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.idx), "-lms", "200"], stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), max=float(parts[2]),
+                                     power=float(parts[3]) if parts[3] not in ("[N/A]", "") else None,
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] is None or r["power"] > 200.0] or rows
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((i.get("num_threads") or 0) for i in info) if info else None
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+
+def oracle_sample(wl, steps: int, seed: int = 0, groups=None):
+    """Times `steps` steady-state oracle steps (attention + eviction) on the
+    host cores, from a full random cache.  `groups` restricts the cache to
+    that many of its (independent) KV heads with their query heads; the
+    token count is credited in proportion.  Returns (seconds, tokens)."""
+    from oracle import h2o_oracle as orc   # test infrastructure: CPU baseline only
+    full = wl.n_kv_heads
+    groups = full if groups is None else groups
+    wl = wl.scaled(n_kv_heads=groups, n_q_heads=groups * wl.group)
+    rng = np.random.default_rng(seed)
+    ref = orc.OracleCache(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.capacity,
+                          wl.window)
+    C = wl.capacity
+    g = torch.Generator().manual_seed(seed)
+    K = torch.randn(wl.batch, wl.n_kv_heads, C, wl.head_dim, generator=g).to(torch.bfloat16)
+    V = torch.randn(wl.batch, wl.n_kv_heads, C, wl.head_dim, generator=g).to(torch.bfloat16)
+    pos = np.tile(rng.permutation(4 * C)[:C].astype(np.int32), (wl.batch, wl.n_kv_heads, 1))
+    ref.load(K.double().numpy(), V.double().numpy(),
+             (rng.random((wl.batch, wl.n_kv_heads, C)) * 8).astype(np.float32), pos, C, 4 * C)
+    chunks = []
+    for c in range(steps):
+        gc = torch.Generator().manual_seed(seed + 1 + c)
+        sh_q = (wl.batch, wl.chunk, wl.n_q_heads, wl.head_dim)
+        sh_kv = (wl.batch, wl.chunk, wl.n_kv_heads, wl.head_dim)
+        chunks.append(tuple(torch.randn(s, generator=gc).to(torch.bfloat16).double().numpy()
+                            for s in (sh_q, sh_kv, sh_kv)))
+    t = time.perf_counter()
+    for q, kn, vn in chunks:
+        ref.step(q, kn, vn)
+    dt = time.perf_counter() - t
+    return dt, steps * wl.batch * wl.chunk * groups / full
+
+
+def cpu_baseline(wl, steps: int = 2):
+    dt, tokens = oracle_sample(wl, steps)
+    return {"value": tokens / dt, "unit": UNIT, "cores": cpu_cores(), "blas_threads": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{steps} steady-state steps of the full workload (1 cache, C={wl.capacity}, "
+                      f"n_q={wl.chunk}) in numpy fp64, from a full random cache: {dt:.2f} s"}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=120),
+            device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, world, rank, local):
+    from kv_cache_sparse_b200 import binding
+    from kv_cache_sparse_b200.build import build
+    if rank == 0 or world == 1:
+        build()
+    barrier(world)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = WL
+    shape = binding.CacheShape(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
+                               wl.capacity, wl.chunk, wl.window, wl.torch_dtype())
+    cache = binding.H2OCache(shape, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    seed = 1000 * rank
+    # fill phase (untimed): C / n_q steps bring the cache to steady state
+    fill = wl.capacity // wl.chunk
+    for c in range(fill):
+        cache.step(*device_chunk(wl, seed, c, dev))
+    K, W = args.steps, args.warmup
+    chunks = [device_chunk(wl, seed, fill + c, dev) for c in range(W + K)]
+    out = torch.empty(wl.batch, wl.chunk, wl.n_q_heads, wl.head_dim, dtype=wl.torch_dtype(),
+                      device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for c in range(W):
+        cache.step(*chunks[c], out=out)
+    torch.cuda.synchronize(dev)
+    if cache.check() != 0:
+        raise SystemExit("device error during warm-up")
+    cache.set_timing(True)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    kern = np.zeros((K, 4))
+    kept = []
+    launches0 = cache.info()["kernel_launches"]
+    with ClockSampler(local) as clocks:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        for k in range(K):
+            flush.zero_()                       # L2 flush, outside the step's events
+            t0 = cache.info()["t0"]
+            starts[k].record(stream)
+            cache.step(*chunks[W + k], out=out)
+            ends[k].record(stream)
+            kern[k] = cache.kernel_ms()          # waits for this step's last event
+            kept.append(int((cache.pos >= t0).sum().item()))
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    launches = cache.info()["kernel_launches"] - launches0
+    if cache.check() != 0:
+        raise SystemExit("device error during the timed steps")
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    tokens = sum_over_ranks(K * wl.batch * wl.chunk, world)
+    value = tokens / (total_ms / 1e3)
+
+    # ---- e2e: the same step through the host-buffer entry point (pinned memory)
+    hq = [tuple(t.cpu().pin_memory() for t in chunks[W + k]) for k in range(min(K, 8))]
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_s = [torch.cuda.Event(enable_timing=True) for _ in hq]
+    e2e_e = [torch.cuda.Event(enable_timing=True) for _ in hq]
+    cache.set_timing(False)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for k, (q, kn, vn) in enumerate(hq):
+        flush.zero_()
+        e2e_s[k].record(stream)
+        cache.step_host(q, kn, vn, hout)
+        e2e_e[k].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e)), world)
+    e2e_tokens = sum_over_ranks(len(hq) * wl.batch * wl.chunk, world)
+    h2d = sum(t.numel() * t.element_size() for t in hq[0])
+    d2h = hout.numel() * hout.element_size()
+
+    # ---- roofline of the dominant kernel
+    peaks, peaks_kind = load_peaks()
+    avg = kern.mean(axis=0)
+    n = wl.capacity
+    flops = attention_flops(wl, n, wl.chunk)
+    ebytes = evict_bytes(wl, n, wl.chunk, float(np.mean(kept)))
+    tc_peak = peaks["bf16_tflops"]
+    hbm_peak = peaks["hbm_gbs"]
+    kernels = {}
+    for i, name in enumerate(KERNELS):
+        kernels[name] = {"ms": round(float(avg[i]), 5),
+                         "share": round(float(avg[i] / max(avg.sum(), 1e-12)), 4)}
+    dom = int(np.argmax(avg))
+    if dom == 0:
+        achieved = flops / (avg[0] * 1e-3) / 1e12
+        roof = {"kernel": KERNELS[0], "bound": "tensor", "achieved": round(achieved, 2),
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
+                "traffic": None, "peak_kind": f"{peaks_kind} bf16 dense (burst)",
+                "per_launch": f"{flops:.4e} FLOP (QK^T + PV over visible pairs)"}
+    else:
+        # the summed-weights kernel: its FLOPs are the QK^T recompute
+        rf = flops / 2
+        achieved = rf / (avg[dom] * 1e-3) / 1e12
+        roof = {"kernel": KERNELS[dom], "bound": "tensor", "achieved": round(achieved, 2),
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
+                "traffic": None, "peak_kind": f"{peaks_kind} bf16 dense (burst)",
+                "per_launch": f"{rf:.4e} FLOP (QK^T recompute)"}
+    attn_ms = avg[0] + avg[1]
+    evict_ms = avg[2] + avg[3]
+    extra = {
+        "attention_tc_frac": round(flops / (attn_ms * 1e-3) / 1e12 / tc_peak, 4),
+        "attention_tflops": round(flops / (attn_ms * 1e-3) / 1e12, 2),
+        "evict_gbs": round(ebytes / (evict_ms * 1e-3) / 1e9, 1),
+        "evict_hbm_frac": round(ebytes / (evict_ms * 1e-3) / 1e9 / hbm_peak, 4),
+        "evict_bytes_per_step": int(ebytes),
+        "kept_new_tokens_per_step": float(np.mean(kept)),
+        "kernels": kernels,
+        "step_ms_p50": round(float(np.median(step_ms)), 5),
+    }
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(total_ms / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/K/V with 2% heavy-hitter keys, drawn on device)",
+        "config": {"workload": wl.name, "caches_per_gpu": wl.batch, "n_q_heads": wl.n_q_heads,
+                   "n_kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "chunk": wl.chunk,
+                   "capacity": wl.capacity, "recent_window": wl.window,
+                   "state": "steady (cache full)", "parallelism": f"independent caches x{world}",
+                   "l2": "flushed before every timed step (256 MiB write, outside the events)"},
+        "roofline": roof,
+        "e2e": {"value": round(e2e_tokens / (e2e_ms / 1e3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "path": "h2o_chunk_step_host, pinned host buffers"},
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+    }
+    line.update(extra)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_steps)
+    return line
+
+
+def run_reference(args, world, rank):
+    """The oracle on the host cores, same workload and metric.  Each step is a
+    bounded sample: the full step restricted to as many of the cache's
+    independent KV groups as fit a ~120 s budget for the whole run."""
+    if rank != 0:
+        return None
+    wl = WL
+    t1, _ = oracle_sample(wl, 1, seed=100, groups=1)       # one group, to size the sample
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    groups = int(max(1, min(wl.n_kv_heads, budget // max(t1, 1e-3))))
+    for k in range(max(0, args.warmup - 1)):
+        oracle_sample(wl, 1, seed=200 + k, groups=groups)
+    total, tokens = 0.0, 0.0
+    for k in range(args.steps):
+        dt, tok = oracle_sample(wl, 1, seed=k, groups=groups)
+        total += dt
+        tokens += tok
+    value = tokens / total
+    sample = (f"each step: one steady-state step of the workload restricted to {groups} of its "
+              f"{wl.n_kv_heads} independent KV groups (with their {wl.group} query heads each), "
+              f"numpy fp64 from a full random cache; tokens credited x{groups}/{wl.n_kv_heads}")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "caches_per_gpu": wl.batch, "chunk": wl.chunk,
+                   "capacity": wl.capacity, "recent_window": wl.window,
+                   "state": "steady (cache full)"},
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": cpu_cores(),
+                         "blas_threads": blas_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        line = run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        line = run_ours(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -180,6 +180,16 @@ H2O_API h2o_status h2o_cache_check(h2o_cache* c, void* stream);
 H2O_API h2o_status h2o_cache_info(const h2o_cache* c, int32_t* n, int32_t* t0,
                           uint64_t* kernel_launches);
 
+/* Per-kernel timing.  While enabled, every step records a CUDA event on its
+ * stream before its first kernel and after each kernel.  h2o_cache_kernel_ms
+ * waits for the last recorded event and writes the device durations (ms) of
+ * the last step's kernels: [0] attention forward, [1] summed weights,
+ * [2] score update + selection, [3] K/V scatter (a kernel that did not run
+ * reads 0).  Disabled by default; enabling creates the events on the
+ * current device. */
+H2O_API h2o_status h2o_cache_set_timing(h2o_cache* c, int enable);
+H2O_API h2o_status h2o_cache_kernel_ms(h2o_cache* c, float* ms4);
+
 /* Frees the host handle only. */
 H2O_API void h2o_cache_destroy(h2o_cache* c);
 

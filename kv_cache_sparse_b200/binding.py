@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "H2O_OK", 1: "H2O_ERR_INVALID_ARG", 2: "H2O_ERR_SHAPE", 3: "H
 
 EXPORTED = ["h2o_required_bytes", "h2o_cache_create", "h2o_chunk_step", "h2o_chunk_step_host",
             "h2o_attention", "h2o_evict", "h2o_cache_read", "h2o_cache_write",
-            "h2o_cache_check", "h2o_cache_info", "h2o_cache_destroy", "h2o_status_string"]
+            "h2o_cache_check", "h2o_cache_info", "h2o_cache_set_timing", "h2o_cache_kernel_ms",
+            "h2o_cache_destroy", "h2o_status_string"]
 
 
 class H2OError(RuntimeError):
@@ -68,6 +69,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.h2o_cache_check.argtypes = [P, P]
     lib.h2o_cache_info.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I),
                                    ctypes.POINTER(ctypes.c_uint64)]
+    lib.h2o_cache_set_timing.argtypes = [P, V]
+    lib.h2o_cache_kernel_ms.argtypes = [P, ctypes.POINTER(ctypes.c_float)]
     lib.h2o_cache_destroy.argtypes = [P]
     lib.h2o_cache_destroy.restype = None
     lib.h2o_status_string.argtypes = [V]
@@ -247,6 +250,16 @@ class H2OCache:
     def check(self, stream=None) -> int:
         """Synchronises and returns the device status (0 = ok)."""
         return lib().h2o_cache_check(self._h, _stream(stream))
+
+    def set_timing(self, enable: bool = True):
+        _check("h2o_cache_set_timing", lib().h2o_cache_set_timing(self._h, int(enable)))
+
+    def kernel_ms(self):
+        """Durations (ms) of the last step's kernels: attention forward,
+        summed weights, selection, scatter."""
+        ms = (ctypes.c_float * 4)()
+        _check("h2o_cache_kernel_ms", lib().h2o_cache_kernel_ms(self._h, ms))
+        return list(ms)
 
     def info(self):
         n, t0, launches = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_uint64()

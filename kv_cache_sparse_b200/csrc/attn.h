@@ -32,6 +32,8 @@ cudaError_t launch_attn_f32(int head_dim, const float* q, const float* kc, const
                             cudaStream_t st);
 
 // K3 + K4: score update, selection, placement and K/V scatter.
-cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st);
+// `between` (may be null) is recorded on the stream between K3 and K4.
+cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st,
+                         cudaEvent_t between);
 
 }  // namespace h2o

@@ -243,7 +243,8 @@ __global__ void __launch_bounds__(256) h2o_scatter(const EvictParams e) {
   }
 }
 
-cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st) {
+cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st,
+                         cudaEvent_t between) {
   const size_t smem = static_cast<size_t>(e.n + e.nq) * sizeof(uint32_t);
   static int attr_bits[2] = {0, 0};
   if (!smem_attr_done(reinterpret_cast<const void*>(h2o_select), attr_bits)) {
@@ -255,6 +256,7 @@ cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st) {
   h2o_select<<<units, kSelThreads, smem, st>>>(e);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
+  if (between) cudaEventRecord(between, st);
   const int vpr = e.d * e.esize / 16;
   const int work = 2 * e.nq * vpr;
   int gy = cdiv(work, 256);

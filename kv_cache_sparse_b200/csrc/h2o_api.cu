@@ -37,6 +37,10 @@ struct h2o_cache {
   uint8_t* stage_kn = nullptr;
   uint8_t* stage_vn = nullptr;
   uint8_t* stage_out = nullptr;
+  // per-kernel timing (h2o_cache_set_timing)
+  bool timing = false;
+  cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+  bool ev_used[5] = {false, false, false, false, false};
 };
 
 namespace {
@@ -144,6 +148,12 @@ bool encode_cache(CUtensorMap* tm, const void* base, int BH, int n, int C, int d
 
 h2o_status cuda_status(cudaError_t e) { return e == cudaSuccess ? H2O_OK : H2O_ERR_CUDA; }
 
+// Records timing event i (0: before K1, i: after kernel i) when timing is on.
+void mark(h2o_cache* c, int i, cudaStream_t st) {
+  if (!c->timing) return;
+  if (cudaEventRecord(c->ev[i], st) == cudaSuccess) c->ev_used[i] = true;
+}
+
 h2o_status check_step_args(h2o_cache* c, const void* q, const void* kn, const void* vn, int nq,
                            const void* out) {
   if (!c) return H2O_ERR_INVALID_ARG;
@@ -181,6 +191,8 @@ h2o_status run_attention(h2o_cache* c, const void* q, const void* kn, const void
                          void* out, cudaStream_t st) {
   const h2o_config& g = c->cfg;
   AttnParams p = attn_params(c, nq, out);
+  for (int i = 0; i < 5; ++i) c->ev_used[i] = false;
+  mark(c, 0, st);
   if (g.dtype == H2O_F32) {
     cudaError_t e = launch_attn_f32(g.head_dim, static_cast<const float*>(q),
                                     static_cast<const float*>(c->buf.k),
@@ -188,6 +200,7 @@ h2o_status run_attention(h2o_cache* c, const void* q, const void* kn, const void
                                     static_cast<const float*>(kn), static_cast<const float*>(vn),
                                     p, st);
     c->launches += (c->n < g.capacity) ? 3 : 2;
+    mark(c, 2, st);
     return cuda_status(e);
   }
   AttnMaps m;
@@ -201,9 +214,11 @@ h2o_status run_attention(h2o_cache* c, const void* q, const void* kn, const void
   cudaError_t e = launch_attn_fwd_bf16(g.head_dim, m, p, st);
   if (e != cudaSuccess) return H2O_ERR_CUDA;
   c->launches += 1;
+  mark(c, 1, st);
   e = launch_attn_colsum_bf16(g.head_dim, m, p, st);
   if (e != cudaSuccess) return H2O_ERR_CUDA;
   c->launches += 1;
+  mark(c, 2, st);
   return H2O_OK;
 }
 
@@ -234,9 +249,15 @@ h2o_status run_evict(h2o_cache* c, const float* colsum, int ld, const void* kn, 
   e.k_cache = c->buf.k;
   e.v_cache = c->buf.v;
   e.state = c->buf.state;
-  cudaError_t err = launch_evict(e, g.max_chunk, st);
+  if (!c->ev_used[2]) {  // eviction on its own: time it from here
+    for (int i = 0; i < 5; ++i) c->ev_used[i] = false;
+    mark(c, 2, st);
+  }
+  cudaError_t err = launch_evict(e, g.max_chunk, st, c->timing ? c->ev[3] : nullptr);
   if (err != cudaSuccess) return H2O_ERR_CUDA;
+  if (c->timing) c->ev_used[3] = true;
   c->launches += 2;
+  mark(c, 4, st);
   c->n = c->n + nq < g.capacity ? c->n + nq : g.capacity;
   c->t0 += nq;
   return H2O_OK;
@@ -442,7 +463,41 @@ h2o_status h2o_cache_info(const h2o_cache* c, int32_t* n, int32_t* t0, uint64_t*
   return H2O_OK;
 }
 
-void h2o_cache_destroy(h2o_cache* c) { delete c; }
+h2o_status h2o_cache_set_timing(h2o_cache* c, int enable) {
+  if (!c) return H2O_ERR_INVALID_ARG;
+  if (enable && !c->ev[0]) {
+    for (int i = 0; i < 5; ++i)
+      if (cudaEventCreate(&c->ev[i]) != cudaSuccess) return H2O_ERR_CUDA;
+  }
+  c->timing = enable != 0;
+  for (int i = 0; i < 5; ++i) c->ev_used[i] = false;
+  return H2O_OK;
+}
+
+h2o_status h2o_cache_kernel_ms(h2o_cache* c, float* ms4) {
+  if (!c || !ms4) return H2O_ERR_INVALID_ARG;
+  for (int i = 0; i < 4; ++i) ms4[i] = 0.f;
+  int last = -1;
+  for (int i = 4; i >= 0 && last < 0; --i)
+    if (c->ev_used[i]) last = i;
+  if (last < 0) return H2O_OK;
+  if (cudaEventSynchronize(c->ev[last]) != cudaSuccess) return H2O_ERR_CUDA;
+  for (int k = 0; k < 4; ++k) {
+    if (c->ev_used[k] && c->ev_used[k + 1]) {
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, c->ev[k], c->ev[k + 1]) != cudaSuccess) return H2O_ERR_CUDA;
+      ms4[k] = ms;
+    }
+  }
+  return H2O_OK;
+}
+
+void h2o_cache_destroy(h2o_cache* c) {
+  if (!c) return;
+  for (int i = 0; i < 5; ++i)
+    if (c->ev[i]) cudaEventDestroy(c->ev[i]);
+  delete c;
+}
 
 const char* h2o_status_string(h2o_status s) {
   switch (s) {
