@@ -190,6 +190,31 @@ H2O_API h2o_status h2o_cache_info(const h2o_cache* c, int32_t* n, int32_t* t0,
 H2O_API h2o_status h2o_cache_set_timing(h2o_cache* c, int enable);
 H2O_API h2o_status h2o_cache_kernel_ms(h2o_cache* c, float* ms4);
 
+/* Attention with summed weights (steps 1-2 of the step) that allocates
+ * nothing and needs no handle or workspace.  The paper has no counterpart:
+ * this entry point exists for callers that cannot allocate device memory --
+ * engines or plugin hosts that own the whole memory budget and pass a
+ * plugin only its inputs and outputs, and serving loops that must not
+ * allocate once running.  The row statistics the two kernels share live in
+ * a static device array of the library (16 MiB per GPU that loads it, held
+ * until the process exits), so
+ *   batch * n_q_heads * (n_q rounded up to a multiple of 128) <= 4194304
+ * or the call returns H2O_ERR_SHAPE before launching anything.
+ * Inputs: cfg (capacity, heads, head_dim, dtype, scale; max_chunk bounds
+ * n_q; recent_window unused), k_cache / v_cache (device, cache layout) with
+ * n valid slots, q, k_new, v_new (device, chunk layouts).  Outputs (device):
+ * out, and colsum_out in the colsum layout for this n_q (required).
+ * The first call on a device looks up the array's device address on the
+ * current device (cudaGetSymbolAddress); make that first call before any
+ * stream capture.  All calls on a device share the array and it keeps the
+ * last call's contents (nothing in it needs clearing between calls), so
+ * calls that overlap on the GPU race on it: serialise them. */
+H2O_API h2o_status h2o_attention_static_scratch(const h2o_config* cfg, const void* k_cache,
+                                                const void* v_cache, int32_t n, const void* q,
+                                                const void* k_new, const void* v_new,
+                                                int32_t n_q, void* out, float* colsum_out,
+                                                void* stream);
+
 /* Frees the host handle only. */
 H2O_API void h2o_cache_destroy(h2o_cache* c);
 
