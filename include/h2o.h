@@ -80,7 +80,8 @@ typedef enum {
   H2O_ERR_ALIGN = 4,       /* pointer not 16-byte (workspace: 256-byte) aligned */
   H2O_ERR_CUDA = 5,        /* a CUDA runtime call failed                     */
   H2O_ERR_TIMEOUT = 6,     /* a kernel's bounded wait expired (device bit 1) */
-  H2O_ERR_STATE = 7        /* inconsistent eviction plan (device bit 2)      */
+  H2O_ERR_STATE = 7        /* inconsistent eviction plan (device bit 2) or a
+                              kernel's shared-memory layout check (bit 4)    */
 } h2o_status;
 
 typedef enum { H2O_BF16 = 0, H2O_F32 = 1 } h2o_dtype;
@@ -184,8 +185,8 @@ H2O_API h2o_status h2o_cache_info(const h2o_cache* c, int32_t* n, int32_t* t0,
  * stream before its first kernel and after each kernel.  h2o_cache_kernel_ms
  * waits for the last recorded event and writes the device durations (ms) of
  * the last step's kernels: [0] attention forward, [1] summed weights,
- * [2] score update + selection, [3] K/V scatter (a kernel that did not run
- * reads 0).  Disabled by default; enabling creates the events on the
+ * [2] score update + selection + K/V scatter (one kernel), [3] reserved,
+ * reads 0 (a kernel that did not run reads 0).  Disabled by default; enabling creates the events on the
  * current device. */
 H2O_API h2o_status h2o_cache_set_timing(h2o_cache* c, int enable);
 H2O_API h2o_status h2o_cache_kernel_ms(h2o_cache* c, float* ms4);
@@ -214,6 +215,12 @@ H2O_API h2o_status h2o_attention_static_scratch(const h2o_config* cfg, const voi
                                                 const void* k_new, const void* v_new,
                                                 int32_t n_q, void* out, float* colsum_out,
                                                 void* stream);
+
+/* Diagnostic: for x[i] <= 0 (device arrays of n floats) writes the
+ * polynomial base-2 exponential the kernels use for part of their
+ * probabilities (y_poly) and CUDA's exp2f (y_lib), for accuracy tests. */
+H2O_API h2o_status h2o_selftest_exp2(const float* x, float* y_poly, float* y_lib, int32_t n,
+                                     void* stream);
 
 /* Frees the host handle only. */
 H2O_API void h2o_cache_destroy(h2o_cache* c);

@@ -31,9 +31,7 @@ cudaError_t launch_attn_f32(int head_dim, const float* q, const float* kc, const
                             const float* kn, const float* vn, const AttnParams& p,
                             cudaStream_t st);
 
-// K3 + K4: score update, selection, placement and K/V scatter.
-// `between` (may be null) is recorded on the stream between K3 and K4.
-cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st,
-                         cudaEvent_t between);
+// K3 (with the K/V scatter fused): score update, selection, placement.
+cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st);
 
 }  // namespace h2o

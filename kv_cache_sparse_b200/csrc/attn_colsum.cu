@@ -25,13 +25,14 @@ template <int D>
 struct ColLayout {
   static constexpr int kRegions = D / 64;
   static constexpr int kTileBytes = 128 * D * 2;
-  static constexpr int kQStages = 2;
+  static constexpr int kQStages = 2;    // Q tiles, released when their MMA completes
+  static constexpr int kLseStages = 4;  // row statistics, released by the summing threads
   static constexpr int kKOff = 0;
   static constexpr int kQOff = kKOff + kTileBytes;
   static constexpr int kLseOff = kQOff + kQStages * kTileBytes;  // 512 bytes per stage
-  static constexpr int kBarOff = kLseOff + kQStages * 512;
-  // k_full, q_full[S], q_empty[S], s_full[2], s_empty[2], drain
-  static constexpr int kNumBars = 1 + 2 * kQStages + 4 + 1;
+  static constexpr int kBarOff = kLseOff + kLseStages * 512;
+  // k_full, q_full[QS], q_empty[QS], lse_full[LS], lse_empty[LS], s_full[2], s_empty[2], drain
+  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kLseStages + 4 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kRedOff = kMiscOff + 16;
   static constexpr int kBytes = kRedOff + 128 * 4;
@@ -40,13 +41,39 @@ struct ColLayout {
   static constexpr int kThreads = 320;
 };
 
+// Every kPolyEvery-th probability is computed with the FMA-pipe polynomial,
+// the rest with the MUFU ex2 instruction, so that both units share the work.
+constexpr int kPolyEvery = 4;
+
+template <bool kDiag>
+__device__ __forceinline__ void sum_tile(const uint32_t (&v0)[32], const uint32_t (&v1)[32],
+                                         const float4* lse4, float c, int first_col,
+                                         float (&part)[4]) {
+#pragma unroll
+  for (int q4 = 0; q4 < 16; ++q4) {
+    const float4 ls = lse4[q4];
+    const float l4[4] = {ls.x, ls.y, ls.z, ls.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int col = q4 * 4 + e;
+      const uint32_t sx = q4 < 8 ? v0[col] : v1[col - 32];
+      const float x = fmaf(__uint_as_float(sx), c, -l4[e]);
+      const float pr = (col % kPolyEvery == kPolyEvery - 1) ? ex2_poly(x) : ex2_approx(x);
+      if (kDiag)
+        part[e] += (col >= first_col) ? pr : 0.f;
+      else
+        part[e] += pr;
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(320, 2)
     attn_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_kc,
                        const __grid_constant__ CUtensorMap tm_kn, const AttnParams p) {
   using L = ColLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
@@ -74,7 +101,9 @@ __global__ void __launch_bounds__(320, 2)
   const uint32_t bar_k = sbase + L::kBarOff;
   const uint32_t bar_q_full0 = bar_k + 8;
   const uint32_t bar_q_empty0 = bar_q_full0 + 8 * L::kQStages;
-  const uint32_t bar_s_full0 = bar_q_empty0 + 8 * L::kQStages;
+  const uint32_t bar_l_full0 = bar_q_empty0 + 8 * L::kQStages;
+  const uint32_t bar_l_empty0 = bar_l_full0 + 8 * L::kLseStages;
+  const uint32_t bar_s_full0 = bar_l_empty0 + 8 * L::kLseStages;
   const uint32_t bar_s_empty0 = bar_s_full0 + 16;
   const uint32_t bar_drain = bar_s_empty0 + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
@@ -85,7 +114,11 @@ __global__ void __launch_bounds__(320, 2)
     mbar_init(bar_k, 1);
     for (int s = 0; s < L::kQStages; ++s) {
       mbar_init(bar_q_full0 + 8 * s, 1);
-      mbar_init(bar_q_empty0 + 8 * s, 1 + 256);  // MMA commit + every summing thread
+      mbar_init(bar_q_empty0 + 8 * s, 1);  // the MMA's commit
+    }
+    for (int s = 0; s < L::kLseStages; ++s) {
+      mbar_init(bar_l_full0 + 8 * s, 1);
+      mbar_init(bar_l_empty0 + 8 * s, 256);  // every summing thread
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_s_full0 + 8 * s, 1);
@@ -113,26 +146,35 @@ __global__ void __launch_bounds__(320, 2)
         else
           tma_load_3d(sbase + L::kKOff + r * 16384, &tm_kc, bar_k, r * 64, j0, b * p.Hkv + g);
       }
-      int issued = 0;
+      int issued_q = 0, issued_l = 0;
       for (int u = 0; u < R; ++u) {
+        const int h = g * p.G + u / span;
+        const int qt = qt_min + u % span;
         const int s = u % L::kQStages;
         if (u >= L::kQStages &&
             !mbar_wait(bar_q_empty0 + 8 * s, ((u / L::kQStages) + 1) & 1, p.err, abort_flag))
           break;
-        const int h = g * p.G + u / span;
-        const int qt = qt_min + u % span;
-        const uint32_t bar = bar_q_full0 + 8 * s;
-        mbar_arrive_expect_tx(bar, L::kTileBytes + 512);
-        const uint32_t dst = sbase + L::kQOff + s * L::kTileBytes;
+        mbar_arrive_expect_tx(bar_q_full0 + 8 * s, L::kTileBytes);
         for (int r = 0; r < L::kRegions; ++r)
-          tma_load_4d(dst + r * 16384, &tm_q, bar, r * 64, h, qt * 128, b);
-        bulk_load(sbase + L::kLseOff + s * 512,
-                  p.lse2 + (static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + qt * 128, 512, bar);
-        issued = u + 1;
+          tma_load_4d(sbase + L::kQOff + s * L::kTileBytes + r * 16384, &tm_q, bar_q_full0 + 8 * s,
+                      r * 64, h, qt * 128, b);
+        issued_q = u + 1;
+        const int sl = u % L::kLseStages;
+        if (u >= L::kLseStages &&
+            !mbar_wait(bar_l_empty0 + 8 * sl, ((u / L::kLseStages) + 1) & 1, p.err, abort_flag))
+          break;
+        mbar_arrive_expect_tx(bar_l_full0 + 8 * sl, 512);
+        bulk_load(sbase + L::kLseOff + sl * 512,
+                  p.lse2 + (static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + qt * 128, 512,
+                  bar_l_full0 + 8 * sl);
+        issued_l = u + 1;
       }
+      // drain: every issued copy has landed before the CTA can exit
       mbar_wait_drain(bar_k, 0, p.err);
-      for (int u = (issued > L::kQStages ? issued - L::kQStages : 0); u < issued; ++u)
+      for (int u = (issued_q > L::kQStages ? issued_q - L::kQStages : 0); u < issued_q; ++u)
         mbar_wait_drain(bar_q_full0 + 8 * (u % L::kQStages), (u / L::kQStages) & 1, p.err);
+      for (int u = (issued_l > L::kLseStages ? issued_l - L::kLseStages : 0); u < issued_l; ++u)
+        mbar_wait_drain(bar_l_full0 + 8 * (u % L::kLseStages), (u / L::kLseStages) & 1, p.err);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -167,7 +209,7 @@ __global__ void __launch_bounds__(320, 2)
     float acc = 0.f;
     bool ok = true;
     for (int u = 0; u < R; ++u) {
-      const int s = u % L::kQStages;
+      const int sl = u % L::kLseStages;
       const int sb = u & 1;
       ok = mbar_wait(bar_s_full0 + 8 * sb, (u >> 1) & 1, p.err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
@@ -179,39 +221,18 @@ __global__ void __launch_bounds__(320, 2)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar_s_empty0 + 8 * sb);
-      // lse2 of this row tile (already landed: the MMA waited for it)
-      ok = mbar_wait(bar_q_full0 + 8 * s, (u / L::kQStages) & 1, p.err, abort_flag);
+      ok = mbar_wait(bar_l_full0 + 8 * sl, (u / L::kLseStages) & 1, p.err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      const float4* lse4 = reinterpret_cast<const float4*>(smem + L::kLseOff + s * 512) + half * 16;
+      const float4* lse4 = reinterpret_cast<const float4*>(smem + L::kLseOff + sl * 512) + half * 16;
       const int qt = qt_min + u % span;
-      // on the diagonal tile query i0+col sees key j0+row iff row <= col
-      const int first_col = (is_chunk && qt == kt) ? row - half * 64 : 0;
-      float part = 0.f;
-#pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        const float4 ls = lse4[q4];
-        const float l4[4] = {ls.x, ls.y, ls.z, ls.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int col = q4 * 4 + e;
-          const float pr = ex2_approx(__uint_as_float(v0[col]) * c - l4[e]);
-          part += (col >= first_col) ? pr : 0.f;
-        }
-      }
-#pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        const float4 ls = lse4[8 + q4];
-        const float l4[4] = {ls.x, ls.y, ls.z, ls.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int col = 32 + q4 * 4 + e;
-          const float pr = ex2_approx(__uint_as_float(v1[q4 * 4 + e]) * c - l4[e]);
-          part += (col >= first_col) ? pr : 0.f;
-        }
-      }
-      acc += part;
-      mbar_arrive(bar_q_empty0 + 8 * s);
+      float part[4] = {0.f, 0.f, 0.f, 0.f};
+      if (is_chunk && qt == kt)  // diagonal tile: query i0+col sees key j0+row iff row <= col
+        sum_tile<true>(v0, v1, lse4, c, row - half * 64, part);
+      else
+        sum_tile<false>(v0, v1, lse4, c, 0, part);
+      acc += (part[0] + part[1]) + (part[2] + part[3]);
+      mbar_arrive(bar_l_empty0 + 8 * sl);
     }
     // combine the two column halves in a fixed order
     if (half == 1) red[row] = acc;

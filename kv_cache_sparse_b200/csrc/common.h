@@ -9,6 +9,10 @@ namespace h2o {
 // Device error bits, latched in state[2].
 constexpr int kDevErrTimeout = 1;  // a bounded mbarrier wait expired
 constexpr int kDevErrPlan = 2;     // freed-slot and kept-token counts disagree
+constexpr int kDevErrSmem = 4;     // dynamic shared memory too small after alignment
+
+// Largest dynamic shared memory a CTA may request on sm_100 (227 KiB).
+constexpr int kMaxDynSmem = 232448;
 
 // Longest time a kernel thread waits on one mbarrier phase before it gives up.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

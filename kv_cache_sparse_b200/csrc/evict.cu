@@ -20,9 +20,9 @@
 //   4. Ordered compaction (block scans over contiguous per-thread ranges)
 //      lists the free slots (evicted or empty) and the kept new tokens in
 //      ascending order; the k-th kept token goes to the k-th free slot.  The
-//      CTA writes the score and position of the placed tokens and the plan.
-// h2o_scatter (many CTAs per (cache, KV head)): copies the K and V rows of the
-// placed tokens into their slots with 16-byte vector loads and stores.
+//      CTA writes the score and position of the placed tokens and the plan,
+//      then copies their K and V rows into the slots (one warp per token,
+//      16-byte vector loads and stores).
 #include "attn.h"
 #include "sm100.cuh"
 
@@ -31,6 +31,7 @@ namespace h2o {
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr uint32_t kProtectedKey = 0xFFFFFFFFu;
+constexpr int kSubHists = 8;  // spreads the shared-memory atomics of the first radix passes
 
 __device__ __forceinline__ uint32_t score_key(float s) {
   uint32_t u = __float_as_uint(s);
@@ -65,39 +66,97 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total
   return before;
 }
 
+// Copies the K and V rows of new token `tok` into slot `slot`: one warp, one
+// 16-byte vector per lane and pass (K vectors first, then V vectors).
+__device__ __forceinline__ void move_rows(const EvictParams& e, int b, int g, int slot, int tok,
+                                          int lane) {
+  const int vpr = e.d * e.esize / 16;  // vectors per row
+  const size_t row_bytes = static_cast<size_t>(e.d) * e.esize;
+  const size_t src_off = ((static_cast<size_t>(b) * e.nq + tok) * e.Hkv + g) * row_bytes;
+  const size_t dst_off = ((static_cast<size_t>(b) * e.Hkv + g) * e.C + slot) * row_bytes;
+  for (int v = lane; v < 2 * vpr; v += 32) {
+    const bool is_v = v >= vpr;
+    const int vv = is_v ? v - vpr : v;
+    const uint4* src =
+        reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(is_v ? e.v_new : e.k_new) + src_off);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(is_v ? e.v_cache : e.k_cache) + dst_off);
+    dst[vv] = __ldg(src + vv);
+  }
+}
+
+constexpr int kLoadBatch = 8;  // global loads in flight per thread in the first pass
+
 __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e) {
   extern __shared__ uint32_t keys[];  // [n + nq]
+  __shared__ int sub_hist[kSubHists][256];  // warp w counts into sub_hist[w % kSubHists]
   __shared__ int hist[256];
   __shared__ int warp_sums[kSelWarps];
   __shared__ int sel_bin, sel_above;
 
   const int bg = blockIdx.x;
+  const int b = bg / e.Hkv, g = bg % e.Hkv;
   const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
   const int n = e.n, nq = e.nq, C = e.C;
   const int NC = n + nq;
-  float* score = e.scores + static_cast<size_t>(bg) * C;
-  int* pos = e.pos + static_cast<size_t>(bg) * C;
-  const float* cs = e.colsum + static_cast<size_t>(bg) * e.colsum_ld;
-  int* slots = e.plan_slots + static_cast<size_t>(bg) * e.plan_ld;
-  int* toks = e.plan_tokens + static_cast<size_t>(bg) * e.plan_ld;
+  float* __restrict__ score = e.scores + static_cast<size_t>(bg) * C;
+  int* __restrict__ pos = e.pos + static_cast<size_t>(bg) * C;
+  const float* __restrict__ cs = e.colsum + static_cast<size_t>(bg) * e.colsum_ld;
+  int* __restrict__ slots = e.plan_slots + static_cast<size_t>(bg) * e.plan_ld;
+  int* __restrict__ toks = e.plan_tokens + static_cast<size_t>(bg) * e.plan_ld;
   const bool evict = NC > C;
   const long long limit = static_cast<long long>(e.t0) + nq - e.W;
+  // an old slot (position < t0) can be protected only when W > nq
+  const bool old_protectable = evict && e.W > nq;
+  if (bg == 0 && tid == 0) {
+    e.state[0] = min(C, n + nq);
+    e.state[1] = e.t0 + nq;
+  }
 
-  // 1. accumulate scores, build the keys
-  for (int x = tid; x < NC; x += kSelThreads) {
-    float s;
-    long long ps;
-    if (x < n) {
-      s = score[x] + cs[x];
-      score[x] = s;
-      ps = pos[x];
-    } else {
-      s = cs[C + (x - n)];
-      ps = static_cast<long long>(e.t0) + (x - n);
+  // 1. accumulate scores and build the keys; loads are batched so that
+  //    kLoadBatch of them are in flight per thread
+  for (int x0 = tid; x0 < n; x0 += kLoadBatch * kSelThreads) {
+    float sc[kLoadBatch], cv[kLoadBatch];
+    int ps[kLoadBatch];
+#pragma unroll
+    for (int k = 0; k < kLoadBatch; ++k) {
+      const int x = x0 + k * kSelThreads;
+      sc[k] = 0.f;
+      cv[k] = 0.f;
+      ps[k] = -1;
+      if (x < n) {
+        sc[k] = score[x];
+        cv[k] = cs[x];
+        if (old_protectable) ps[k] = pos[x];
+      }
     }
-    keys[x] = (evict && ps >= limit) ? kProtectedKey : score_key(s);
+#pragma unroll
+    for (int k = 0; k < kLoadBatch; ++k) {
+      const int x = x0 + k * kSelThreads;
+      if (x < n) {
+        const float s = sc[k] + cv[k];
+        score[x] = s;
+        keys[x] = (old_protectable && ps[k] >= limit) ? kProtectedKey : score_key(s);
+      }
+    }
+  }
+  for (int i0 = tid; i0 < nq; i0 += kLoadBatch * kSelThreads) {
+    float cv[kLoadBatch];
+#pragma unroll
+    for (int k = 0; k < kLoadBatch; ++k) {
+      const int i = i0 + k * kSelThreads;
+      cv[k] = i < nq ? cs[C + i] : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < kLoadBatch; ++k) {
+      const int i = i0 + k * kSelThreads;
+      if (i < nq)
+        keys[n + i] = (evict && static_cast<long long>(e.t0) + i >= limit) ? kProtectedKey
+                                                                           : score_key(cv[k]);
+    }
   }
   if (!evict) {
+    // fill phase: every new token goes to slot n + i
     for (int i = tid; i < nq; i += kSelThreads) {
       slots[i] = n + i;
       toks[i] = i;
@@ -105,6 +164,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
       pos[n + i] = e.t0 + i;
     }
     if (tid == 0) e.plan_count[bg] = nq;
+    for (int q = warp; q < nq; q += kSelWarps) move_rows(e, b, g, n + q, q, lane);
     return;
   }
   __syncthreads();
@@ -113,8 +173,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
   uint32_t prefix = 0, pmask = 0;
   int k = C;  // rank (1-based, descending) still to locate
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
+    for (int i = tid; i < kSubHists * 256; i += kSelThreads) (&sub_hist[0][0])[i] = 0;
     __syncthreads();
+    int* my_hist = sub_hist[warp % kSubHists];
     const int iters = (NC + kSelThreads - 1) / kSelThreads;
     for (int it = 0; it < iters; ++it) {
       const int x = it * kSelThreads + tid;
@@ -124,7 +185,14 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
         if ((key & pmask) == prefix) bin = (key >> shift) & 255;
       }
       const unsigned same = __match_any_sync(0xffffffffu, bin);
-      if (bin < 256 && (__ffs(same) - 1) == (tid & 31)) atomicAdd(&hist[bin], __popc(same));
+      if (bin < 256 && (__ffs(same) - 1) == lane) atomicAdd(&my_hist[bin], __popc(same));
+    }
+    __syncthreads();
+    if (tid < 256) {
+      int total = 0;
+#pragma unroll
+      for (int h = 0; h < kSubHists; ++h) total += sub_hist[h][tid];
+      hist[tid] = total;
     }
     __syncthreads();
     if (tid < 32) {
@@ -167,12 +235,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
   for (int x = lo; x < hi; ++x) n_eq += (keys[x] == T);
   int tot;
   int eq_before = block_excl_scan(n_eq, warp_sums, &tot);
-  int n_free = 0, n_new = 0;
+  int free_old = 0, n_new = 0;
   for (int x = lo; x < hi; ++x) {
     const uint32_t key = keys[x];
     bool kept = key > T;
     if (key == T) kept = (eq_before++ < k);
-    if (x < n) n_free += !kept;
+    if (x < n) free_old += !kept;
     else n_new += kept;
     keys[x] = kept ? 1u : 0u;  // from here on: kept flag
   }
@@ -180,10 +248,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
   const int empty = C - n;
   const int e_per = (empty + kSelThreads - 1) / kSelThreads;
   const int e_lo = n + min(empty, tid * e_per), e_hi = n + min(empty, (tid + 1) * e_per);
-  n_free += e_hi - e_lo;
   // free slots are ordered: evicted slots (< n) of threads 0..1023, then the
   // empty slots (>= n) of threads 0..1023; scan the two parts separately
-  const int free_old = n_free - (e_hi - e_lo);
   int tot_free_old, tot_empty, tot_new;
   const int fo_before = block_excl_scan(free_old, warp_sums, &tot_free_old);
   const int em_before = block_excl_scan(e_hi - e_lo, warp_sums, &tot_empty);
@@ -206,45 +272,17 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
   int em = tot_free_old + em_before;
   for (int s = e_lo; s < e_hi; ++s) slots[em++] = s;
   __syncthreads();
-  // 4. scores and positions of the placed tokens
+  // 4. scores and positions of the placed tokens, then their K/V rows
   for (int q = tid; q < tot_new; q += kSelThreads) {
     const int s = slots[q], i = toks[q];
     score[s] = cs[C + i];
     pos[s] = e.t0 + i;
   }
   if (tid == 0) e.plan_count[bg] = tot_new;
+  for (int q = warp; q < tot_new; q += kSelWarps) move_rows(e, b, g, slots[q], toks[q], lane);
 }
 
-// One 16-byte vector per thread; rows of d * esize bytes (a multiple of 16).
-__global__ void __launch_bounds__(256) h2o_scatter(const EvictParams e) {
-  const int bg = blockIdx.x;
-  const int b = bg / e.Hkv, g = bg % e.Hkv;
-  const int count = e.plan_count[bg];
-  const int vpr = e.d * e.esize / 16;  // vectors per row
-  const int total = 2 * count * vpr;   // K rows then V rows
-  const int* slots = e.plan_slots + static_cast<size_t>(bg) * e.plan_ld;
-  const int* toks = e.plan_tokens + static_cast<size_t>(bg) * e.plan_ld;
-  const size_t row_bytes = static_cast<size_t>(e.d) * e.esize;
-  for (int w = blockIdx.y * blockDim.x + threadIdx.x; w < total; w += gridDim.y * blockDim.x) {
-    const int which = w / (count * vpr);  // 0: K, 1: V
-    const int r = w % (count * vpr);
-    const int q = r / vpr, v = r % vpr;
-    const int s = slots[q], i = toks[q];
-    const uint8_t* src = static_cast<const uint8_t*>(which ? e.v_new : e.k_new) +
-                         ((static_cast<size_t>(b) * e.nq + i) * e.Hkv + g) * row_bytes;
-    uint8_t* dst = static_cast<uint8_t*>(which ? e.v_cache : e.k_cache) +
-                   ((static_cast<size_t>(b) * e.Hkv + g) * e.C + s) * row_bytes;
-    const uint4 val = __ldg(reinterpret_cast<const uint4*>(src) + v);
-    reinterpret_cast<uint4*>(dst)[v] = val;
-  }
-  if (bg == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
-    e.state[0] = min(e.C, e.n + e.nq);
-    e.state[1] = e.t0 + e.nq;
-  }
-}
-
-cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st,
-                         cudaEvent_t between) {
+cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(e.n + e.nq) * sizeof(uint32_t);
   static int attr_bits[2] = {0, 0};
   if (!smem_attr_done(reinterpret_cast<const void*>(h2o_select), attr_bits)) {
@@ -252,17 +290,7 @@ cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st,
                                            kMaxCandidates * 4);
     if (err != cudaSuccess) return err;
   }
-  const int units = e.B * e.Hkv;
-  h2o_select<<<units, kSelThreads, smem, st>>>(e);
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-  if (between) cudaEventRecord(between, st);
-  const int vpr = e.d * e.esize / 16;
-  const int work = 2 * e.nq * vpr;
-  int gy = cdiv(work, 256);
-  const int target = 4 * 148;  // spread the copy over every SM
-  gy = max(1, min(gy, cdiv(target, units)));
-  h2o_scatter<<<dim3(units, gy), 256, 0, st>>>(e);
+  h2o_select<<<e.B * e.Hkv, kSelThreads, smem, st>>>(e);
   (void)max_chunk;
   return cudaGetLastError();
 }

@@ -2,11 +2,11 @@
 //
 // Validates arguments, lays out the caller's workspace, encodes the TMA
 // descriptors of each call and launches the four kernels of a step on the
-// caller's stream:
+// caller's stream (three kernels; the K/V scatter is fused into K3):
 //   K1 attention forward + row statistics   (attn_fwd.cu, tcgen05)
 //   K2 summed attention weights per key     (attn_colsum.cu, tcgen05)
-//   K3 score update + top-C selection       (evict.cu)
-//   K4 K/V scatter into the freed slots     (evict.cu)
+//   K3 score update + top-C selection + K/V scatter into the freed slots
+//                                           (evict.cu)
 // Float32 caches use the fp32 kernels of attn_f32.cu for K1/K2.
 #include <math.h>
 #include <stdlib.h>
@@ -253,11 +253,10 @@ h2o_status run_evict(h2o_cache* c, const float* colsum, int ld, const void* kn, 
     for (int i = 0; i < 5; ++i) c->ev_used[i] = false;
     mark(c, 2, st);
   }
-  cudaError_t err = launch_evict(e, g.max_chunk, st, c->timing ? c->ev[3] : nullptr);
+  cudaError_t err = launch_evict(e, g.max_chunk, st);
   if (err != cudaSuccess) return H2O_ERR_CUDA;
-  if (c->timing) c->ev_used[3] = true;
-  c->launches += 2;
-  mark(c, 4, st);
+  c->launches += 1;
+  mark(c, 3, st);
   c->n = c->n + nq < g.capacity ? c->n + nq : g.capacity;
   c->t0 += nq;
   return H2O_OK;
@@ -451,7 +450,7 @@ h2o_status h2o_cache_check(h2o_cache* c, void* stream) {
   if (cudaMemcpy(&word, c->buf.state + 2, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
     return H2O_ERR_CUDA;
   if (word & kDevErrTimeout) return H2O_ERR_TIMEOUT;
-  if (word & kDevErrPlan) return H2O_ERR_STATE;
+  if (word & (kDevErrPlan | kDevErrSmem)) return H2O_ERR_STATE;
   return H2O_OK;
 }
 

@@ -42,14 +42,19 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// One bounded probe of the phase with the given parity.  The hint lets the
+// hardware suspend the thread (up to kWaitSuspendNs) until the phase
+// completes instead of returning at once, so waiting warps do not spin.
+constexpr uint32_t kWaitSuspendNs = 100000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kWaitSuspendNs)
       : "memory");
   return ok != 0;
 }
@@ -250,6 +255,33 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x for x <= 0 on the FMA pipe, to take part of the exponentials off the
+// MUFU unit.  Argument reduction after Cody and Waite: r = round(x) (adding
+// 1.5 * 2^23 rounds x to an integer held in the low mantissa bits of t), f =
+// x - r in [-1/2, 1/2] (exact); 2^f is a degree-4 polynomial whose
+// coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez
+// exchange; fitted by kv_cache_sparse_b200/fit_exp2.py: 2.6e-6); 2^r is added
+// to the exponent field.  x is clamped to -125 so that the result stays a
+// normal float; for x < -125 it returns ~2^-125 instead of a smaller value.
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float r = t - 12582912.0f;
+  const float f = x - r;
+  float p = fmaf(0.0095701019080826049f, f, 0.05591786031930443f);
+  p = fmaf(p, f, 0.2402474482794402f);
+  p = fmaf(p, f, 0.6931218147367707f);
+  p = fmaf(p, f, 0.99999926144571449f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -132,7 +132,7 @@ def test_launch_count_and_state_word():
     q, kn, vn = ChunkSource(SMALL_QWEN, seed=3).chunk(0)
     before = gpu.info()["kernel_launches"]
     gpu.step(q.cuda(), kn.cuda(), vn.cuda())
-    assert gpu.info()["kernel_launches"] - before == 4
+    assert gpu.info()["kernel_launches"] - before == 3
     assert gpu.check() == 0
     st = gpu.state.cpu().tolist()
     assert st[0] == 256 and st[1] == 256 and st[2] == 0
