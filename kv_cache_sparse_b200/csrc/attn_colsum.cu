@@ -179,12 +179,12 @@ __global__ void __launch_bounds__(320, 2)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, false, false);
-      bool ok = mbar_wait(bar_k, 0, p.err, abort_flag);
+      bool ok = mbar_wait_spin(bar_k, 0, p.err, abort_flag);
       for (int u = 0; u < R && ok; ++u) {
         const int s = u % L::kQStages;
         const int sb = u & 1;
-        ok = mbar_wait(bar_q_full0 + 8 * s, (u / L::kQStages) & 1, p.err, abort_flag);
-        if (ok && u >= 2) ok = mbar_wait(bar_s_empty0 + 8 * sb, ((u >> 1) + 1) & 1, p.err, abort_flag);
+        ok = mbar_wait_spin(bar_q_full0 + 8 * s, (u / L::kQStages) & 1, p.err, abort_flag);
+        if (ok && u >= 2) ok = mbar_wait_spin(bar_s_empty0 + 8 * sb, ((u >> 1) + 1) & 1, p.err, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint32_t qbase = sbase + L::kQOff + s * L::kTileBytes;

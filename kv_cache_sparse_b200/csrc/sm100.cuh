@@ -59,6 +59,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// One non-suspending probe (for the single MMA-issuing thread, whose warp has
+// nothing else to do: waking it from a suspension costs hundreds of cycles on
+// the critical path).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Spinning variant of mbar_wait (same limit and abort protocol).
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, int* err,
+                                               volatile int* abort) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t start = global_timer_ns();
+  uint32_t n = 0;
+  while (true) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((++n & 255) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - start > kWaitLimitNs) {
+        *abort = 1;
+        atomicOr(err, kDevErrTimeout);
+        return false;
+      }
+    }
+  }
+}
+
 // Waits for the phase with the given parity to complete.  Gives up after
 // kWaitLimitNs (or at once when another thread of the CTA already gave up,
 // signalled through *abort), latches kDevErrTimeout in *err and returns false.
@@ -178,6 +212,18 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem], kind::f16.  A (M = 128 rows on the TMEM
+// lanes) holds two bf16 K-elements per 32-bit column: 8 columns per K = 16.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives once on the mbarrier when all previously issued tcgen05 operations
 // of this thread have completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -275,6 +321,26 @@ __device__ __forceinline__ float ex2_poly(float x) {
   p = fmaf(p, f, 0.6931218147367707f);
   p = fmaf(p, f, 0.99999926144571449f);
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Two fp32 operations per instruction (packed f32x2, sm_100):
+// (a0, a1) * (b0, b1) + (c0, c1), and (a0, a1) + (b0, b1), round to nearest.
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                      float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0,
+                                      float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
 // Three-input maximum (one instruction on sm_100).
