@@ -166,8 +166,11 @@ class H2OCache:
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h is not None and h.value:
-            lib().h2o_cache_destroy(h)
+        if h is not None and h.value and _lib is not None:
+            try:
+                _lib.h2o_cache_destroy(h)
+            except Exception:  # interpreter shutdown
+                pass
             self._h = None
 
     # ----------------------------------------------------------------- shapes

@@ -3,9 +3,9 @@
 // colsum[b, g, key] = sum over the G query heads of KV head g and the chunk's
 // queries of softmax probability P[h, i, key] ("Learning how to Forget", §1:
 // the SDPA kernel returns summed attention weights, the H2O score input).
-// P is rebuilt from the logits and the row statistic lse2 written by the
-// forward kernel: P = 2^(x - lse2), x = scale*log2(e)*<q, k>.  Nothing of P
-// is stored.
+// P is rebuilt from the logits and the row statistic written by the forward
+// kernel (minus lse2): P = 2^(x - lse2), x = scale*log2(e)*<q, k>.  Nothing
+// of P is stored.
 //
 // Key-stationary: one CTA per (cache, KV head, tile of 128 keys).  The MMA
 // computes S^T = K_tile Q_rows^T with the keys on the 128 TMEM lanes, so every
@@ -41,29 +41,37 @@ struct ColLayout {
   static constexpr int kThreads = 320;
 };
 
-// Every kPolyEvery-th probability is computed with the FMA-pipe polynomial,
-// the rest with the MUFU ex2 instruction, so that both units share the work.
+// Every fourth probability is computed with the FMA-pipe polynomial, the rest
+// with the MUFU ex2 instruction, so that both units share the work.
 constexpr int kPolyEvery = 4;
 
 template <bool kDiag>
 __device__ __forceinline__ void sum_tile(const uint32_t (&v0)[32], const uint32_t (&v1)[32],
-                                         const float4* lse4, float c, int first_col,
+                                         const float4* nlse4, float c, int first_col,
                                          float (&part)[4]) {
+  // x = s * c + (-lse2) two columns at a time (packed f32x2), then 2^x and
+  // the running sums, also packed
 #pragma unroll
   for (int q4 = 0; q4 < 16; ++q4) {
-    const float4 ls = lse4[q4];
-    const float l4[4] = {ls.x, ls.y, ls.z, ls.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int col = q4 * 4 + e;
-      const uint32_t sx = q4 < 8 ? v0[col] : v1[col - 32];
-      const float x = fmaf(__uint_as_float(sx), c, -l4[e]);
-      const float pr = (col % kPolyEvery == kPolyEvery - 1) ? ex2_poly(x) : ex2_approx(x);
-      if (kDiag)
-        part[e] += (col >= first_col) ? pr : 0.f;
-      else
-        part[e] += pr;
+    const float4 nl = nlse4[q4];
+    const int col = q4 * 4;
+    const uint32_t s0 = q4 < 8 ? v0[col] : v1[col - 32];
+    const uint32_t s1 = q4 < 8 ? v0[col + 1] : v1[col - 31];
+    const uint32_t s2 = q4 < 8 ? v0[col + 2] : v1[col - 30];
+    const uint32_t s3 = q4 < 8 ? v0[col + 3] : v1[col - 29];
+    float x0, x1, x2, x3;
+    ffma2(x0, x1, __uint_as_float(s0), __uint_as_float(s1), c, c, nl.x, nl.y);
+    ffma2(x2, x3, __uint_as_float(s2), __uint_as_float(s3), c, c, nl.z, nl.w);
+    float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2);
+    float p3 = (kPolyEvery == 4) ? ex2_poly(x3) : ex2_approx(x3);
+    if (kDiag) {  // query i0+col sees key j0+row iff row <= col
+      p0 = (col >= first_col) ? p0 : 0.f;
+      p1 = (col + 1 >= first_col) ? p1 : 0.f;
+      p2 = (col + 2 >= first_col) ? p2 : 0.f;
+      p3 = (col + 3 >= first_col) ? p3 : 0.f;
     }
+    fadd2(part[0], part[1], part[0], part[1], p0, p1);
+    fadd2(part[2], part[3], part[2], part[3], p2, p3);
   }
 }
 
@@ -165,7 +173,7 @@ __global__ void __launch_bounds__(320, 2)
           break;
         mbar_arrive_expect_tx(bar_l_full0 + 8 * sl, 512);
         bulk_load(sbase + L::kLseOff + sl * 512,
-                  p.lse2 + (static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + qt * 128, 512,
+                  p.nlse2 + (static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + qt * 128, 512,
                   bar_l_full0 + 8 * sl);
         issued_l = u + 1;
       }
@@ -224,13 +232,14 @@ __global__ void __launch_bounds__(320, 2)
       ok = mbar_wait(bar_l_full0 + 8 * sl, (u / L::kLseStages) & 1, p.err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      const float4* lse4 = reinterpret_cast<const float4*>(smem + L::kLseOff + sl * 512) + half * 16;
+      const float4* nlse4 =
+          reinterpret_cast<const float4*>(smem + L::kLseOff + sl * 512) + half * 16;
       const int qt = qt_min + u % span;
       float part[4] = {0.f, 0.f, 0.f, 0.f};
       if (is_chunk && qt == kt)  // diagonal tile: query i0+col sees key j0+row iff row <= col
-        sum_tile<true>(v0, v1, lse4, c, row - half * 64, part);
+        sum_tile<true>(v0, v1, nlse4, c, row - half * 64, part);
       else
-        sum_tile<false>(v0, v1, lse4, c, 0, part);
+        sum_tile<false>(v0, v1, nlse4, c, 0, part);
       acc += (part[0] + part[1]) + (part[2] + part[3]);
       mbar_arrive(bar_l_empty0 + 8 * sl);
     }

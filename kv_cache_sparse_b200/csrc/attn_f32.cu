@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kF32Threads)
   float* orow = reinterpret_cast<float*>(p.out) + ((static_cast<size_t>(b) * p.nq + i) * p.Hq + h) * d;
   if (threadIdx.x < d) orow[threadIdx.x] = o0;
   if (threadIdx.x + 128 < d) orow[threadIdx.x + 128] = o1;
-  if (threadIdx.x == 0) p.lse2[(static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + i] = lse2;
+  if (threadIdx.x == 0) p.nlse2[(static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + i] = -lse2;
 }
 
 __global__ void __launch_bounds__(kF32Threads)
@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kF32Threads)
     const float* qr = q + ((static_cast<size_t>(b) * p.nq + i) * p.Hq + h) * d;
     float s = 0.f;
     for (int t = 0; t < d; ++t) s = fmaf(qr[t], ks[t], s);
-    acc += exp2f(s * c - p.lse2[(static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + i]);
+    acc += exp2f(s * c + p.nlse2[(static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + i]);
   }
   const float total = block_reduce_sum(acc, red);
   if (threadIdx.x == 0) {

@@ -5,8 +5,9 @@
 // sees the n valid cache slots of KV head h / G and the chunk keys j <= i
 // ("Learning how to Forget", §1: SDPA over a fixed-size KV cache plus the new
 // chunk; FlashInfer-style 1 << N_q << N_k regime named in §2).  It also stores
-// the row statistic lse2 = log2(sum_j 2^(x_ij)), x = scale*log2(e)*<q,k>,
-// which the column-sum kernel uses to rebuild the normalised probabilities.
+// the row statistic lse2 = log2(sum_j 2^(x_ij)), x = scale*log2(e)*<q,k>
+// (negated), which the column-sum kernel uses to rebuild the normalised
+// probabilities.
 //
 // One CTA = two 128-row query tiles ("A" and "B") of the same KV head --
 // normally two heads of one GQA group at the same 128 queries -- that share
@@ -365,8 +366,8 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
         }
-        p.lse2[(static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + i] =
-            (i < p.nq) ? m_used + __log2f(l) : INFINITY;
+        p.nlse2[(static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + i] =
+            (i < p.nq) ? -(m_used + __log2f(l)) : -INFINITY;
       }
     }
   }

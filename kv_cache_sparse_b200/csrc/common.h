@@ -36,7 +36,9 @@ struct AttnParams {
   int nq_pad;           // row stride of the row statistics (multiple of 128)
   float scale_log2;     // softmax scale * log2(e)
   void* out;            // [B, nq, Hq, d]
-  float* lse2;          // [B, Hq, nq_pad], log2-domain log-sum-exp per row
+  float* nlse2;         // [B, Hq, nq_pad]: minus the log2-domain log-sum-exp of
+                        // each row (-inf for padding rows), so 2^(x + nlse2)
+                        // is the row's normalised probability
   float* colsum;        // [B, Hkv, colsum_ld]
   int colsum_ld;        // row stride of colsum (>= C + nq)
   int* err;             // device error word (state + 2)

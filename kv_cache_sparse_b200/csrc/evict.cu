@@ -279,7 +279,21 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
     pos[s] = e.t0 + i;
   }
   if (tid == 0) e.plan_count[bg] = tot_new;
-  for (int q = warp; q < tot_new; q += kSelWarps) move_rows(e, b, g, slots[q], toks[q], lane);
+  // K/V rows: warp w moves rows w, w + 32, ...; lane L first fetches the
+  // (slot, token) of the warp's L-th row, so that the copies do not wait on
+  // one another's plan reads
+  for (int q0 = warp; q0 < tot_new; q0 += kSelWarps * 32) {
+    const int q = q0 + lane * kSelWarps;
+    const int my_slot = q < tot_new ? slots[q] : 0;
+    const int my_tok = q < tot_new ? toks[q] : 0;
+    const int rows = min(32, (tot_new - q0 + kSelWarps - 1) / kSelWarps);
+#pragma unroll 4
+    for (int r = 0; r < rows; ++r) {
+      const int sl = __shfl_sync(0xffffffffu, my_slot, r);
+      const int tk = __shfl_sync(0xffffffffu, my_tok, r);
+      move_rows(e, b, g, sl, tk, lane);
+    }
+  }
 }
 
 cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st) {

@@ -179,7 +179,7 @@ AttnParams attn_params(h2o_cache* c, int nq, void* out) {
   const float scale = g.softmax_scale > 0.f ? g.softmax_scale : 1.f / sqrtf((float)g.head_dim);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.out = out;
-  p.lse2 = c->lse2;
+  p.nlse2 = c->lse2;
   p.colsum = c->colsum;
   p.colsum_ld = c->colsum_ld;
   p.err = c->buf.state + 2;

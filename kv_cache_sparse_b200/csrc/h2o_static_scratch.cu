@@ -136,7 +136,7 @@ extern "C" H2O_API h2o_status h2o_attention_static_scratch(
   const float scale = g.softmax_scale > 0.f ? g.softmax_scale : 1.f / sqrtf((float)g.head_dim);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.out = out;
-  p.lse2 = lse2;
+  p.nlse2 = lse2;  // holds minus the row log-sum-exp
   p.colsum = colsum_out;  // written in place: [batch, H_kv, capacity + n_q]
   p.colsum_ld = g.capacity + n_q;
   p.err = err;
