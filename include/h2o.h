@@ -222,6 +222,14 @@ H2O_API h2o_status h2o_attention_static_scratch(const h2o_config* cfg, const voi
 H2O_API h2o_status h2o_selftest_exp2(const float* x, float* y_poly, float* y_lib, int32_t n,
                                      void* stream);
 
+/* Diagnostic of the failure path: one warp waits, with the same bounded
+ * wait the kernels use, on a barrier nothing completes.  After limit_us
+ * (1 .. 2,000,000) the wait gives up, ORs the timeout bit (1) into
+ * *err_word (device int32) and the kernel returns; the context stays
+ * usable.  No trap, no hang. */
+H2O_API h2o_status h2o_selftest_wait_timeout(int32_t* err_word, uint32_t limit_us,
+                                             void* stream);
+
 /* Frees the host handle only. */
 H2O_API void h2o_cache_destroy(h2o_cache* c);
 

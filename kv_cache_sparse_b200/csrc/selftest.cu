@@ -1,6 +1,10 @@
-// selftest.cu -- diagnostic entry point: evaluates the kernels' polynomial
-// base-2 exponential next to CUDA's exp2f on caller-provided inputs, so that
-// tests can check it against the library function on the device.
+// selftest.cu -- diagnostic entry points:
+//   h2o_selftest_exp2         the kernels' polynomial base-2 exponential next
+//                             to CUDA's exp2f, for accuracy tests;
+//   h2o_selftest_wait_timeout one warp waits, with the kernels' bounded wait,
+//                             on an mbarrier nothing arrives at; the wait gives
+//                             up after the given limit, latches the timeout
+//                             bit and the kernel returns (no trap, no hang).
 #include "../../include/h2o.h"
 #include "sm100.cuh"
 
@@ -14,7 +18,29 @@ __global__ void exp2_compare(const float* x, float* y_poly, float* y_lib, int n)
   }
 }
 
+__global__ void wait_timeout_probe(int* err, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = h2o::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    h2o::mbar_init(b, 1);
+    abort_flag = 0;
+    h2o::fence_barrier_init();
+  }
+  __syncthreads();
+  // phase 0 of a fresh barrier never completes: nothing arrives
+  h2o::mbar_wait_until(b, 0, err, &abort_flag, limit_ns);
+}
+
 }  // namespace
+
+extern "C" H2O_API h2o_status h2o_selftest_wait_timeout(int32_t* err_word, uint32_t limit_us,
+                                                        void* stream) {
+  if (!err_word || limit_us == 0 || limit_us > 2000000) return H2O_ERR_INVALID_ARG;
+  wait_timeout_probe<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      err_word, static_cast<uint64_t>(limit_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? H2O_OK : H2O_ERR_CUDA;
+}
 
 extern "C" H2O_API h2o_status h2o_selftest_exp2(const float* x, float* y_poly, float* y_lib,
                                                 int32_t n, void* stream) {

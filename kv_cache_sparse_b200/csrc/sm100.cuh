@@ -94,21 +94,26 @@ __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, in
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs (or at once when another thread of the CTA already gave up,
+// limit_ns (or at once when another thread of the CTA already gave up,
 // signalled through *abort), latches kDevErrTimeout in *err and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err,
-                                          volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait_until(uint32_t bar, uint32_t parity, int* err,
+                                                volatile int* abort, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t start = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - start > kWaitLimitNs) {
+    if (global_timer_ns() - start > limit_ns) {
       *abort = 1;
       atomicOr(err, kDevErrTimeout);
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err,
+                                          volatile int* abort) {
+  return mbar_wait_until(bar, parity, err, abort, kWaitLimitNs);
 }
 
 // Waits without the abort shortcut; used while draining before exit, so that
