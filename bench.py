@@ -53,6 +53,21 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the last ncu capture of `kernel`
+    (profiles/traffic.json), or None when its source changed since."""
+    from kv_cache_sparse_b200.ncu_summary import TRAFFIC_FILE, source_digest
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)[kernel]
+        src = os.path.join(ROOT, "kv_cache_sparse_b200", "csrc", rec["source"])
+        if source_digest(src) != rec["source_sha256_16"]:
+            return None
+        return rec["bytes_per_launch"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def attention_flops(wl, n, nq):
     """Algorithmic FLOPs of one step's attention: QK^T and PV over the
     visible (query, key) pairs, 2*d each, for every query head and cache."""
@@ -330,17 +345,19 @@ def run_ours(args, world, rank, local):
     dom = int(np.argmax(avg))
     if dom == 0:
         achieved = flops / (avg[0] * 1e-3) / 1e12
+        tr = recorded_traffic("attn_fwd_kernel") if wl is WL else None
         roof = {"kernel": KERNELS[0], "bound": "tensor", "achieved": round(achieved, 2),
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
-                "traffic": None, "peak_kind": f"{peaks_kind} bf16 dense (burst)",
+                "traffic": tr, "peak_kind": f"{peaks_kind} bf16 dense (burst)",
                 "per_launch": f"{flops:.4e} FLOP (QK^T + PV over visible pairs)"}
     else:
         # the summed-weights kernel: its FLOPs are the QK^T recompute
         rf = flops / 2
         achieved = rf / (avg[dom] * 1e-3) / 1e12
+        tr = recorded_traffic(KERNELS[dom]) if wl is WL else None
         roof = {"kernel": KERNELS[dom], "bound": "tensor", "achieved": round(achieved, 2),
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
-                "traffic": None, "peak_kind": f"{peaks_kind} bf16 dense (burst)",
+                "traffic": tr, "peak_kind": f"{peaks_kind} bf16 dense (burst)",
                 "per_launch": f"{rf:.4e} FLOP (QK^T recompute)"}
     attn_ms = avg[0] + avg[1]
     evict_ms = avg[2] + avg[3]

@@ -2,6 +2,7 @@
 
     python -m kv_cache_sparse_b200.ncu_summary launches <launches.csv>
     python -m kv_cache_sparse_b200.ncu_summary report <file.ncu-rep>
+    python -m kv_cache_sparse_b200.ncu_summary traffic <file.ncu-rep> <kernel> <source.cu>
 
 `launches` groups a `--metrics gpu__time_duration.sum` launch list by kernel
 (launches, total time, share); `report` prints the counters used for the
@@ -11,8 +12,24 @@ from __future__ import annotations
 
 import collections
 import csv
+import hashlib
+import json
+import os
 import subprocess
 import sys
+
+TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                            "profiles", "traffic.json")
+
+
+def source_digest(path: str) -> str:
+    """Digest of a kernel source together with the device headers it includes."""
+    h = hashlib.sha256()
+    csrc = os.path.dirname(os.path.abspath(path))
+    for p in (path, os.path.join(csrc, "sm100.cuh"), os.path.join(csrc, "common.h")):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 REPORT_KEYS = [
     "gpu__time_duration.sum", "dram__bytes_read.sum", "dram__bytes_write.sum",
@@ -71,5 +88,33 @@ def report(path):
                 print(f"  {k} = {r[i]} {units[i]}")
 
 
+def traffic(path, kernel, source):
+    """Records dram read + write bytes of one captured launch of `kernel`,
+    with the digest of its source file, in profiles/traffic.json."""
+    out = subprocess.run(["ncu", "-i", path, "--page", "raw", "--csv"], capture_output=True,
+                         text=True, check=True).stdout
+    rows = list(csv.reader(out.splitlines()))
+    hdr, units = rows[0], rows[1]
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    r = rows[2]
+    total = 0.0
+    for k in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+        i = hdr.index(k)
+        total += float(r[i].replace(",", "")) * scale[units[i]]
+    data = {}
+    if os.path.exists(TRAFFIC_FILE):
+        with open(TRAFFIC_FILE) as f:
+            data = json.load(f)
+    data[kernel] = {"bytes_per_launch": total, "source": os.path.basename(source),
+                    "source_sha256_16": source_digest(source)}
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(data, f, indent=1, sort_keys=True)
+    print(kernel, total)
+
+
 if __name__ == "__main__":
-    {"launches": launches, "report": report}[sys.argv[1]](sys.argv[2])
+    cmd = sys.argv[1]
+    if cmd == "traffic":
+        traffic(sys.argv[2], sys.argv[3], sys.argv[4])
+    else:
+        {"launches": launches, "report": report}[cmd](sys.argv[2])
