@@ -233,20 +233,28 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def _reduce(x: float, world: int, op) -> float:
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Step time of the job: the slowest rank's."""
+    return _reduce(x, world, torch.distributed.ReduceOp.MAX)
 
 
 def sum_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
-    return float(t.item())
+    """Work of the job: every rank's units."""
+    return _reduce(x, world, torch.distributed.ReduceOp.SUM)
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank runs its own caches, drawn from its own seed."""
+    return 1000 * rank
 
 
 # ---------------------------------------------------------------- our arm
@@ -264,7 +272,7 @@ def run_ours(args, world, rank, local):
                                wl.capacity, wl.chunk, wl.window, wl.torch_dtype())
     cache = binding.H2OCache(shape, device=dev)
     stream = torch.cuda.current_stream(dev)
-    seed = 1000 * rank
+    seed = rank_seed(rank)
     # fill phase (untimed): C / n_q steps bring the cache to steady state
     fill = wl.capacity // wl.chunk
     for c in range(fill):
