@@ -14,8 +14,12 @@
 // 128 queries of one head; the sum order is fixed, so results are
 // deterministic (no atomics).
 //   warp 0      TMA producer: the key tile once, then Q tiles + their lse2
-//   warp 1      TMEM allocation; one thread issues the tcgen05.mma
-//   warps 2..9  two threads per key: columns 0..63 and 64..127 of each tile
+//   warp 1      TMEM allocation; one thread issues the tcgen05.mma into a
+//               ring of four 128-column S buffers
+//   warps 2..5  row tiles 0, 2, 4, ...; warps 6..9 row tiles 1, 3, 5, ...:
+//               one thread per key, all 128 query columns of its tiles.  The
+//               two warpgroups work out of phase (each one's next S is ready
+//               while it sums), so the exponential units stay busy.
 #include "attn.h"
 #include "sm100.cuh"
 
@@ -25,19 +29,20 @@ template <int D>
 struct ColLayout {
   static constexpr int kRegions = D / 64;
   static constexpr int kTileBytes = 128 * D * 2;
-  static constexpr int kQStages = 2;    // Q tiles, released when their MMA completes
-  static constexpr int kLseStages = 4;  // row statistics, released by the summing threads
+  static constexpr int kQStages = 4;    // Q tiles, released when their MMA completes
+  static constexpr int kLseStages = 8;  // row statistics, released by the summing group
+  static constexpr int kSBufs = 4;      // TMEM S buffers (two per summing group)
   static constexpr int kKOff = 0;
   static constexpr int kQOff = kKOff + kTileBytes;
   static constexpr int kLseOff = kQOff + kQStages * kTileBytes;  // 512 bytes per stage
   static constexpr int kBarOff = kLseOff + kLseStages * 512;
-  // k_full, q_full[QS], q_empty[QS], lse_full[LS], lse_empty[LS], s_full[2], s_empty[2], drain
-  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kLseStages + 4 + 1;
+  // k_full, q_full[QS], q_empty[QS], lse_full[LS], lse_empty[LS], s_full[SB], s_empty[SB], drain
+  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kLseStages + 2 * kSBufs + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kRedOff = kMiscOff + 16;
   static constexpr int kBytes = kRedOff + 128 * 4;
   static constexpr int kAlloc = kBytes + 1024;
-  static constexpr int kTmemCols = 256;
+  static constexpr int kTmemCols = 512;
   static constexpr int kThreads = 320;
 };
 
@@ -76,7 +81,7 @@ __device__ __forceinline__ void sum_tile(const uint32_t (&v0)[32], const uint32_
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 2)
+__global__ void __launch_bounds__(320, 1)
     attn_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_kc,
                        const __grid_constant__ CUtensorMap tm_kn, const AttnParams p) {
@@ -112,8 +117,8 @@ __global__ void __launch_bounds__(320, 2)
   const uint32_t bar_l_full0 = bar_q_empty0 + 8 * L::kQStages;
   const uint32_t bar_l_empty0 = bar_l_full0 + 8 * L::kLseStages;
   const uint32_t bar_s_full0 = bar_l_empty0 + 8 * L::kLseStages;
-  const uint32_t bar_s_empty0 = bar_s_full0 + 16;
-  const uint32_t bar_drain = bar_s_empty0 + 16;
+  const uint32_t bar_s_empty0 = bar_s_full0 + 8 * L::kSBufs;
+  const uint32_t bar_drain = bar_s_empty0 + 8 * L::kSBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   float* red = reinterpret_cast<float*>(smem + L::kRedOff);
@@ -126,11 +131,11 @@ __global__ void __launch_bounds__(320, 2)
     }
     for (int s = 0; s < L::kLseStages; ++s) {
       mbar_init(bar_l_full0 + 8 * s, 1);
-      mbar_init(bar_l_empty0 + 8 * s, 256);  // every summing thread
+      mbar_init(bar_l_empty0 + 8 * s, 128);  // the summing group of that tile
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < L::kSBufs; ++s) {
       mbar_init(bar_s_full0 + 8 * s, 1);
-      mbar_init(bar_s_empty0 + 8 * s, 256);
+      mbar_init(bar_s_empty0 + 8 * s, 128);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -155,6 +160,7 @@ __global__ void __launch_bounds__(320, 2)
           tma_load_3d(sbase + L::kKOff + r * 16384, &tm_kc, bar_k, r * 64, j0, b * p.Hkv + g);
       }
       int issued_q = 0, issued_l = 0;
+      bool waited = false;
       for (int u = 0; u < R; ++u) {
         const int h = g * p.G + u / span;
         const int qt = qt_min + u % span;
@@ -171,6 +177,10 @@ __global__ void __launch_bounds__(320, 2)
         if (u >= L::kLseStages &&
             !mbar_wait(bar_l_empty0 + 8 * sl, ((u / L::kLseStages) + 1) & 1, p.err, abort_flag))
           break;
+        if (!waited) {  // the row statistics come from the preceding forward kernel
+          griddep_wait();
+          waited = true;
+        }
         mbar_arrive_expect_tx(bar_l_full0 + 8 * sl, 512);
         bulk_load(sbase + L::kLseOff + sl * 512,
                   p.nlse2 + (static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + qt * 128, 512,
@@ -190,9 +200,10 @@ __global__ void __launch_bounds__(320, 2)
       bool ok = mbar_wait_spin(bar_k, 0, p.err, abort_flag);
       for (int u = 0; u < R && ok; ++u) {
         const int s = u % L::kQStages;
-        const int sb = u & 1;
+        const int sb = u % L::kSBufs;
         ok = mbar_wait_spin(bar_q_full0 + 8 * s, (u / L::kQStages) & 1, p.err, abort_flag);
-        if (ok && u >= 2) ok = mbar_wait_spin(bar_s_empty0 + 8 * sb, ((u >> 1) + 1) & 1, p.err, abort_flag);
+        if (ok && u >= L::kSBufs)
+          ok = mbar_wait_spin(bar_s_empty0 + 8 * sb, ((u / L::kSBufs) + 1) & 1, p.err, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint32_t qbase = sbase + L::kQOff + s * L::kTileBytes;
@@ -210,43 +221,45 @@ __global__ void __launch_bounds__(320, 2)
     }
   } else {
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;  // 0: columns 0..63, 1: columns 64..127
+    const int grp = (warp - 2) >> 2;   // row tiles u with u % 2 == grp
     const int row = quad * 32 + lane;  // key j0 + row
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16) + half * 64;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float c = p.scale_log2;
     float acc = 0.f;
     bool ok = true;
-    for (int u = 0; u < R; ++u) {
+    for (int u = grp; u < R; u += 2) {
       const int sl = u % L::kLseStages;
-      const int sb = u & 1;
-      ok = mbar_wait(bar_s_full0 + 8 * sb, (u >> 1) & 1, p.err, abort_flag);
+      const int sb = u % L::kSBufs;
+      ok = mbar_wait(bar_s_full0 + 8 * sb, (u / L::kSBufs) & 1, p.err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      uint32_t v0[32], v1[32];
-      tmem_ld32(lane_base + sb * 128, v0);
-      tmem_ld32(lane_base + sb * 128 + 32, v1);
+      uint32_t v[4][32];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) tmem_ld32(lane_base + sb * 128 + 32 * k, v[k]);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar_s_empty0 + 8 * sb);
       ok = mbar_wait(bar_l_full0 + 8 * sl, (u / L::kLseStages) & 1, p.err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      const float4* nlse4 =
-          reinterpret_cast<const float4*>(smem + L::kLseOff + sl * 512) + half * 16;
+      const float4* nlse4 = reinterpret_cast<const float4*>(smem + L::kLseOff + sl * 512);
       const int qt = qt_min + u % span;
       float part[4] = {0.f, 0.f, 0.f, 0.f};
-      if (is_chunk && qt == kt)  // diagonal tile: query i0+col sees key j0+row iff row <= col
-        sum_tile<true>(v0, v1, nlse4, c, row - half * 64, part);
-      else
-        sum_tile<false>(v0, v1, nlse4, c, 0, part);
+      if (is_chunk && qt == kt) {  // diagonal tile: query i0+col sees key j0+row iff row <= col
+        sum_tile<true>(v[0], v[1], nlse4, c, row, part);
+        sum_tile<true>(v[2], v[3], nlse4 + 16, c, row - 64, part);
+      } else {
+        sum_tile<false>(v[0], v[1], nlse4, c, 0, part);
+        sum_tile<false>(v[2], v[3], nlse4 + 16, c, 0, part);
+      }
       acc += (part[0] + part[1]) + (part[2] + part[3]);
       mbar_arrive(bar_l_empty0 + 8 * sl);
     }
-    // combine the two column halves in a fixed order
-    if (half == 1) red[row] = acc;
+    // combine the two groups' sums in a fixed order
+    if (grp == 1) red[row] = acc;
     named_bar_sync(1, 256);
-    if (half == 0 && ok) {
+    if (grp == 0 && ok) {
       const float total = acc + red[row];
       const int key = j0 + row;
       if (is_chunk) {
@@ -261,6 +274,7 @@ __global__ void __launch_bounds__(320, 2)
 
   tc_fence_before();
   __syncthreads();
+  griddep_launch_dependents();  // the summed weights of this CTA are written
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
@@ -276,9 +290,17 @@ static cudaError_t launch_colsum(const AttnMaps& m, const AttnParams& p, cudaStr
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(cdiv(p.C, 128) + cdiv(p.nq, 128), p.B * p.Hkv);
-  attn_colsum_kernel<D><<<grid, L::kThreads, L::kAlloc, st>>>(m.q, m.kc, m.kn, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cdiv(p.C, 128) + cdiv(p.nq, 128), p.B * p.Hkv);
+  cfg.blockDim = dim3(L::kThreads);
+  cfg.dynamicSmemBytes = L::kAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_colsum_kernel<D>, m.q, m.kc, m.kn, p);
 }
 
 cudaError_t launch_attn_colsum_bf16(int head_dim, const AttnMaps& m, const AttnParams& p,

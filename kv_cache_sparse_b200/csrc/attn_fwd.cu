@@ -73,6 +73,9 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // the column-sum kernel may start setting up on idle SMs; it waits for this
+  // grid to complete before it reads the row statistics
+  griddep_launch_dependents();
 
   // ---- work: items (head of the group, query tile) of one (cache, KV head),
   // longest first, taken two at a time

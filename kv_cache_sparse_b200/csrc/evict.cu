@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
   const long long limit = static_cast<long long>(e.t0) + nq - e.W;
   // an old slot (position < t0) can be protected only when W > nq
   const bool old_protectable = evict && e.W > nq;
+  griddep_wait();  // the summed weights come from the preceding kernel
   if (bg == 0 && tid == 0) {
     e.state[0] = min(C, n + nq);
     e.state[1] = e.t0 + nq;
@@ -304,9 +305,18 @@ cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st) {
                                            kMaxCandidates * 4);
     if (err != cudaSuccess) return err;
   }
-  h2o_select<<<e.B * e.Hkv, kSelThreads, smem, st>>>(e);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(e.B * e.Hkv);
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   (void)max_chunk;
-  return cudaGetLastError();
+  return cudaLaunchKernelEx(&cfg, h2o_select, e);
 }
 
 }  // namespace h2o

@@ -173,6 +173,21 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- dependent launch
+
+// Lets the next kernel of the stream (launched with programmatic stream
+// serialization) start its CTAs now; its griddep_wait still waits for this
+// grid to complete.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Waits until the preceding kernel of the stream has completed and its
+// memory is visible (returns at once when there is no such dependency).
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- named barriers
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
