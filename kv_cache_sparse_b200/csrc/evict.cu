@@ -28,10 +28,7 @@
 
 namespace h2o {
 
-constexpr int kSelThreads = 1024;
-constexpr int kSelWarps = kSelThreads / 32;
 constexpr uint32_t kProtectedKey = 0xFFFFFFFFu;
-constexpr int kSubHists = 8;  // spreads the shared-memory atomics of the first radix passes
 
 __device__ __forceinline__ uint32_t score_key(float s) {
   uint32_t u = __float_as_uint(s);
@@ -40,7 +37,9 @@ __device__ __forceinline__ uint32_t score_key(float s) {
 
 // Exclusive scan of one value per thread over the block; returns the prefix,
 // writes the block total to *total.  All threads must call it.
+template <int NT>
 __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total) {
+  constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
@@ -52,17 +51,17 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total
   if (lane == 31) warp_sums[w] = x;
   __syncthreads();
   if (w == 0) {
-    int s = warp_sums[lane];
+    int s = lane < NW ? warp_sums[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, s, o);
       if (lane >= o) s += y;
     }
-    warp_sums[lane] = s;  // inclusive
+    if (lane < NW) warp_sums[lane] = s;  // inclusive
   }
   __syncthreads();
   const int before = (w > 0 ? warp_sums[w - 1] : 0) + x - v;
-  *total = warp_sums[kSelWarps - 1];
+  *total = warp_sums[NW - 1];
   return before;
 }
 
@@ -85,12 +84,15 @@ __device__ __forceinline__ void move_rows(const EvictParams& e, int b, int g, in
 }
 
 constexpr int kLoadBatch = 8;  // global loads in flight per thread in the first pass
+constexpr int kBins = 256;     // radix passes of 8 bits, most significant first
 
-__global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e) {
-  extern __shared__ uint32_t keys[];  // [n + nq]
-  __shared__ int sub_hist[kSubHists][256];  // warp w counts into sub_hist[w % kSubHists]
-  __shared__ int hist[256];
-  __shared__ int warp_sums[kSelWarps];
+template <int NT>
+__global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1)) h2o_select(const EvictParams e) {
+  constexpr int NW = NT / 32;
+  constexpr int kSub = (NT == 1024) ? 8 : 2;  // sub-histograms spread the first passes' atomics
+  extern __shared__ uint32_t keys[];          // [n + nq]
+  __shared__ int hist[kSub][kBins];           // warp w counts into hist[w % kSub]
+  __shared__ int warp_sums[32];
   __shared__ int sel_bin, sel_above;
 
   const int bg = blockIdx.x;
@@ -116,12 +118,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
 
   // 1. accumulate scores and build the keys; loads are batched so that
   //    kLoadBatch of them are in flight per thread
-  for (int x0 = tid; x0 < n; x0 += kLoadBatch * kSelThreads) {
+  for (int x0 = tid; x0 < n; x0 += kLoadBatch * NT) {
     float sc[kLoadBatch], cv[kLoadBatch];
     int ps[kLoadBatch];
 #pragma unroll
     for (int k = 0; k < kLoadBatch; ++k) {
-      const int x = x0 + k * kSelThreads;
+      const int x = x0 + k * NT;
       sc[k] = 0.f;
       cv[k] = 0.f;
       ps[k] = -1;
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
     }
 #pragma unroll
     for (int k = 0; k < kLoadBatch; ++k) {
-      const int x = x0 + k * kSelThreads;
+      const int x = x0 + k * NT;
       if (x < n) {
         const float s = sc[k] + cv[k];
         score[x] = s;
@@ -141,16 +143,16 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
       }
     }
   }
-  for (int i0 = tid; i0 < nq; i0 += kLoadBatch * kSelThreads) {
+  for (int i0 = tid; i0 < nq; i0 += kLoadBatch * NT) {
     float cv[kLoadBatch];
 #pragma unroll
     for (int k = 0; k < kLoadBatch; ++k) {
-      const int i = i0 + k * kSelThreads;
+      const int i = i0 + k * NT;
       cv[k] = i < nq ? cs[C + i] : 0.f;
     }
 #pragma unroll
     for (int k = 0; k < kLoadBatch; ++k) {
-      const int i = i0 + k * kSelThreads;
+      const int i = i0 + k * NT;
       if (i < nq)
         keys[n + i] = (evict && static_cast<long long>(e.t0) + i >= limit) ? kProtectedKey
                                                                            : score_key(cv[k]);
@@ -158,84 +160,91 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
   }
   if (!evict) {
     // fill phase: every new token goes to slot n + i
-    for (int i = tid; i < nq; i += kSelThreads) {
+    for (int i = tid; i < nq; i += NT) {
       slots[i] = n + i;
       toks[i] = i;
       score[n + i] = cs[C + i];
       pos[n + i] = e.t0 + i;
     }
     if (tid == 0) e.plan_count[bg] = nq;
-    for (int q = warp; q < nq; q += kSelWarps) move_rows(e, b, g, n + q, q, lane);
+    for (int q = warp; q < nq; q += NW) move_rows(e, b, g, n + q, q, lane);
     return;
   }
   __syncthreads();
 
-  // 2. radix select of the C-th largest key
+  // 2. radix select of the C-th largest key: four 8-bit digits, MSB first
   uint32_t prefix = 0, pmask = 0;
   int k = C;  // rank (1-based, descending) still to locate
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < kSubHists * 256; i += kSelThreads) (&sub_hist[0][0])[i] = 0;
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    constexpr int nb = kBins;
+    for (int i = tid; i < kSub * kBins; i += NT) (&hist[0][0])[i] = 0;
     __syncthreads();
-    int* my_hist = sub_hist[warp % kSubHists];
-    const int iters = (NC + kSelThreads - 1) / kSelThreads;
+    int* my_hist = hist[warp % kSub];
+    const int iters = (NC + NT - 1) / NT;
     for (int it = 0; it < iters; ++it) {
-      const int x = it * kSelThreads + tid;
-      int bin = 256;
+      const int x = it * NT + tid;
+      int bin = -1;
       if (x < NC) {
         const uint32_t key = keys[x];
-        if ((key & pmask) == prefix) bin = (key >> shift) & 255;
+        if ((key & pmask) == prefix) bin = static_cast<int>((key >> shift) & (nb - 1));
       }
       const unsigned same = __match_any_sync(0xffffffffu, bin);
-      if (bin < 256 && (__ffs(same) - 1) == lane) atomicAdd(&my_hist[bin], __popc(same));
+      if (bin >= 0 && (__ffs(same) - 1) == lane) atomicAdd(&my_hist[bin], __popc(same));
     }
     __syncthreads();
-    if (tid < 256) {
-      int total = 0;
+    if (kSub > 1) {
+      for (int i = tid; i < nb; i += NT) {
+        int t = 0;
 #pragma unroll
-      for (int h = 0; h < kSubHists; ++h) total += sub_hist[h][tid];
-      hist[tid] = total;
-    }
-    __syncthreads();
-    if (tid < 32) {
-      // lane L looks at bins 255-8L .. 248-8L (descending)
-      int cnt[8], loc = 0;
-#pragma unroll
-      for (int e8 = 0; e8 < 8; ++e8) {
-        cnt[e8] = hist[255 - 8 * tid - e8];
-        loc += cnt[e8];
+        for (int h = 0; h < kSub; ++h) t += hist[h][i];
+        hist[0][i] = t;
       }
+      __syncthreads();
+    }
+    if (warp == 0) {
+      // lane L looks at bins nb-1-L*per .. nb-per-L*per (descending)
+      constexpr int per = nb / 32;
+      int loc = 0;
+#pragma unroll
+      for (int e8 = 0; e8 < per; ++e8) loc += hist[0][nb - 1 - lane * per - e8];
       int inc = loc;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (tid >= o) inc += y;
+        if (lane >= o) inc += y;
       }
       int run = inc - loc;  // keys in higher bins than this lane's
-#pragma unroll
-      for (int e8 = 0; e8 < 8; ++e8) {
-        if (run < k && run + cnt[e8] >= k) {
-          sel_bin = 255 - 8 * tid - e8;
-          sel_above = run;
+      if (run < k && run + loc >= k) {
+        for (int e8 = 0; e8 < per; ++e8) {
+          const int bin = nb - 1 - lane * per - e8;
+          const int cnt = hist[0][bin];
+          if (run + cnt >= k) {
+            sel_bin = bin;
+            sel_above = run;
+            break;
+          }
+          run += cnt;
         }
-        run += cnt[e8];
       }
     }
     __syncthreads();
     prefix |= static_cast<uint32_t>(sel_bin) << shift;
-    pmask |= 0xFFu << shift;
+    pmask |= static_cast<uint32_t>(nb - 1) << shift;
     k -= sel_above;
     __syncthreads();
   }
   const uint32_t T = prefix;  // C-th largest key; keep the first k keys equal to T
 
-  // 3. ordered pass over contiguous ranges: rank the T-keys, count free slots
-  //    and kept new tokens
-  const int per = (NC + kSelThreads - 1) / kSelThreads;
+  // 3. ordered pass over contiguous ranges: rank the T-keys by index, then
+  //    count freed old slots and kept new tokens (one packed scan)
+  const int per = (NC + NT - 1) / NT;
   const int lo = min(NC, tid * per), hi = min(NC, lo + per);
   int n_eq = 0;
   for (int x = lo; x < hi; ++x) n_eq += (keys[x] == T);
   int tot;
-  int eq_before = block_excl_scan(n_eq, warp_sums, &tot);
+  int eq_before = block_excl_scan<NT>(n_eq, warp_sums, &tot);
   int free_old = 0, n_new = 0;
   for (int x = lo; x < hi; ++x) {
     const uint32_t key = keys[x];
@@ -245,23 +254,23 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
     else n_new += kept;
     keys[x] = kept ? 1u : 0u;  // from here on: kept flag
   }
-  // empty slots n .. C-1 are free too; give them to the threads in order
+  // counts and totals stay below 2^16 (candidates <= kMaxCandidates)
+  int pk_tot;
+  const int pk_before = block_excl_scan<NT>(free_old | (n_new << 16), warp_sums, &pk_tot);
+  const int fo_before = pk_before & 0xFFFF, nw_before = pk_before >> 16;
+  const int tot_free_old = pk_tot & 0xFFFF, tot_new = pk_tot >> 16;
+  // empty slots n .. C-1 are free too: thread t takes a fixed share, in order
   const int empty = C - n;
-  const int e_per = (empty + kSelThreads - 1) / kSelThreads;
+  const int e_per = (empty + NT - 1) / NT;
   const int e_lo = n + min(empty, tid * e_per), e_hi = n + min(empty, (tid + 1) * e_per);
-  // free slots are ordered: evicted slots (< n) of threads 0..1023, then the
-  // empty slots (>= n) of threads 0..1023; scan the two parts separately
-  int tot_free_old, tot_empty, tot_new;
-  const int fo_before = block_excl_scan(free_old, warp_sums, &tot_free_old);
-  const int em_before = block_excl_scan(e_hi - e_lo, warp_sums, &tot_empty);
-  const int nw_before = block_excl_scan(n_new, warp_sums, &tot_new);
-  if (tot_free_old + tot_empty != tot_new) {
+  if (tot_free_old + empty != tot_new) {
     if (tid == 0) {
       atomicOr(e.state + 2, kDevErrPlan);
       e.plan_count[bg] = 0;
     }
     return;
   }
+  // free slots in order: evicted old slots (< n) first, then the empty ones
   int fo = fo_before, nw = nw_before;
   for (int x = lo; x < hi; ++x) {
     if (x < n) {
@@ -270,24 +279,24 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
       toks[nw++] = x - n;
     }
   }
-  int em = tot_free_old + em_before;
+  int em = tot_free_old + (e_lo - n);
   for (int s = e_lo; s < e_hi; ++s) slots[em++] = s;
   __syncthreads();
   // 4. scores and positions of the placed tokens, then their K/V rows
-  for (int q = tid; q < tot_new; q += kSelThreads) {
+  for (int q = tid; q < tot_new; q += NT) {
     const int s = slots[q], i = toks[q];
     score[s] = cs[C + i];
     pos[s] = e.t0 + i;
   }
   if (tid == 0) e.plan_count[bg] = tot_new;
-  // K/V rows: warp w moves rows w, w + 32, ...; lane L first fetches the
+  // K/V rows: warp w moves rows w, w + NW, ...; lane L first fetches the
   // (slot, token) of the warp's L-th row, so that the copies do not wait on
   // one another's plan reads
-  for (int q0 = warp; q0 < tot_new; q0 += kSelWarps * 32) {
-    const int q = q0 + lane * kSelWarps;
+  for (int q0 = warp; q0 < tot_new; q0 += NW * 32) {
+    const int q = q0 + lane * NW;
     const int my_slot = q < tot_new ? slots[q] : 0;
     const int my_tok = q < tot_new ? toks[q] : 0;
-    const int rows = min(32, (tot_new - q0 + kSelWarps - 1) / kSelWarps);
+    const int rows = min(32, (tot_new - q0 + NW - 1) / NW);
 #pragma unroll 4
     for (int r = 0; r < rows; ++r) {
       const int sl = __shfl_sync(0xffffffffu, my_slot, r);
@@ -297,17 +306,19 @@ __global__ void __launch_bounds__(kSelThreads, 1) h2o_select(const EvictParams e
   }
 }
 
-cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st) {
+template <int NT>
+static cudaError_t launch_select(const EvictParams& e, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(e.n + e.nq) * sizeof(uint32_t);
   static int attr_bits[2] = {0, 0};
-  if (!smem_attr_done(reinterpret_cast<const void*>(h2o_select), attr_bits)) {
-    cudaError_t err = cudaFuncSetAttribute(h2o_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (!smem_attr_done(reinterpret_cast<const void*>(h2o_select<NT>), attr_bits)) {
+    cudaError_t err = cudaFuncSetAttribute(h2o_select<NT>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            kMaxCandidates * 4);
     if (err != cudaSuccess) return err;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(e.B * e.Hkv);
-  cfg.blockDim = dim3(kSelThreads);
+  cfg.blockDim = dim3(NT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -315,8 +326,15 @@ cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, h2o_select<NT>, e);
+}
+
+cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st) {
   (void)max_chunk;
-  return cudaLaunchKernelEx(&cfg, h2o_select, e);
+  // few (cache, KV head) units: one large CTA each, to cut the latency of
+  // each selection; many units: smaller CTAs, several per SM
+  if (e.B * e.Hkv >= 2 * 148) return launch_select<256>(e, st);
+  return launch_select<1024>(e, st);
 }
 
 }  // namespace h2o

@@ -28,6 +28,8 @@ CASES = [
     (1, 8, 128, 8192, 8192, 1024, 256, None, torch.bfloat16),  # full-size shape
     (1, 2, 64, 256, 256, 64, 0, None, torch.float32),    # fp32 cache
     (4, 2, 64, 33, 20, 20, 5, 3, torch.float32),         # tiny, odd sizes
+    (40, 8, 64, 96, 96, 32, 8, 3, torch.bfloat16),       # 320 units: the many-cache variant
+    (40, 8, 64, 300, 250, 100, 120, None, torch.bfloat16),  # many units, partial fill, W > nq
 ]
 
 
