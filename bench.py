@@ -320,26 +320,35 @@ def run_ours(args, world, rank, local):
     tokens = sum_over_ranks(K * wl.batch * wl.chunk, world)
     value = tokens / (total_ms / 1e3)
 
-    # ---- e2e: the same step through the host-buffer entry point (pinned memory)
+    # ---- e2e: K steps through the host-buffer entry point (pinned memory).
+    # Each call uploads its chunk, runs the step and downloads O; the library
+    # overlaps a call's copies with its neighbours' kernels.  One region spans
+    # all K calls, from the first upload to the last download (joined onto the
+    # stream before the end event), and includes the L2 flush before each step.
     chunk_bytes = sum(t.numel() * t.element_size() for t in chunks[0])
-    n_e2e = max(1, min(K, 8, int(2e9 // chunk_bytes)))  # bounded pinned host memory
-    hq = [tuple(t.cpu().pin_memory() for t in chunks[W + (k % K)]) for k in range(n_e2e)]
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    e2e_s = [torch.cuda.Event(enable_timing=True) for _ in hq]
-    e2e_e = [torch.cuda.Event(enable_timing=True) for _ in hq]
+    n_host = max(1, min(K, 8, int(2e9 // chunk_bytes)))  # bounded pinned host memory
+    hq = [tuple(t.cpu().pin_memory() for t in chunks[W + k]) for k in range(n_host)]
+    hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    cache.step_host(*hq[0], hout[0])                   # creates the copy streams
+    torch.cuda.synchronize(dev)
+    e2e_s = torch.cuda.Event(enable_timing=True)
+    e2e_e = torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
-    for k, (q, kn, vn) in enumerate(hq):
+    e2e_s.record(stream)
+    for k in range(K):
         flush.zero_()
-        e2e_s[k].record(stream)
-        cache.step_host(q, kn, vn, hout)
-        e2e_e[k].record(stream)
+        cache.step_host(*hq[k % n_host], hout[k % 2], join=False)
+    cache.host_join(stream)
+    e2e_e.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
-    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e2e_s, e2e_e)), world)
-    e2e_tokens = sum_over_ranks(len(hq) * wl.batch * wl.chunk, world)
+    if cache.check() != 0:
+        raise SystemExit("device error during the host-buffer steps")
+    e2e_ms = max_over_ranks(e2e_s.elapsed_time(e2e_e), world)
+    e2e_tokens = sum_over_ranks(K * wl.batch * wl.chunk, world)
     h2d = sum(t.numel() * t.element_size() for t in hq[0])
-    d2h = hout.numel() * hout.element_size()
+    d2h = hout[0].numel() * hout[0].element_size()
 
     # ---- roofline of the dominant kernel
     peaks, peaks_kind = load_peaks()
@@ -399,7 +408,8 @@ def run_ours(args, world, rank, local):
         "roofline": roof,
         "e2e": {"value": round(e2e_tokens / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                "path": "h2o_chunk_step_host, pinned host buffers"},
+                "path": "h2o_chunk_step_host, pinned host buffers, copies overlapped with "
+                        "neighbouring steps, L2 flush inside the region"},
         "gpu_launches": int(launches),
         "clocks": clocks.summary(),
     }

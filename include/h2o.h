@@ -48,7 +48,8 @@
  *     that expired, an inconsistent eviction plan) are latched in state[2]
  *     and returned by h2o_cache_check().
  *   - All memory is owned by the caller; the library allocates nothing on
- *     the device.  h2o_cache_destroy() frees only the host handle.
+ *     the device.  h2o_cache_destroy() frees the host handle and the copy
+ *     streams and events that h2o_chunk_step_host creates on first use.
  *   - All caches of a handle advance together (one n_q per call).  A handle
  *     must not be used from two host threads at once.
  *   - Supported: head_dim 64 or 128; dtype BF16 (tensor-core path) or F32
@@ -139,14 +140,29 @@ H2O_API h2o_status h2o_chunk_step(h2o_cache* c, const void* q, const void* k_new
                           const void* v_new, int32_t n_q, void* out,
                           float* colsum_out, void* stream);
 
-/* Same step with HOST buffers (pinned memory recommended): the inputs are
- * copied into the workspace's staging area, the step runs, and out (and
- * colsum_out, may be NULL) are copied back, all on `stream`.  The host
- * buffers must stay untouched until the stream reaches this point. */
+/* Same step with HOST buffers (pinned memory recommended).  The inputs are
+ * uploaded into one of two staging sets of the workspace (alternate calls
+ * use alternate sets), the step runs on `stream`, and out is downloaded
+ * back.  The uploads and downloads run on two streams the cache owns, one
+ * per direction, ordered with `stream` by events, so one call's copies
+ * overlap the kernels of the calls before and after it.
+ *   - The input host buffers must stay untouched until `stream` has passed
+ *     this call's step (the step waits for the upload).
+ *   - out_host is complete once h2o_cache_host_join has been called on a
+ *     stream and that stream has passed the join; until then it may still
+ *     be in transfer.
+ *   - colsum_out_host (may be NULL) is copied on `stream` itself, after the
+ *     step.
+ * The workspace holds both staging sets (h2o_required_bytes counts them). */
 H2O_API h2o_status h2o_chunk_step_host(h2o_cache* c, const void* q_host,
                                const void* k_new_host, const void* v_new_host,
                                int32_t n_q, void* out_host,
                                float* colsum_out_host, void* stream);
+
+/* Makes `stream` wait until every download issued by h2o_chunk_step_host
+ * on this cache so far has landed in host memory (no-op before the first
+ * host call).  Does not block the host. */
+H2O_API h2o_status h2o_cache_host_join(h2o_cache* c, void* stream);
 
 /* Steps 1-2 only: out and colsum_out (both device; colsum_out may be NULL)
  * for the current cache contents.  The cache state does not change. */
@@ -230,7 +246,9 @@ H2O_API h2o_status h2o_selftest_exp2(const float* x, float* y_poly, float* y_lib
 H2O_API h2o_status h2o_selftest_wait_timeout(int32_t* err_word, uint32_t limit_us,
                                              void* stream);
 
-/* Frees the host handle only. */
+/* Waits for the copies h2o_chunk_step_host still has in flight, then frees
+ * the host handle and its copy streams and events.  Device buffers stay the
+ * caller's. */
 H2O_API void h2o_cache_destroy(h2o_cache* c);
 
 H2O_API const char* h2o_status_string(h2o_status s);

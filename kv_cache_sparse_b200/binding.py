@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "H2O_OK", 1: "H2O_ERR_INVALID_ARG", 2: "H2O_ERR_SHAPE", 3: "H
                 4: "H2O_ERR_ALIGN", 5: "H2O_ERR_CUDA", 6: "H2O_ERR_TIMEOUT", 7: "H2O_ERR_STATE"}
 
 EXPORTED = ["h2o_required_bytes", "h2o_cache_create", "h2o_chunk_step", "h2o_chunk_step_host",
-            "h2o_attention", "h2o_evict", "h2o_cache_read", "h2o_cache_write",
+            "h2o_cache_host_join", "h2o_attention", "h2o_evict", "h2o_cache_read", "h2o_cache_write",
             "h2o_cache_check", "h2o_cache_info", "h2o_cache_set_timing", "h2o_cache_kernel_ms",
             "h2o_cache_destroy", "h2o_status_string"]
 
@@ -206,13 +206,23 @@ class H2OCache:
             _stream(stream)))
         return (out, colsum) if return_colsum else out
 
-    def step_host(self, q, k_new, v_new, out, colsum=None, stream=None):
-        """The step on HOST (ideally pinned) tensors; copies run on the stream."""
+    def step_host(self, q, k_new, v_new, out, colsum=None, stream=None, join=True):
+        """The step on HOST (ideally pinned) tensors.  Uploads and downloads
+        run on the cache's own copy streams and overlap neighbouring steps;
+        with join=True the stream then waits for this step's download, so
+        `out` is complete once the stream is synchronised.  With join=False
+        call host_join() before reading `out`."""
         n_q = q.shape[1]
         _check("h2o_chunk_step_host", lib().h2o_chunk_step_host(
             self._h, _ptr(q), _ptr(k_new), _ptr(v_new), n_q, _ptr(out), _ptr(colsum),
             _stream(stream)))
+        if join:
+            self.host_join(stream)
         return out
+
+    def host_join(self, stream=None):
+        """Makes the stream wait for every download step_host has issued."""
+        _check("h2o_cache_host_join", lib().h2o_cache_host_join(self._h, _stream(stream)))
 
     def attention(self, q, k_new, v_new, stream=None):
         n_q = self._check_inputs(q, k_new, v_new)

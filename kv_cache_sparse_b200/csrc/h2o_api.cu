@@ -33,10 +33,20 @@ struct h2o_cache {
   int* plan_slots = nullptr;
   int* plan_tokens = nullptr;
   int* plan_count = nullptr;
-  uint8_t* stage_q = nullptr;
-  uint8_t* stage_kn = nullptr;
-  uint8_t* stage_vn = nullptr;
-  uint8_t* stage_out = nullptr;
+  // h2o_chunk_step_host: two staging sets, used by alternate calls, so the
+  // copies of one call overlap the kernels of its neighbours.  The copies run
+  // on two internal streams (one per direction); events order them with the
+  // caller's stream.
+  int device = 0;
+  uint8_t* stage_q[2] = {nullptr, nullptr};
+  uint8_t* stage_kn[2] = {nullptr, nullptr};
+  uint8_t* stage_vn[2] = {nullptr, nullptr};
+  uint8_t* stage_out[2] = {nullptr, nullptr};
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t ev_in[2] = {nullptr, nullptr};    // inputs of the set uploaded
+  cudaEvent_t ev_step[2] = {nullptr, nullptr};  // step that read the set done
+  cudaEvent_t ev_out[2] = {nullptr, nullptr};   // output of the set downloaded
+  uint64_t host_calls = 0;
   // per-kernel timing (h2o_cache_set_timing)
   bool timing = false;
   cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
@@ -52,7 +62,7 @@ size_t esize_of(h2o_dtype t) { return t == H2O_BF16 ? 2 : 4; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct Layout {
-  size_t lse, colsum, slots, tokens, count, sq, skn, svn, sout, total;
+  size_t lse, colsum, slots, tokens, count, sq[2], skn[2], svn[2], sout[2], total;
   int nq_pad, colsum_ld;
 };
 
@@ -74,10 +84,12 @@ Layout workspace_layout(const h2o_config& c) {
   L.tokens = take(BHkv * c.max_chunk * 4);
   L.count = take(BHkv * 4);
   const size_t rows = static_cast<size_t>(c.batch) * c.max_chunk * c.head_dim * e;
-  L.sq = take(rows * c.n_q_heads);
-  L.skn = take(rows * c.n_kv_heads);
-  L.svn = take(rows * c.n_kv_heads);
-  L.sout = take(rows * c.n_q_heads);
+  for (int i = 0; i < 2; ++i) {
+    L.sq[i] = take(rows * c.n_q_heads);
+    L.skn[i] = take(rows * c.n_kv_heads);
+    L.svn[i] = take(rows * c.n_kv_heads);
+    L.sout[i] = take(rows * c.n_q_heads);
+  }
   L.total = off;
   return L;
 }
@@ -269,6 +281,24 @@ h2o_status copy_colsum(h2o_cache* c, float* dst, int nq, cudaStream_t st) {
                                        cudaMemcpyDefault, st));
 }
 
+// Creates the two copy streams and the six events of h2o_chunk_step_host on
+// the cache's device, on first use.
+h2o_status host_streams(h2o_cache* c) {
+  if (c->h2d) return H2O_OK;
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return H2O_ERR_CUDA;
+  if (cur != c->device && cudaSetDevice(c->device) != cudaSuccess) return H2O_ERR_CUDA;
+  cudaError_t e = cudaStreamCreateWithFlags(&c->h2d, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->d2h, cudaStreamNonBlocking);
+  for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+    e = cudaEventCreateWithFlags(&c->ev_in[i], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_step[i], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_out[i], cudaEventDisableTiming);
+  }
+  if (cur != c->device) cudaSetDevice(cur);
+  return cuda_status(e);
+}
+
 }  // namespace
 
 namespace h2o {
@@ -324,10 +354,17 @@ h2o_status h2o_cache_create(const h2o_config* cfg, const h2o_buffers* bufs, void
   c->plan_slots = reinterpret_cast<int*>(ws + L.slots);
   c->plan_tokens = reinterpret_cast<int*>(ws + L.tokens);
   c->plan_count = reinterpret_cast<int*>(ws + L.count);
-  c->stage_q = ws + L.sq;
-  c->stage_kn = ws + L.skn;
-  c->stage_vn = ws + L.svn;
-  c->stage_out = ws + L.sout;
+  for (int i = 0; i < 2; ++i) {
+    c->stage_q[i] = ws + L.sq[i];
+    c->stage_kn[i] = ws + L.skn[i];
+    c->stage_vn[i] = ws + L.svn[i];
+    c->stage_out[i] = ws + L.sout[i];
+  }
+  cudaPointerAttributes pa;
+  if (cudaPointerGetAttributes(&pa, bufs->workspace) == cudaSuccess && pa.device >= 0)
+    c->device = pa.device;
+  else
+    cudaGetDevice(&c->device);
   h2o_sizes sz;
   h2o_required_bytes(cfg, &sz);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -382,18 +419,43 @@ h2o_status h2o_chunk_step_host(h2o_cache* c, const void* q_host, const void* k_n
   if (n_q < 0 || n_q > c->cfg.max_chunk) return H2O_ERR_INVALID_ARG;
   if (n_q == 0) return H2O_OK;
   if (!q_host || !k_new_host || !v_new_host || !out_host) return H2O_ERR_INVALID_ARG;
+  if (host_streams(c) != H2O_OK) return H2O_ERR_CUDA;
   const h2o_config& g = c->cfg;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t rows = static_cast<size_t>(g.batch) * n_q * g.head_dim * esize_of(g.dtype);
   const size_t bq = rows * g.n_q_heads, bkv = rows * g.n_kv_heads;
-  cudaError_t e = cudaMemcpyAsync(c->stage_q, q_host, bq, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(c->stage_kn, k_new_host, bkv, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(c->stage_vn, v_new_host, bkv, cudaMemcpyHostToDevice, st);
+  const int x = static_cast<int>(c->host_calls & 1);
+  // upload into set x once the step two calls back has finished reading it
+  cudaError_t e = cudaStreamWaitEvent(c->h2d, c->ev_step[x], 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->stage_q[x], q_host, bq, cudaMemcpyHostToDevice, c->h2d);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->stage_kn[x], k_new_host, bkv, cudaMemcpyHostToDevice, c->h2d);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->stage_vn[x], v_new_host, bkv, cudaMemcpyHostToDevice, c->h2d);
+  if (e == cudaSuccess) e = cudaEventRecord(c->ev_in[x], c->h2d);
+  // the step waits for its inputs and for the download that last read out[x]
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, c->ev_in[x], 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, c->ev_out[x], 0);
   if (e != cudaSuccess) return H2O_ERR_CUDA;
-  h2o_status s = h2o_chunk_step(c, c->stage_q, c->stage_kn, c->stage_vn, n_q, c->stage_out,
-                                colsum_out_host, stream);
+  h2o_status s = h2o_chunk_step(c, c->stage_q[x], c->stage_kn[x], c->stage_vn[x], n_q,
+                                c->stage_out[x], colsum_out_host, stream);
   if (s != H2O_OK) return s;
-  return cuda_status(cudaMemcpyAsync(out_host, c->stage_out, bq, cudaMemcpyDeviceToHost, st));
+  e = cudaEventRecord(c->ev_step[x], st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(c->d2h, c->ev_step[x], 0);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(out_host, c->stage_out[x], bq, cudaMemcpyDeviceToHost, c->d2h);
+  if (e == cudaSuccess) e = cudaEventRecord(c->ev_out[x], c->d2h);
+  if (e != cudaSuccess) return H2O_ERR_CUDA;
+  ++c->host_calls;
+  return H2O_OK;
+}
+
+h2o_status h2o_cache_host_join(h2o_cache* c, void* stream) {
+  if (!c) return H2O_ERR_INVALID_ARG;
+  if (c->host_calls == 0) return H2O_OK;
+  // the download stream is in order: its latest event covers every earlier call
+  const int last = static_cast<int>((c->host_calls - 1) & 1);
+  return cuda_status(cudaStreamWaitEvent(static_cast<cudaStream_t>(stream), c->ev_out[last], 0));
 }
 
 h2o_status h2o_cache_read(const h2o_cache* c, void* k, void* v, float* scores, int32_t* pos,
@@ -495,6 +557,16 @@ void h2o_cache_destroy(h2o_cache* c) {
   if (!c) return;
   for (int i = 0; i < 5; ++i)
     if (c->ev[i]) cudaEventDestroy(c->ev[i]);
+  // copies still in flight write caller memory: let them finish first
+  if (c->h2d) cudaStreamSynchronize(c->h2d);
+  if (c->d2h) cudaStreamSynchronize(c->d2h);
+  for (int i = 0; i < 2; ++i) {
+    if (c->ev_in[i]) cudaEventDestroy(c->ev_in[i]);
+    if (c->ev_step[i]) cudaEventDestroy(c->ev_step[i]);
+    if (c->ev_out[i]) cudaEventDestroy(c->ev_out[i]);
+  }
+  if (c->h2d) cudaStreamDestroy(c->h2d);
+  if (c->d2h) cudaStreamDestroy(c->d2h);
   delete c;
 }
 

@@ -105,6 +105,35 @@ def test_host_entry_point_matches_device_entry_point():
         assert torch.equal(gh.bits(sa[key]), gh.bits(sb[key])), key
 
 
+def test_pipelined_host_steps_match_device_steps():
+    """Several host-buffer steps in flight at once (no join between them, a
+    side stream, chunk sizes that change between calls): after one join every
+    output and the final cache equal the device-buffer path bit for bit."""
+    wl = SMALL_QWEN.scaled(name="pipelined", capacity=300, window=40, chunk=100, seq_len=700)
+    src = ChunkSource(wl, seed=3)
+    shape = shape_for(wl)
+    a = binding.H2OCache(shape)
+    b = binding.H2OCache(shape)
+    sizes = (100, 37, 100, 1, 64, 100, 99)
+    chunks = [src.chunk(c, n_q=nq) for c, nq in enumerate(sizes)]
+    ref = [a.step(*(t.cuda() for t in ch)) for ch in chunks]
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    host_in = [tuple(t.pin_memory() for t in ch) for ch in chunks]
+    outs = [torch.full(ch[0].shape, float("nan"), dtype=ch[0].dtype).pin_memory()
+            for ch in chunks]
+    with torch.cuda.stream(side):
+        for (q, kn, vn), out in zip(host_in, outs):
+            b.step_host(q, kn, vn, out, stream=side, join=False)
+        b.host_join(side)
+    side.synchronize()
+    for r, out in zip(ref, outs):
+        assert torch.equal(gh.bits(r), gh.bits(out))
+    sa, sb = a.read(), b.read()
+    for key in ("k", "v", "scores", "pos"):
+        assert torch.equal(gh.bits(sa[key]), gh.bits(sb[key])), key
+
+
 def test_checkpoint_resume_bit_exact():
     wl = SMALL_QWEN
     src = ChunkSource(wl, seed=2)
