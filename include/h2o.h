@@ -232,12 +232,6 @@ H2O_API h2o_status h2o_attention_static_scratch(const h2o_config* cfg, const voi
                                                 int32_t n_q, void* out, float* colsum_out,
                                                 void* stream);
 
-/* Diagnostic: for x[i] <= 0 (device arrays of n floats) writes the
- * polynomial base-2 exponential the kernels use for part of their
- * probabilities (y_poly) and CUDA's exp2f (y_lib), for accuracy tests. */
-H2O_API h2o_status h2o_selftest_exp2(const float* x, float* y_poly, float* y_lib, int32_t n,
-                                     void* stream);
-
 /* Diagnostic of the failure path: one warp waits, with the same bounded
  * wait the kernels use, on a barrier nothing completes.  After limit_us
  * (1 .. 2,000,000) the wait gives up, ORs the timeout bit (1) into

@@ -14,12 +14,15 @@
 // 128 queries of one head; the sum order is fixed, so results are
 // deterministic (no atomics).
 //   warp 0      TMA producer: the key tile once, then Q tiles + their lse2
-//   warp 1      TMEM allocation; one thread issues the tcgen05.mma into a
-//               ring of four 128-column S buffers
-//   warps 2..5  row tiles 0, 2, 4, ...; warps 6..9 row tiles 1, 3, 5, ...:
-//               one thread per key, all 128 query columns of its tiles.  The
-//               two warpgroups work out of phase (each one's next S is ready
-//               while it sums), so the exponential units stay busy.
+//   warp 1      TMEM allocation; one thread issues the tcgen05.mma, S of row
+//               tile u into the 128-column TMEM buffer u % 4
+//   warps 2..17 four summing warpgroups; group g takes row tiles u = g, g+4,
+//               g+8, ...: one thread per key, all 128 query columns of the
+//               tile, read from TMEM in two halves of 64.  A group frees its
+//               S buffer as soon as the second half is in registers, so the
+//               MMA of its next tile runs while it sums; with four groups the
+//               waits and loads of one are covered by the others, and the
+//               exponential units stay busy.
 #include "attn.h"
 #include "sm100.cuh"
 
@@ -29,9 +32,10 @@ template <int D>
 struct ColLayout {
   static constexpr int kRegions = D / 64;
   static constexpr int kTileBytes = 128 * D * 2;
-  static constexpr int kQStages = 4;    // Q tiles, released when their MMA completes
-  static constexpr int kLseStages = 8;  // row statistics, released by the summing group
-  static constexpr int kSBufs = 4;      // TMEM S buffers (two per summing group)
+  static constexpr int kGroups = 4;                // summing warpgroups
+  static constexpr int kQStages = 4;               // Q tiles, released when their MMA completes
+  static constexpr int kLseStages = 2 * kGroups;   // row statistics, released by the summing group
+  static constexpr int kSBufs = kGroups;           // TMEM S buffers, one per summing group
   static constexpr int kKOff = 0;
   static constexpr int kQOff = kKOff + kTileBytes;
   static constexpr int kLseOff = kQOff + kQStages * kTileBytes;  // 512 bytes per stage
@@ -40,15 +44,11 @@ struct ColLayout {
   static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kLseStages + 2 * kSBufs + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kRedOff = kMiscOff + 16;
-  static constexpr int kBytes = kRedOff + 128 * 4;
+  static constexpr int kBytes = kRedOff + (kGroups - 1) * 128 * 4;
   static constexpr int kAlloc = kBytes + 1024;
   static constexpr int kTmemCols = 512;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 64 + 128 * kGroups;
 };
-
-// Every fourth probability is computed with the FMA-pipe polynomial, the rest
-// with the MUFU ex2 instruction, so that both units share the work.
-constexpr int kPolyEvery = 4;
 
 template <bool kDiag>
 __device__ __forceinline__ void sum_tile(const uint32_t (&v0)[32], const uint32_t (&v1)[32],
@@ -67,8 +67,7 @@ __device__ __forceinline__ void sum_tile(const uint32_t (&v0)[32], const uint32_
     float x0, x1, x2, x3;
     ffma2(x0, x1, __uint_as_float(s0), __uint_as_float(s1), c, c, nl.x, nl.y);
     ffma2(x2, x3, __uint_as_float(s2), __uint_as_float(s3), c, c, nl.z, nl.w);
-    float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2);
-    float p3 = (kPolyEvery == 4) ? ex2_poly(x3) : ex2_approx(x3);
+    float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
     if (kDiag) {  // query i0+col sees key j0+row iff row <= col
       p0 = (col >= first_col) ? p0 : 0.f;
       p1 = (col + 1 >= first_col) ? p1 : 0.f;
@@ -81,7 +80,7 @@ __device__ __forceinline__ void sum_tile(const uint32_t (&v0)[32], const uint32_
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(64 + 128 * ColLayout<D>::kGroups, 1)
     attn_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_kc,
                        const __grid_constant__ CUtensorMap tm_kn, const AttnParams p) {
@@ -197,13 +196,13 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, false, false);
-      bool ok = mbar_wait_spin(bar_k, 0, p.err, abort_flag);
+      bool ok = mbar_wait(bar_k, 0, p.err, abort_flag);
       for (int u = 0; u < R && ok; ++u) {
         const int s = u % L::kQStages;
         const int sb = u % L::kSBufs;
-        ok = mbar_wait_spin(bar_q_full0 + 8 * s, (u / L::kQStages) & 1, p.err, abort_flag);
+        ok = mbar_wait(bar_q_full0 + 8 * s, (u / L::kQStages) & 1, p.err, abort_flag);
         if (ok && u >= L::kSBufs)
-          ok = mbar_wait_spin(bar_s_empty0 + 8 * sb, ((u / L::kSBufs) + 1) & 1, p.err, abort_flag);
+          ok = mbar_wait(bar_s_empty0 + 8 * sb, ((u / L::kSBufs) + 1) & 1, p.err, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint32_t qbase = sbase + L::kQOff + s * L::kTileBytes;
@@ -221,46 +220,54 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else {
     const int quad = warp & 3;
-    const int grp = (warp - 2) >> 2;   // row tiles u with u % 2 == grp
+    const int grp = (warp - 2) >> 2;   // row tiles u with u % kGroups == grp
     const int row = quad * 32 + lane;  // key j0 + row
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float c = p.scale_log2;
     float acc = 0.f;
     bool ok = true;
-    for (int u = grp; u < R; u += 2) {
+    for (int u = grp; u < R; u += L::kGroups) {
       const int sl = u % L::kLseStages;
       const int sb = u % L::kSBufs;
       ok = mbar_wait(bar_s_full0 + 8 * sb, (u / L::kSBufs) & 1, p.err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      uint32_t v[4][32];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) tmem_ld32(lane_base + sb * 128 + 32 * k, v[k]);
+      uint32_t v[2][32];
+      tmem_ld32(lane_base + sb * 128, v[0]);
+      tmem_ld32(lane_base + sb * 128 + 32, v[1]);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar_s_empty0 + 8 * sb);
       ok = mbar_wait(bar_l_full0 + 8 * sl, (u / L::kLseStages) & 1, p.err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       const float4* nlse4 = reinterpret_cast<const float4*>(smem + L::kLseOff + sl * 512);
       const int qt = qt_min + u % span;
+      const bool diag = is_chunk && qt == kt;  // query i0+col sees key j0+row iff row <= col
       float part[4] = {0.f, 0.f, 0.f, 0.f};
-      if (is_chunk && qt == kt) {  // diagonal tile: query i0+col sees key j0+row iff row <= col
+      if (diag)
         sum_tile<true>(v[0], v[1], nlse4, c, row, part);
-        sum_tile<true>(v[2], v[3], nlse4 + 16, c, row - 64, part);
-      } else {
+      else
         sum_tile<false>(v[0], v[1], nlse4, c, 0, part);
-        sum_tile<false>(v[2], v[3], nlse4 + 16, c, 0, part);
-      }
+      // second half of the query columns; then the S buffer is free
+      tmem_ld32(lane_base + sb * 128 + 64, v[0]);
+      tmem_ld32(lane_base + sb * 128 + 96, v[1]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar_s_empty0 + 8 * sb);
+      if (diag)
+        sum_tile<true>(v[0], v[1], nlse4 + 16, c, row - 64, part);
+      else
+        sum_tile<false>(v[0], v[1], nlse4 + 16, c, 0, part);
       acc += (part[0] + part[1]) + (part[2] + part[3]);
       mbar_arrive(bar_l_empty0 + 8 * sl);
     }
-    // combine the two groups' sums in a fixed order
-    if (grp == 1) red[row] = acc;
-    named_bar_sync(1, 256);
+    // combine the groups' sums in a fixed order
+    if (grp > 0) red[(grp - 1) * 128 + row] = acc;
+    named_bar_sync(1, 128 * L::kGroups);
     if (grp == 0 && ok) {
-      const float total = acc + red[row];
+      float total = acc;
+#pragma unroll
+      for (int gr = 1; gr < L::kGroups; ++gr) total += red[(gr - 1) * 128 + row];
       const int key = j0 + row;
       if (is_chunk) {
         if (key < p.nq) out[p.C + key] = total;

@@ -1,22 +1,11 @@
-// selftest.cu -- diagnostic entry points:
-//   h2o_selftest_exp2         the kernels' polynomial base-2 exponential next
-//                             to CUDA's exp2f, for accuracy tests;
-//   h2o_selftest_wait_timeout one warp waits, with the kernels' bounded wait,
-//                             on an mbarrier nothing arrives at; the wait gives
-//                             up after the given limit, latches the timeout
-//                             bit and the kernel returns (no trap, no hang).
+// selftest.cu -- diagnostic entry point h2o_selftest_wait_timeout: one warp
+// waits, with the kernels' bounded wait, on an mbarrier nothing arrives at;
+// the wait gives up after the given limit, latches the timeout bit and the
+// kernel returns (no trap, no hang).
 #include "../../include/h2o.h"
 #include "sm100.cuh"
 
 namespace {
-
-__global__ void exp2_compare(const float* x, float* y_poly, float* y_lib, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) {
-    y_poly[i] = h2o::ex2_poly(x[i]);
-    y_lib[i] = exp2f(x[i]);
-  }
-}
 
 __global__ void wait_timeout_probe(int* err, uint64_t limit_ns) {
   __shared__ __align__(8) uint64_t bar;
@@ -39,13 +28,5 @@ extern "C" H2O_API h2o_status h2o_selftest_wait_timeout(int32_t* err_word, uint3
   if (!err_word || limit_us == 0 || limit_us > 2000000) return H2O_ERR_INVALID_ARG;
   wait_timeout_probe<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       err_word, static_cast<uint64_t>(limit_us) * 1000ull);
-  return cudaGetLastError() == cudaSuccess ? H2O_OK : H2O_ERR_CUDA;
-}
-
-extern "C" H2O_API h2o_status h2o_selftest_exp2(const float* x, float* y_poly, float* y_lib,
-                                                int32_t n, void* stream) {
-  if (n < 0 || (n > 0 && (!x || !y_poly || !y_lib))) return H2O_ERR_INVALID_ARG;
-  if (n == 0) return H2O_OK;
-  exp2_compare<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_lib, n);
   return cudaGetLastError() == cudaSuccess ? H2O_OK : H2O_ERR_CUDA;
 }

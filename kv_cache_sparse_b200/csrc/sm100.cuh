@@ -323,26 +323,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x for x <= 0 on the FMA pipe, to take part of the exponentials off the
-// MUFU unit.  Argument reduction after Cody and Waite: r = round(x) (adding
-// 1.5 * 2^23 rounds x to an integer held in the low mantissa bits of t), f =
-// x - r in [-1/2, 1/2] (exact); 2^f is a degree-4 polynomial whose
-// coefficients minimise the maximum relative error on [-1/2, 1/2] (Remez
-// exchange; fitted by kv_cache_sparse_b200/fit_exp2.py: 2.6e-6); 2^r is added
-// to the exponent field.  x is clamped to -125 so that the result stays a
-// normal float; for x < -125 it returns ~2^-125 instead of a smaller value.
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float r = t - 12582912.0f;
-  const float f = x - r;
-  float p = fmaf(0.0095701019080826049f, f, 0.05591786031930443f);
-  p = fmaf(p, f, 0.2402474482794402f);
-  p = fmaf(p, f, 0.6931218147367707f);
-  p = fmaf(p, f, 0.99999926144571449f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Two fp32 operations per instruction (packed f32x2, sm_100):
 // (a0, a1) * (b0, b1) + (c0, c1), and (a0, a1) + (b0, b1), round to nearest.
 __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
