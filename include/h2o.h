@@ -106,7 +106,8 @@ typedef struct {
   size_t pos_bytes;         /* int32 positions                               */
   size_t state_bytes;       /* 4 x int32                                     */
   size_t workspace_bytes;   /* row statistics, summed weights, eviction plan,
-                               and staging for h2o_chunk_step_host           */
+                               the logits and split-KV partials of n_q = 1
+                               calls, and staging for h2o_chunk_step_host    */
 } h2o_sizes;
 
 /* Caller-owned device buffers (sizes from h2o_required_bytes). */
@@ -135,7 +136,9 @@ H2O_API h2o_status h2o_cache_create(const h2o_config* cfg, const h2o_buffers* bu
  * placement) for all caches.  q, k_new, v_new, out: device pointers in the
  * layouts above with 1 <= n_q <= max_chunk (n_q = 0 is a no-op).
  * colsum_out (device, may be NULL) receives the summed weights in the colsum
- * layout.  Advances n and t0. */
+ * layout.  Advances n and t0.  A decode step (n_q = 1, at most 8 query heads
+ * per KV head) runs as two launches (split-KV attention; merge, summed
+ * weights and the single-token eviction), other steps as three. */
 H2O_API h2o_status h2o_chunk_step(h2o_cache* c, const void* q, const void* k_new,
                           const void* v_new, int32_t n_q, void* out,
                           float* colsum_out, void* stream);

@@ -31,6 +31,11 @@ cudaError_t launch_attn_f32(int head_dim, const float* q, const float* kc, const
                             const float* kn, const float* vn, const AttnParams& p,
                             cudaStream_t st);
 
+// Decode step (n_q = 1, G <= kDecodeMaxG): split-KV partials, then the merge,
+// summed weights and (if p.evict) the single-token eviction.  esize 2 (bf16)
+// or 4 (float), head_dim 64 or 128.
+cudaError_t launch_decode(const DecodeParams& p, int esize, int head_dim, cudaStream_t st);
+
 // K3 (with the K/V scatter fused): score update, selection, placement.
 cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st);
 

@@ -64,4 +64,31 @@ struct EvictParams {
   int* state;               // [4]: n, t0, err, reserved
 };
 
+// ---------------------------------------------------------------- decode (n_q = 1)
+
+constexpr int kDecodeChunk = 256;  // keys per split-KV partial
+constexpr int kDecodeMaxG = 8;     // largest GQA group the decode kernels take
+
+struct DecodeParams {
+  int B, Hkv, G, C;         // caches, KV heads, heads per group, capacity
+  int n, t0, W;             // valid slots, position of the new token, window
+  int n_chunks;             // cdiv(n + 1, kDecodeChunk): key n is the new token
+  int part_ld;              // chunks per (cache, KV head) in part
+  float scale_log2;         // softmax scale * log2(e)
+  const void* q;            // [B, 1, Hq, d]
+  const void* k_new;        // [B, 1, Hkv, d]
+  const void* v_new;
+  void* k_cache;            // [B, Hkv, C, d]
+  void* v_cache;
+  void* out;                // [B, 1, Hq, d]
+  float* logits;            // [B*Hkv, G, C + 1]: x = scale*log2(e)*<q, k>, key n = new token
+  float* part;              // [B*Hkv, part_ld, G, d + 2]: unnormalised O, max, sum per chunk
+  float* colsum;            // [B*Hkv, colsum_ld]: slots, zeros up to C, then the new key at C
+  int colsum_ld;
+  float* scores;            // [B, Hkv, C]   (eviction only)
+  int* pos;                 // [B, Hkv, C]
+  int* state;               // [4]: n, t0, err, reserved
+  int evict;                // 1: score update and placement after the attention
+};
+
 }  // namespace h2o

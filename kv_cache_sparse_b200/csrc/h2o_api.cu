@@ -7,7 +7,9 @@
 //   K2 summed attention weights per key     (attn_colsum.cu, tcgen05)
 //   K3 score update + top-C selection + K/V scatter into the freed slots
 //                                           (evict.cu)
-// Float32 caches use the fp32 kernels of attn_f32.cu for K1/K2.
+// Float32 caches use the fp32 kernels of attn_f32.cu for K1/K2.  A call with
+// n_q = 1 (a decode step) runs the two split-KV kernels of decode.cu instead,
+// when the group has at most kDecodeMaxG query heads.
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
@@ -33,6 +35,9 @@ struct h2o_cache {
   int* plan_slots = nullptr;
   int* plan_tokens = nullptr;
   int* plan_count = nullptr;
+  float* dec_logits = nullptr;  // decode: [B*Hkv, G, C + 1]
+  float* dec_part = nullptr;    // decode: [B*Hkv, dec_part_ld, G, d + 2]
+  int dec_part_ld = 0;
   // h2o_chunk_step_host: two staging sets, used by alternate calls, so the
   // copies of one call overlap the kernels of its neighbours.  The copies run
   // on two internal streams (one per direction); events order them with the
@@ -62,8 +67,8 @@ size_t esize_of(h2o_dtype t) { return t == H2O_BF16 ? 2 : 4; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct Layout {
-  size_t lse, colsum, slots, tokens, count, sq[2], skn[2], svn[2], sout[2], total;
-  int nq_pad, colsum_ld;
+  size_t lse, colsum, slots, tokens, count, dlog, dpart, sq[2], skn[2], svn[2], sout[2], total;
+  int nq_pad, colsum_ld, dpart_ld;
 };
 
 Layout workspace_layout(const h2o_config& c) {
@@ -83,6 +88,12 @@ Layout workspace_layout(const h2o_config& c) {
   L.slots = take(BHkv * c.max_chunk * 4);
   L.tokens = take(BHkv * c.max_chunk * 4);
   L.count = take(BHkv * 4);
+  // decode steps (n_q = 1): stored logits and the split-KV partials
+  const size_t G = static_cast<size_t>(c.n_q_heads / c.n_kv_heads);
+  L.dpart_ld = cdiv(c.capacity + 1, kDecodeChunk);
+  const bool dec = G <= static_cast<size_t>(kDecodeMaxG);
+  L.dlog = take(dec ? BHkv * G * (static_cast<size_t>(c.capacity) + 1) * 4 : 0);
+  L.dpart = take(dec ? BHkv * L.dpart_ld * G * (c.head_dim + 2) * 4 : 0);
   const size_t rows = static_cast<size_t>(c.batch) * c.max_chunk * c.head_dim * e;
   for (int i = 0; i < 2; ++i) {
     L.sq[i] = take(rows * c.n_q_heads);
@@ -274,6 +285,57 @@ h2o_status run_evict(h2o_cache* c, const float* colsum, int ld, const void* kn, 
   return H2O_OK;
 }
 
+bool decode_path(const h2o_cache* c, int nq) {
+  return nq == 1 && c->cfg.n_q_heads / c->cfg.n_kv_heads <= kDecodeMaxG;
+}
+
+// The step for one new token per cache (decode.cu): split-KV attention with
+// summed weights into the workspace's colsum, and, if evict, the score update
+// and placement.  Advances n and t0 when evicting.
+h2o_status run_decode(h2o_cache* c, const void* q, const void* kn, const void* vn, void* out,
+                      bool evict, cudaStream_t st) {
+  const h2o_config& g = c->cfg;
+  DecodeParams d;
+  d.B = g.batch;
+  d.Hkv = g.n_kv_heads;
+  d.G = g.n_q_heads / g.n_kv_heads;
+  d.C = g.capacity;
+  d.n = c->n;
+  d.t0 = c->t0;
+  d.W = g.recent_window;
+  d.n_chunks = cdiv(c->n + 1, kDecodeChunk);
+  d.part_ld = c->dec_part_ld;
+  const float scale = g.softmax_scale > 0.f ? g.softmax_scale : 1.f / sqrtf((float)g.head_dim);
+  d.scale_log2 = scale * 1.4426950408889634f;
+  d.q = q;
+  d.k_new = kn;
+  d.v_new = vn;
+  d.k_cache = c->buf.k;
+  d.v_cache = c->buf.v;
+  d.out = out;
+  d.logits = c->dec_logits;
+  d.part = c->dec_part;
+  d.colsum = c->colsum;
+  d.colsum_ld = c->colsum_ld;
+  d.scores = c->buf.scores;
+  d.pos = c->buf.pos;
+  d.state = c->buf.state;
+  d.evict = evict ? 1 : 0;
+  for (int i = 0; i < 5; ++i) c->ev_used[i] = false;
+  mark(c, 0, st);
+  if (launch_decode(d, static_cast<int>(esize_of(g.dtype)), g.head_dim, st) != cudaSuccess)
+    return H2O_ERR_CUDA;
+  c->launches += 2;
+  mark(c, 1, st);  // both kernels are reported as the first part
+  mark(c, 2, st);
+  mark(c, 3, st);
+  if (evict) {
+    c->n = c->n + 1 < g.capacity ? c->n + 1 : g.capacity;
+    c->t0 += 1;
+  }
+  return H2O_OK;
+}
+
 h2o_status copy_colsum(h2o_cache* c, float* dst, int nq, cudaStream_t st) {
   const size_t w = (static_cast<size_t>(c->cfg.capacity) + nq) * sizeof(float);
   return cuda_status(cudaMemcpy2DAsync(dst, w, c->colsum, c->colsum_ld * sizeof(float), w,
@@ -354,6 +416,9 @@ h2o_status h2o_cache_create(const h2o_config* cfg, const h2o_buffers* bufs, void
   c->plan_slots = reinterpret_cast<int*>(ws + L.slots);
   c->plan_tokens = reinterpret_cast<int*>(ws + L.tokens);
   c->plan_count = reinterpret_cast<int*>(ws + L.count);
+  c->dec_logits = reinterpret_cast<float*>(ws + L.dlog);
+  c->dec_part = reinterpret_cast<float*>(ws + L.dpart);
+  c->dec_part_ld = L.dpart_ld;
   for (int i = 0; i < 2; ++i) {
     c->stage_q[i] = ws + L.sq[i];
     c->stage_kn[i] = ws + L.skn[i];
@@ -386,7 +451,8 @@ h2o_status h2o_attention(h2o_cache* c, const void* q, const void* k_new, const v
   h2o_status s = check_step_args(c, q, k_new, v_new, n_q, out);
   if (s != H2O_OK || n_q == 0) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = run_attention(c, q, k_new, v_new, n_q, out, st);
+  s = decode_path(c, n_q) ? run_decode(c, q, k_new, v_new, out, false, st)
+                          : run_attention(c, q, k_new, v_new, n_q, out, st);
   if (s == H2O_OK && colsum_out) s = copy_colsum(c, colsum_out, n_q, st);
   return s;
 }
@@ -406,6 +472,13 @@ h2o_status h2o_chunk_step(h2o_cache* c, const void* q, const void* k_new, const 
   h2o_status s = check_step_args(c, q, k_new, v_new, n_q, out);
   if (s != H2O_OK || n_q == 0) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (decode_path(c, n_q)) {
+    // the summed weights are final before the eviction changes the scores
+    // and the cache, so they can be copied after it
+    s = run_decode(c, q, k_new, v_new, out, true, st);
+    if (s == H2O_OK && colsum_out) s = copy_colsum(c, colsum_out, n_q, st);
+    return s;
+  }
   s = run_attention(c, q, k_new, v_new, n_q, out, st);
   if (s == H2O_OK && colsum_out) s = copy_colsum(c, colsum_out, n_q, st);
   if (s == H2O_OK) s = run_evict(c, c->colsum, c->colsum_ld, k_new, v_new, n_q, st);
