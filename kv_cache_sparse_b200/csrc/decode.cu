@@ -218,7 +218,8 @@ __global__ void __launch_bounds__(kPartialThreads) decode_partial(const DecodePa
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kFinishThreads) decode_finish(const DecodeParams p) {
-  __shared__ float fac[kDecodeMaxG][kMaxChunks];  // 2^(chunk max - head max)
+  __shared__ float fac[kDecodeMaxG][kMaxChunks];   // 2^(chunk max - head max)
+  __shared__ float psum[kDecodeMaxG][kMaxChunks];  // chunk sums
   __shared__ float mh[kDecodeMaxG], lh[kDecodeMaxG], lse[kDecodeMaxG];
   __shared__ unsigned long long wmin[kFinishThreads / 32];
   const int G = p.G;
@@ -231,29 +232,37 @@ __global__ void __launch_bounds__(kFinishThreads) decode_finish(const DecodePara
   const float* part = p.part + static_cast<size_t>(bg) * p.part_ld * G * (D + 2);
   auto pidx = [&](int c, int h) { return (static_cast<size_t>(c) * G + h) * (D + 2); };
 
-  // ---- merge the chunks, in chunk order
-  if (tid < G) {
-    float m = -INFINITY;
-    for (int c = 0; c < NCk; ++c) m = fmaxf(m, part[pidx(c, tid) + D]);
-    mh[tid] = m;
-  }
-  __syncthreads();
+  // ---- merge the chunks: chunk maxima and sums into shared memory, then
+  // one warp per head reduces them (fixed tree order)
   for (int i = tid; i < NCk * G; i += kFinishThreads) {
     const int c = i / G, h = i % G;
-    fac[h][c] = ex2_approx(part[pidx(c, h) + D] - mh[h]);
+    fac[h][c] = part[pidx(c, h) + D];       // chunk max, turned into the factor below
+    psum[h][c] = part[pidx(c, h) + D + 1];  // chunk sum
   }
   __syncthreads();
-  if (tid < G) {
+  if (warp < G) {
+    float m = -INFINITY;
+    for (int c = lane; c < NCk; c += 32) m = fmaxf(m, fac[warp][c]);
+    m = warp_max(m);
     float l = 0.f;
-    for (int c = 0; c < NCk; ++c) l = fmaf(part[pidx(c, tid) + D + 1], fac[tid][c], l);
-    lh[tid] = l;
-    lse[tid] = mh[tid] + __log2f(l);
+    for (int c = lane; c < NCk; c += 32) {
+      const float f = ex2_approx(fac[warp][c] - m);
+      fac[warp][c] = f;
+      l = fmaf(psum[warp][c], f, l);
+    }
+    l = warp_sum(l);
+    if (lane == 0) {
+      mh[warp] = m;
+      lh[warp] = l;
+      lse[warp] = m + __log2f(l);
+    }
   }
   __syncthreads();
   T* out = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.Hkv * G + g * G) * D;
   for (int i = tid; i < G * D; i += kFinishThreads) {
     const int h = i / D, d = i % D;
     float acc = 0.f;
+#pragma unroll 8
     for (int c = 0; c < NCk; ++c) acc = fmaf(part[pidx(c, h) + d], fac[h][c], acc);
     store(out + i, acc / lh[h]);
   }
@@ -261,6 +270,7 @@ __global__ void __launch_bounds__(kFinishThreads) decode_finish(const DecodePara
   // ---- summed weights: slots, zeros up to C, the new key at C
   const float* lg = p.logits + static_cast<size_t>(bg) * G * (C + 1);
   float* cs = p.colsum + static_cast<size_t>(bg) * p.colsum_ld;
+#pragma unroll 4
   for (int j = tid; j <= n; j += kFinishThreads) {
     float s = 0.f;
     for (int h = 0; h < G; ++h) s += ex2_approx(lg[static_cast<size_t>(h) * (C + 1) + j] - lse[h]);

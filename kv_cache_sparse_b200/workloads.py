@@ -51,6 +51,15 @@ class Workload:
     drift_step: float = 0.0         # norm of the per-token mean step of K
     layers: int = 1
     seqs: int = 1
+    prefill_chunk: int = 0          # chunk of the filling steps (0: ``chunk``)
+
+    @property
+    def fill_chunk(self) -> int:
+        return self.prefill_chunk or self.chunk
+
+    @property
+    def max_chunk(self) -> int:
+        return max(self.chunk, self.fill_chunk)
 
     @property
     def steps(self) -> int:
@@ -89,8 +98,20 @@ STREAM1M = Workload("qwen3_4b_stream_1m_c32768_q1024_w1024", batch=1,
                     capacity=32768, window=1024, seq_len=1 << 20, dtype="bf16",
                     heavy_p=0.01, drift_step=0.01)
 
-WORKLOADS = {w.name: w for w in (TINY, QWEN_C8K, QWEN_C16K, STACK36, STREAM1M)}
-ORDERED = [TINY, QWEN_C8K, QWEN_C16K, STACK36, STREAM1M]
+# Generation after a chunked prefill: one new token per cache and step (the
+# decode step, n_q = 1), for one cache and for the 36-layer x 4-sequence stack.
+# The cache is filled by prefill chunks of 1024 tokens.
+DECODE_C8K = Workload("qwen3_4b_decode_c8192_w256", batch=1, n_q_heads=32,
+                      n_kv_heads=8, head_dim=128, chunk=1, capacity=8192, window=256,
+                      seq_len=8192 + 512, dtype="bf16", heavy_p=0.02, prefill_chunk=1024)
+DECODE_STACK36 = Workload("qwen3_4b_decode_36layer_x4seq_c8192_w256", batch=144,
+                          n_q_heads=32, n_kv_heads=8, head_dim=128, chunk=1,
+                          capacity=8192, window=256, seq_len=8192 + 512, dtype="bf16",
+                          heavy_p=0.02, layers=36, seqs=4, prefill_chunk=1024)
+
+WORKLOADS = {w.name: w for w in (TINY, QWEN_C8K, QWEN_C16K, STACK36, STREAM1M, DECODE_C8K,
+                                 DECODE_STACK36)}
+ORDERED = [TINY, QWEN_C8K, QWEN_C16K, STACK36, STREAM1M, DECODE_C8K, DECODE_STACK36]
 
 
 def _seed64(*words: int) -> int:
