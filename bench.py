@@ -191,7 +191,7 @@ def oracle_sample(wl, steps: int, seed: int = 0, groups=None):
     wl = wl.scaled(n_kv_heads=groups, n_q_heads=groups * wl.group, batch=1)
     rng = np.random.default_rng(seed)
     ref = orc.OracleCache(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.capacity,
-                          wl.window)
+                          wl.window, policy=wl.policy, sinks=wl.sinks)
     C = wl.capacity
     g = torch.Generator().manual_seed(seed)
     K = torch.randn(wl.batch, wl.n_kv_heads, C, wl.head_dim, generator=g).to(torch.bfloat16)
@@ -282,7 +282,8 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     wl = WORKLOADS[args.workload]
     shape = binding.CacheShape(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
-                               wl.capacity, wl.max_chunk, wl.window, wl.torch_dtype())
+                               wl.capacity, wl.max_chunk, wl.window, wl.torch_dtype(), 0.0,
+                               wl.policy, wl.sinks)
     cache = binding.H2OCache(shape, device=dev)
     stream = torch.cuda.current_stream(dev)
     seed = rank_seed(rank)
@@ -375,7 +376,7 @@ def run_ours(args, world, rank, local):
     hbm_peak = peaks["hbm_gbs"]
     kernels = {}
     for i, name in enumerate(KERNELS):
-        if avg[i] <= 0:
+        if avg[i] <= 0 or (i == 1 and wl.policy != "h2o"):  # no summed weights launched
             continue
         kernels[name] = {"ms": round(float(avg[i]), 5),
                          "share": round(float(avg[i] / max(avg.sum(), 1e-12)), 4)}
@@ -435,7 +436,8 @@ def run_ours(args, world, rank, local):
         "data": "synthetic (seeded N(0,1) Q/K/V with 2% heavy-hitter keys, drawn on device)",
         "config": {"workload": wl.name, "caches_per_gpu": wl.batch, "n_q_heads": wl.n_q_heads,
                    "n_kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "chunk": wl.chunk,
-                   "capacity": wl.capacity, "recent_window": wl.window,
+                   "capacity": wl.capacity, "recent_window": wl.window, "policy": wl.policy,
+                   "sink_tokens": wl.sinks,
                    "state": "steady (cache full)", "parallelism": f"independent caches x{world}",
                    "l2": "flushed before every timed step (256 MiB write, outside the events)"},
         "roofline": roof,
@@ -479,7 +481,8 @@ def run_reference(args, world, rank):
         "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "caches_per_gpu": wl.batch, "chunk": wl.chunk,
-                   "capacity": wl.capacity, "recent_window": wl.window,
+                   "capacity": wl.capacity, "recent_window": wl.window, "policy": wl.policy,
+                   "sink_tokens": wl.sinks,
                    "state": "steady (cache full)"},
         "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": cpu_cores(),
                          "blas_threads": blas_threads(), "kind": "oracle", "sample": sample},

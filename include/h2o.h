@@ -87,6 +87,15 @@ typedef enum {
 
 typedef enum { H2O_BF16 = 0, H2O_F32 = 1 } h2o_dtype;
 
+/* Eviction policy.  H2O ranks the unprotected candidates by their
+ * accumulated attention (the summed weights added to the score each step);
+ * LR and SLR are score-free: they rank by position (the most recent stay),
+ * SLR also always keeps the sequence's first sink_tokens positions.  The
+ * recent window protects in every policy; placement is the same.  LR and SLR
+ * keep no scores (placed tokens get 0) and skip the summed-weights kernel
+ * unless colsum_out asks for them. */
+typedef enum { H2O_POLICY_H2O = 0, H2O_POLICY_LR = 1, H2O_POLICY_SLR = 2 } h2o_policy;
+
 typedef struct {
   int32_t batch;          /* independent caches (layers x sequences), >= 1   */
   int32_t n_q_heads;      /* H_q                                             */
@@ -97,6 +106,10 @@ typedef struct {
   int32_t recent_window;  /* W, 0 <= W <= C                                  */
   h2o_dtype dtype;        /* element type of q, k, v, out and the cache      */
   float softmax_scale;    /* <= 0 selects 1/sqrt(head_dim)                   */
+  int32_t policy;         /* h2o_policy                                      */
+  int32_t sink_tokens;    /* SLR: positions < sink_tokens always stay;
+                             0 <= sink_tokens, sink_tokens + recent_window
+                             <= capacity; ignored by the other policies      */
 } h2o_config;
 
 /* Byte sizes of the caller-owned device buffers for a configuration. */

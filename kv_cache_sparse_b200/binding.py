@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libh2o.so")
 
 H2O_OK = 0
 H2O_BF16, H2O_F32 = 0, 1
+POLICIES = {"h2o": 0, "lr": 1, "slr": 2}  # h2o_policy
 STATUS_NAMES = {0: "H2O_OK", 1: "H2O_ERR_INVALID_ARG", 2: "H2O_ERR_SHAPE", 3: "H2O_ERR_DTYPE",
                 4: "H2O_ERR_ALIGN", 5: "H2O_ERR_CUDA", 6: "H2O_ERR_TIMEOUT", 7: "H2O_ERR_STATE"}
 
@@ -38,7 +39,8 @@ class Config(ctypes.Structure):
                 ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("capacity", ctypes.c_int32), ("max_chunk", ctypes.c_int32),
                 ("recent_window", ctypes.c_int32), ("dtype", ctypes.c_int),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("policy", ctypes.c_int32),
+                ("sink_tokens", ctypes.c_int32)]
 
 
 class Sizes(ctypes.Structure):
@@ -116,11 +118,14 @@ class CacheShape:
     recent_window: int
     dtype: torch.dtype = torch.bfloat16
     softmax_scale: float = 0.0
+    policy: str = "h2o"     # "h2o", "lr" or "slr"
+    sink_tokens: int = 0    # "slr": the first positions that always stay
 
     def config(self) -> Config:
         dt = {torch.bfloat16: H2O_BF16, torch.float32: H2O_F32}[self.dtype]
         return Config(self.batch, self.n_q_heads, self.n_kv_heads, self.head_dim, self.capacity,
-                      self.max_chunk, self.recent_window, dt, self.softmax_scale)
+                      self.max_chunk, self.recent_window, dt, self.softmax_scale,
+                      POLICIES[self.policy], self.sink_tokens)
 
 
 def required_bytes(shape: CacheShape) -> Sizes:

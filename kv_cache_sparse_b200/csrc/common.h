@@ -46,6 +46,10 @@ struct AttnParams {
 
 // ---------------------------------------------------------------- eviction
 
+constexpr int kPolicyH2O = 0;
+constexpr int kPolicyLR = 1;
+constexpr int kPolicySLR = 2;
+
 struct EvictParams {
   int B, Hkv, C, d, esize;  // esize: bytes per element of K/V
   int n, t0, nq, W;
@@ -62,6 +66,8 @@ struct EvictParams {
   void* k_cache;            // [B, Hkv, C, d]
   void* v_cache;
   int* state;               // [4]: n, t0, err, reserved
+  int policy;               // kPolicyH2O (rank by score), kPolicyLR / kPolicySLR (by position)
+  int sinks;                // kPolicySLR: positions < sinks are protected
 };
 
 // ---------------------------------------------------------------- decode (n_q = 1)
@@ -89,6 +95,8 @@ struct DecodeParams {
   int* pos;                 // [B, Hkv, C]
   int* state;               // [4]: n, t0, err, reserved
   int evict;                // 1: score update and placement after the attention
+  int policy;               // as in EvictParams
+  int sinks;
 };
 
 }  // namespace h2o

@@ -293,10 +293,14 @@ __global__ void __launch_bounds__(kFinishThreads) decode_finish(const DecodePara
     p.state[0] = min(C, n + 1);
     p.state[1] = p.t0 + 1;
   }
+  const bool by_score = p.policy == kPolicyH2O;
+  const int sinks = p.policy == kPolicySLR ? p.sinks : 0;
+  const float snew = by_score ? cnew : 0.f;  // the score-free policies keep none
   if (n < C) {  // room left: the new token takes slot n
-    for (int s = tid; s < n; s += kFinishThreads) score[s] = __fadd_rn(score[s], cs[s]);
+    if (by_score)
+      for (int s = tid; s < n; s += kFinishThreads) score[s] = __fadd_rn(score[s], cs[s]);
     if (tid == 0) {
-      score[n] = cnew;
+      score[n] = snew;
       pos[n] = p.t0;
     }
     if (warp == 0) {
@@ -305,23 +309,31 @@ __global__ void __launch_bounds__(kFinishThreads) decode_finish(const DecodePara
     }
     return;
   }
-  // full: candidates with position < t0 + 1 - W are unprotected; the one with
-  // the lowest score (then the highest index: slot s -> s, new token -> C)
-  // leaves.  Scores are >= 0, so their bit patterns order like the values.
+  // full: candidates with position < t0 + 1 - W (and, under SLR, >= the sink
+  // count) are unprotected; the one with the lowest rank value (then the
+  // highest index: slot s -> s, new token -> C) leaves.  The rank value is the
+  // score (>= 0, so its bit pattern orders like the value) or, for the
+  // score-free policies, the position.
   const long long limit = static_cast<long long>(p.t0) + 1 - p.W;
   unsigned long long best = ~0ull;
   for (int s = tid; s < C; s += kFinishThreads) {
-    const float sc = __fadd_rn(score[s], cs[s]);
-    score[s] = sc;
-    if (pos[s] < limit) {
-      const unsigned long long key =
-          (static_cast<unsigned long long>(__float_as_uint(sc)) << 32) | (0xffffffffu - s);
+    const int ps = pos[s];
+    uint32_t rank;
+    if (by_score) {
+      const float sc = __fadd_rn(score[s], cs[s]);
+      score[s] = sc;
+      rank = __float_as_uint(sc);
+    } else {
+      rank = static_cast<uint32_t>(ps);
+    }
+    if (ps < limit && ps >= sinks) {
+      const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - s);
       best = key < best ? key : best;
     }
   }
-  if (tid == 0 && p.t0 < limit) {  // W = 0: the new token competes too
-    const unsigned long long key =
-        (static_cast<unsigned long long>(__float_as_uint(cnew)) << 32) | (0xffffffffu - C);
+  if (tid == 0 && p.t0 < limit && p.t0 >= sinks) {  // W = 0: the new token competes too
+    const uint32_t rank = by_score ? __float_as_uint(cnew) : static_cast<uint32_t>(p.t0);
+    const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - C);
     best = key < best ? key : best;
   }
 #pragma unroll
@@ -345,7 +357,7 @@ __global__ void __launch_bounds__(kFinishThreads) decode_finish(const DecodePara
     const int e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(best & 0xffffffffu));
     if (e < C) {  // an old slot leaves; the new token takes it
       if (lane == 0) {
-        score[e] = cnew;
+        score[e] = snew;
         pos[e] = p.t0;
       }
       copy_row(kc + static_cast<size_t>(e) * row_bytes, kn, static_cast<int>(row_bytes), lane);

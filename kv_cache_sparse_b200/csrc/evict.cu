@@ -7,7 +7,10 @@
 // h2o_select (one 1024-thread CTA per (cache, KV head); candidates in shared
 // memory):
 //   1. score[s] <- fl32(score[s] + colsum[s]) for the n valid slots; new token
-//      i's candidate score is colsum[C + i].
+//      i's candidate score is colsum[C + i].  The score-free policies (LR,
+//      SLR) rank by position instead: a candidate's key is its position, no
+//      score is accumulated and placed tokens get score 0; SLR also protects
+//      positions below the sink count.
 //   2. If n + nq <= C every new token is kept and goes to slot n + i.
 //   3. Otherwise a candidate at position >= t0 + nq - W is protected.  Each
 //      candidate gets a 32-bit key: 0xFFFFFFFF when protected, else the bit
@@ -108,8 +111,12 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1)) h2o_select(const Evic
   int* __restrict__ toks = e.plan_tokens + static_cast<size_t>(bg) * e.plan_ld;
   const bool evict = NC > C;
   const long long limit = static_cast<long long>(e.t0) + nq - e.W;
-  // an old slot (position < t0) can be protected only when W > nq
-  const bool old_protectable = evict && e.W > nq;
+  const bool by_score = e.policy == kPolicyH2O;
+  const int sinks = e.policy == kPolicySLR ? e.sinks : 0;
+  // an old slot (position < t0) can be protected by the window only when
+  // W > nq, by the sinks only under SLR
+  const bool old_protectable = evict && (e.W > nq || sinks > 0);
+  const bool need_pos = old_protectable || !by_score;
   griddep_wait();  // the summed weights come from the preceding kernel
   if (bg == 0 && tid == 0) {
     e.state[0] = min(C, n + nq);
@@ -128,18 +135,27 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1)) h2o_select(const Evic
       cv[k] = 0.f;
       ps[k] = -1;
       if (x < n) {
-        sc[k] = score[x];
-        cv[k] = cs[x];
-        if (old_protectable) ps[k] = pos[x];
+        if (by_score) {
+          sc[k] = score[x];
+          cv[k] = cs[x];
+        }
+        if (need_pos) ps[k] = pos[x];
       }
     }
 #pragma unroll
     for (int k = 0; k < kLoadBatch; ++k) {
       const int x = x0 + k * NT;
       if (x < n) {
-        const float s = sc[k] + cv[k];
-        score[x] = s;
-        keys[x] = (old_protectable && ps[k] >= limit) ? kProtectedKey : score_key(s);
+        const bool prot = old_protectable && (ps[k] >= limit || ps[k] < sinks);
+        uint32_t key;
+        if (by_score) {
+          const float s = sc[k] + cv[k];
+          score[x] = s;
+          key = score_key(s);
+        } else {
+          key = static_cast<uint32_t>(ps[k]);  // the most recent rank highest
+        }
+        keys[x] = prot ? kProtectedKey : key;
       }
     }
   }
@@ -148,14 +164,17 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1)) h2o_select(const Evic
 #pragma unroll
     for (int k = 0; k < kLoadBatch; ++k) {
       const int i = i0 + k * NT;
-      cv[k] = i < nq ? cs[C + i] : 0.f;
+      cv[k] = (by_score && i < nq) ? cs[C + i] : 0.f;
     }
 #pragma unroll
     for (int k = 0; k < kLoadBatch; ++k) {
       const int i = i0 + k * NT;
-      if (i < nq)
-        keys[n + i] = (evict && static_cast<long long>(e.t0) + i >= limit) ? kProtectedKey
-                                                                           : score_key(cv[k]);
+      if (i < nq) {
+        const long long p = static_cast<long long>(e.t0) + i;
+        const bool prot = evict && (p >= limit || p < sinks);
+        keys[n + i] = prot ? kProtectedKey
+                           : (by_score ? score_key(cv[k]) : static_cast<uint32_t>(p));
+      }
     }
   }
   if (!evict) {
@@ -163,7 +182,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1)) h2o_select(const Evic
     for (int i = tid; i < nq; i += NT) {
       slots[i] = n + i;
       toks[i] = i;
-      score[n + i] = cs[C + i];
+      score[n + i] = by_score ? cs[C + i] : 0.f;
       pos[n + i] = e.t0 + i;
     }
     if (tid == 0) e.plan_count[bg] = nq;
@@ -285,7 +304,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1)) h2o_select(const Evic
   // 4. scores and positions of the placed tokens, then their K/V rows
   for (int q = tid; q < tot_new; q += NT) {
     const int s = slots[q], i = toks[q];
-    score[s] = cs[C + i];
+    score[s] = by_score ? cs[C + i] : 0.f;
     pos[s] = e.t0 + i;
   }
   if (tid == 0) e.plan_count[bg] = tot_new;

@@ -114,6 +114,10 @@ h2o_status check_config(const h2o_config* c) {
   if (c->n_q_heads % c->n_kv_heads != 0) return H2O_ERR_SHAPE;
   if (c->head_dim != 64 && c->head_dim != 128) return H2O_ERR_SHAPE;
   if (c->recent_window < 0 || c->recent_window > c->capacity) return H2O_ERR_SHAPE;
+  if (c->policy < H2O_POLICY_H2O || c->policy > H2O_POLICY_SLR) return H2O_ERR_INVALID_ARG;
+  if (c->policy == H2O_POLICY_SLR &&
+      (c->sink_tokens < 0 || static_cast<long long>(c->sink_tokens) + c->recent_window > c->capacity))
+    return H2O_ERR_SHAPE;
   if (static_cast<long long>(c->capacity) + c->max_chunk > kMaxCandidates) return H2O_ERR_SHAPE;
   if (static_cast<long long>(c->batch) * c->n_kv_heads > 65535) return H2O_ERR_SHAPE;
   if (static_cast<long long>(c->batch) * c->n_q_heads * cdiv(c->max_chunk, 128) > (1ll << 31) - 1)
@@ -210,8 +214,10 @@ AttnParams attn_params(h2o_cache* c, int nq, void* out) {
 }
 
 // K1 + K2 into the workspace (lse2, colsum) and `out`.
+// K1 + K2 (K2 only when the summed weights are needed: the H2O policy, or a
+// caller asking for them).
 h2o_status run_attention(h2o_cache* c, const void* q, const void* kn, const void* vn, int nq,
-                         void* out, cudaStream_t st) {
+                         void* out, cudaStream_t st, bool with_colsum = true) {
   const h2o_config& g = c->cfg;
   AttnParams p = attn_params(c, nq, out);
   for (int i = 0; i < 5; ++i) c->ev_used[i] = false;
@@ -238,9 +244,11 @@ h2o_status run_attention(h2o_cache* c, const void* q, const void* kn, const void
   if (e != cudaSuccess) return H2O_ERR_CUDA;
   c->launches += 1;
   mark(c, 1, st);
-  e = launch_attn_colsum_bf16(g.head_dim, m, p, st);
-  if (e != cudaSuccess) return H2O_ERR_CUDA;
-  c->launches += 1;
+  if (with_colsum) {
+    e = launch_attn_colsum_bf16(g.head_dim, m, p, st);
+    if (e != cudaSuccess) return H2O_ERR_CUDA;
+    c->launches += 1;
+  }
   mark(c, 2, st);
   return H2O_OK;
 }
@@ -272,6 +280,8 @@ h2o_status run_evict(h2o_cache* c, const float* colsum, int ld, const void* kn, 
   e.k_cache = c->buf.k;
   e.v_cache = c->buf.v;
   e.state = c->buf.state;
+  e.policy = g.policy;
+  e.sinks = g.sink_tokens;
   if (!c->ev_used[2]) {  // eviction on its own: time it from here
     for (int i = 0; i < 5; ++i) c->ev_used[i] = false;
     mark(c, 2, st);
@@ -321,6 +331,8 @@ h2o_status run_decode(h2o_cache* c, const void* q, const void* kn, const void* v
   d.pos = c->buf.pos;
   d.state = c->buf.state;
   d.evict = evict ? 1 : 0;
+  d.policy = g.policy;
+  d.sinks = g.sink_tokens;
   for (int i = 0; i < 5; ++i) c->ev_used[i] = false;
   mark(c, 0, st);
   if (launch_decode(d, static_cast<int>(esize_of(g.dtype)), g.head_dim, st) != cudaSuccess)
@@ -479,7 +491,8 @@ h2o_status h2o_chunk_step(h2o_cache* c, const void* q, const void* k_new, const 
     if (s == H2O_OK && colsum_out) s = copy_colsum(c, colsum_out, n_q, st);
     return s;
   }
-  s = run_attention(c, q, k_new, v_new, n_q, out, st);
+  s = run_attention(c, q, k_new, v_new, n_q, out, st,
+                    c->cfg.policy == H2O_POLICY_H2O || colsum_out != nullptr);
   if (s == H2O_OK && colsum_out) s = copy_colsum(c, colsum_out, n_q, st);
   if (s == H2O_OK) s = run_evict(c, c->colsum, c->colsum_ld, k_new, v_new, n_q, st);
   return s;

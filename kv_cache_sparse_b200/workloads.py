@@ -52,6 +52,8 @@ class Workload:
     layers: int = 1
     seqs: int = 1
     prefill_chunk: int = 0          # chunk of the filling steps (0: ``chunk``)
+    policy: str = "h2o"             # eviction policy: "h2o", "lr" or "slr"
+    sinks: int = 0                  # "slr": first positions that always stay
 
     @property
     def fill_chunk(self) -> int:
@@ -109,9 +111,16 @@ DECODE_STACK36 = Workload("qwen3_4b_decode_36layer_x4seq_c8192_w256", batch=144,
                           capacity=8192, window=256, seq_len=8192 + 512, dtype="bf16",
                           heavy_p=0.02, layers=36, seqs=4, prefill_chunk=1024)
 
+# The headline cache under the score-free policies (the summary page's
+# lr-vs-h2o step-time comparison, Table 6): no summed weights are needed.
+LR_C8K = dataclasses.replace(QWEN_C8K, name="qwen3_4b_lr_c8192_q1024_w256", policy="lr")
+SLR_C8K = dataclasses.replace(QWEN_C8K, name="qwen3_4b_slr4_c8192_q1024_w256", policy="slr",
+                              sinks=4)
+
 WORKLOADS = {w.name: w for w in (TINY, QWEN_C8K, QWEN_C16K, STACK36, STREAM1M, DECODE_C8K,
-                                 DECODE_STACK36)}
-ORDERED = [TINY, QWEN_C8K, QWEN_C16K, STACK36, STREAM1M, DECODE_C8K, DECODE_STACK36]
+                                 DECODE_STACK36, LR_C8K, SLR_C8K)}
+ORDERED = [TINY, QWEN_C8K, QWEN_C16K, STACK36, STREAM1M, DECODE_C8K, DECODE_STACK36, LR_C8K,
+           SLR_C8K]
 
 
 def _seed64(*words: int) -> int:

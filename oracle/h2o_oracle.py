@@ -33,6 +33,13 @@ The readings taken here, where the sources are silent:
   index, where cache slot s has index s and new token i has index C + i.
 * Placement: surviving entries keep their slot; the kept new tokens, in
   ascending order, take the freed (and empty) slots in ascending order.
+* The score-free policies ``lr`` and ``slr`` (summary page, Tables 1, 2, 5
+  and 6, named only): ``lr`` keeps the most recent tokens, ``slr`` keeps the
+  first ``sinks`` positions of the sequence as well ("sink" tokens) and the
+  most recent ones otherwise.  Reading: the same selection and placement as
+  H2O with the candidate's position in place of its score (positions are
+  distinct, so there are no ties), the recent window still protecting, and
+  no score kept: old slots keep theirs, placed tokens get 0.
 
 Parity status: attention output, summed weights and the selection are pinned
 by brute force, a library routine (torch SDPA in fp64), closed forms and
@@ -117,31 +124,49 @@ class Placement:
     evicted: List[int] = field(default_factory=list)  # old slots dropped
 
 
+POLICIES = ("h2o", "lr", "slr")
+
+
 def evict_one_head(score: np.ndarray, pos: np.ndarray, n: int, t0: int,
-                   colsum32: np.ndarray, n_q: int, window: int):
-    """Score update + H2O selection + placement for one (cache, KV head).
+                   colsum32: np.ndarray, n_q: int, window: int, policy: str = "h2o",
+                   sinks: int = 0):
+    """Score update + selection + placement for one (cache, KV head).
 
     score [C] float32, pos [C] int32 (-1 empty), colsum32 [C + n_q] float32
-    (layout of ``attention_one_cache``).  Returns (new score, new pos,
-    Placement).  Inputs are not modified.
+    (layout of ``attention_one_cache``; not read by the score-free
+    policies).  ``policy``: "h2o" ranks the unprotected candidates by score,
+    "lr" and "slr" by position; "slr" also protects positions < ``sinks``.
+    Returns (new score, new pos, Placement).  Inputs are not modified.
     """
+    assert policy in POLICIES
     C = score.shape[0]
     score = score.astype(F32).copy()
     pos = pos.astype(np.int32).copy()
-    # one fp32 addition per cached slot
-    score[:n] = (score[:n] + colsum32[:n].astype(F32)).astype(F32)
-    cand_new = colsum32[C:C + n_q].astype(F32)
+    if policy == "h2o":
+        # one fp32 addition per cached slot
+        score[:n] = (score[:n] + colsum32[:n].astype(F32)).astype(F32)
+        cand_new = colsum32[C:C + n_q].astype(F32)
+    else:
+        cand_new = np.zeros(n_q, dtype=F32)
     pl = Placement()
     if n + n_q <= C:
         pl.slots = list(range(n, n + n_q))
         pl.tokens = list(range(n_q))
     else:
         limit = t0 + n_q - window
-        # candidates: (index, score, position, is_new, slot-or-token)
-        cands = [(s, float(score[s]), int(pos[s]), False, s) for s in range(n)]
-        cands += [(C + i, float(cand_new[i]), t0 + i, True, i) for i in range(n_q)]
-        protected = [c for c in cands if c[2] >= limit]
-        unprot = [c for c in cands if c[2] < limit]
+        # candidates: (index, rank value, position, is_new, slot-or-token)
+        if policy == "h2o":
+            cands = [(s, float(score[s]), int(pos[s]), False, s) for s in range(n)]
+            cands += [(C + i, float(cand_new[i]), t0 + i, True, i) for i in range(n_q)]
+        else:
+            cands = [(s, float(pos[s]), int(pos[s]), False, s) for s in range(n)]
+            cands += [(C + i, float(t0 + i), t0 + i, True, i) for i in range(n_q)]
+
+        def is_protected(c):
+            return c[2] >= limit or (policy == "slr" and c[2] < sinks)
+
+        protected = [c for c in cands if is_protected(c)]
+        unprot = [c for c in cands if not is_protected(c)]
         k_keep = C - len(protected)
         ranked = sorted(unprot, key=lambda c: (-c[1], c[0]))
         kept = {c[0] for c in protected} | {c[0] for c in ranked[:k_keep]}
@@ -169,9 +194,12 @@ class OracleCache:
     """
 
     def __init__(self, batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
-                 capacity: int, window: int, scale: Optional[float] = None):
+                 capacity: int, window: int, scale: Optional[float] = None,
+                 policy: str = "h2o", sinks: int = 0):
         assert n_q_heads % n_kv_heads == 0
         assert 0 <= window <= capacity
+        assert policy in POLICIES and 0 <= sinks and (policy != "slr" or sinks + window <= capacity)
+        self.policy, self.sinks = policy, sinks
         self.B, self.H_q, self.H_kv, self.d = batch, n_q_heads, n_kv_heads, head_dim
         self.C, self.W = capacity, window
         self.scale = 1.0 / math.sqrt(head_dim) if scale is None else float(scale)
@@ -222,7 +250,8 @@ class OracleCache:
             row = []
             for g in range(self.H_kv):
                 sc, ps, pl = evict_one_head(self.scores[b, g], self.pos[b, g], self.n,
-                                            self.t0, colsum32[b, g], n_q, self.W)
+                                            self.t0, colsum32[b, g], n_q, self.W,
+                                            self.policy, self.sinks)
                 self.scores[b, g], self.pos[b, g] = sc, ps
                 if pl.slots:
                     self.K[b, g, pl.slots] = Kn[b, pl.tokens, g]

@@ -63,6 +63,10 @@ def test_required_bytes_qwen_shape(lib):
     (dict(dtype=7), 3), (dict(batch=0), 2), (dict(max_chunk=0), 2),
     (dict(dtype=binding.H2O_F32, head_dim=64, n_q_heads=4, n_kv_heads=2, capacity=256,
           max_chunk=64, recent_window=0), 0),
+    (dict(policy=1), 0), (dict(policy=2, sink_tokens=4), 0), (dict(policy=3), 1),
+    (dict(policy=-1), 1), (dict(policy=2, sink_tokens=-1), 2),
+    (dict(policy=2, sink_tokens=8192 - 255), 2), (dict(policy=2, sink_tokens=8192 - 256), 0),
+    (dict(policy=1, sink_tokens=9000), 0),  # the sink count matters only to SLR
 ])
 def test_config_validation(lib, kw, expect):
     st, _ = _req(lib, _cfg(**kw))
