@@ -31,10 +31,12 @@ cudaError_t launch_attn_f32(int head_dim, const float* q, const float* kc, const
                             const float* kn, const float* vn, const AttnParams& p,
                             cudaStream_t st);
 
-// Decode step (n_q = 1, G <= kDecodeMaxG): split-KV partials, then the merge,
+// Decode step (n_q = 1, G in {1, 2, 4, 8}): split-KV partials, then the merge,
 // summed weights and (if p.evict) the single-token eviction.  esize 2 (bf16)
 // or 4 (float), head_dim 64 or 128.
 cudaError_t launch_decode(const DecodeParams& p, int esize, int head_dim, cudaStream_t st);
+// Group sizes the decode kernels take (a warp batch holds 32 / G keys).
+bool decode_supported(int G);
 
 // K3 (with the K/V scatter fused): score update, selection, placement.
 cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st);

@@ -72,14 +72,24 @@ struct EvictParams {
 
 // ---------------------------------------------------------------- decode (n_q = 1)
 
-constexpr int kDecodeChunk = 256;  // keys per split-KV partial
-constexpr int kDecodeMaxG = 8;     // largest GQA group the decode kernels take
+constexpr int kDecodeMaxG = 8;        // largest GQA group the decode kernels take
+constexpr int kDecodeSliceKeys = 1024;  // keys per CTA of the merge kernel
+
+// Keys per split-KV partial: 32 KiB of K (and of V) rows, at most 256 keys.
+__host__ __device__ constexpr int decode_chunk_keys(int head_dim, int esize) {
+  return 32768 / (head_dim * esize) < 256 ? 32768 / (head_dim * esize) : 256;
+}
 
 struct DecodeParams {
   int B, Hkv, G, C;         // caches, KV heads, heads per group, capacity
   int n, t0, W;             // valid slots, position of the new token, window
-  int n_chunks;             // cdiv(n + 1, kDecodeChunk): key n is the new token
+  int n_chunks;             // cdiv(n + 1, decode_chunk_keys): key n is the new token
   int part_ld;              // chunks per (cache, KV head) in part
+  int n_slices;             // cdiv(n + 1, kDecodeSliceKeys): CTAs of the merge per head
+  int slices_ld;            // entries per (cache, KV head) in best
+  unsigned long long* best; // [B*Hkv, slices_ld]: each merge CTA's eviction candidate
+  int* ticket;              // [B*Hkv]: merge CTAs done (zero between steps)
+  int spread_o;             // 1: every merge CTA of a head merges part of O
   float scale_log2;         // softmax scale * log2(e)
   const void* q;            // [B, 1, Hq, d]
   const void* k_new;        // [B, 1, Hkv, d]

@@ -8,23 +8,34 @@
 // bytes per (slot, KV head) for 4·d·G FLOPs, so it is bound by HBM, not by
 // the tensor cores, and runs on the FMA pipe.  The keys are split over many
 // CTAs (split-KV):
-//   decode_partial  grid (cdiv(n + 1, 256), B*Hkv), 256 threads.  The keys
-//                   [256k, 256k + 256) of one (cache, KV head); key n is the
-//                   new token.  Thread = key: the G logits x = c<q_h, k>
-//                   (fp32 FMA over 16-byte loads of the K row), stored for
-//                   the summed weights; the chunk's max and sum of 2^(x - m)
-//                   per head.  Then thread = (8 head-dim elements, key
-//                   group): the chunk's unnormalised P V for the G heads,
-//                   summed over the key groups in a fixed order.
-//   decode_finish   grid B*Hkv, 512 threads.  Merges the chunks of each head
-//                   (max, sum, O) in chunk order, writes O and the summed
-//                   weights colsum[j] = sum_h 2^(x_hj - lse2_h), and when
-//                   evicting adds them to the scores (one fp32 add each) and
-//                   places the new token: the top-C rule of the chunk step
-//                   with N_q = 1 keeps all but one candidate, the unprotected
-//                   one last in (score desc, index asc) order -- the lowest
-//                   score, the highest index among equal scores.
-// Both are deterministic (fixed reduction orders, no atomics).
+//   decode_partial  grid (cdiv(n + 1, KC), B*Hkv), 256 threads; KC keys per
+//                   CTA (32 KiB of rows: 128 for bf16, d = 128).  Two bulk
+//                   copies (cp.async.bulk) bring the chunk's K and V rows into
+//                   shared memory; the new token's row (key n) is copied by a
+//                   warp.  Logits: each lane holds d/32 elements of the G
+//                   query rows; a warp takes 32/G keys at a time, so that its
+//                   32 lanes hold partial sums of 32 (key, head) pairs, and a
+//                   transposing butterfly (5 shuffle rounds, each lane giving
+//                   away half of its values) leaves lane l with the full dot
+//                   product of pair l.  The logits are stored for the summed
+//                   weights; one warp per head takes the chunk's max and sum;
+//                   P V is accumulated per lane over the head-dim slice, the
+//                   eight warps' partial sums added in a fixed order.
+//   decode_finish   grid (cdiv(n + 1, 1024), B*Hkv), 256 threads, programmatic
+//                   dependent launch.  Every CTA merges the chunk statistics
+//                   of each head (lse2) and a share of the outputs O.  Each CTA
+//                   writes the summed weights colsum[j] = sum_h 2^(x_hj -
+//                   lse2_h) of its 1024 keys and, when evicting, adds them to
+//                   its slots' scores and finds its eviction candidate; the
+//                   last CTA of the (cache, KV head) to finish (atomic ticket)
+//                   takes the minimum over the slices and places the new
+//                   token.  The rule is the top-C rule of the chunk step with
+//                   N_q = 1: the unprotected candidate last in (score desc,
+//                   index asc) order leaves -- the lowest score, the highest
+//                   index among equal scores (for the score-free policies the
+//                   position takes the place of the score).
+// Both are deterministic (fixed reduction orders; the atomic only elects the
+// CTA that finishes).
 #include <cuda_bf16.h>
 
 #include "attn.h"
@@ -34,25 +45,39 @@ namespace h2o {
 
 namespace {
 
-constexpr int kPartialThreads = 256;
-constexpr int kFinishThreads = 512;
-constexpr int kMaxChunks = (kMaxCandidates + kDecodeChunk - 1) / kDecodeChunk;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxChunks = (kMaxCandidates + 1 + 63) / 64;  // smallest chunk: 64 keys
 
-__device__ __forceinline__ void load8(const __nv_bfloat16* src, float (&f)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4*>(src);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {  // element 2i is the low half of word i
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
+template <typename T, int E>
+__device__ __forceinline__ void lds_row(const uint8_t* src, float (&f)[E]);
+
+template <>
+__device__ __forceinline__ void lds_row<__nv_bfloat16, 4>(const uint8_t* src, float (&f)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(src);
+  f[0] = __uint_as_float(u.x << 16);
+  f[1] = __uint_as_float(u.x & 0xffff0000u);
+  f[2] = __uint_as_float(u.y << 16);
+  f[3] = __uint_as_float(u.y & 0xffff0000u);
 }
 
-__device__ __forceinline__ void load8(const float* src, float (&f)[8]) {
-  const float4 a = *reinterpret_cast<const float4*>(src);
-  const float4 b = *reinterpret_cast<const float4*>(src + 4);
-  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+template <>
+__device__ __forceinline__ void lds_row<__nv_bfloat16, 2>(const uint8_t* src, float (&f)[2]) {
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(src);
+  f[0] = __uint_as_float(u << 16);
+  f[1] = __uint_as_float(u & 0xffff0000u);
+}
+
+template <>
+__device__ __forceinline__ void lds_row<float, 4>(const uint8_t* src, float (&f)[4]) {
+  const float4 v = *reinterpret_cast<const float4*>(src);
+  f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+}
+
+template <>
+__device__ __forceinline__ void lds_row<float, 2>(const uint8_t* src, float (&f)[2]) {
+  const float2 v = *reinterpret_cast<const float2*>(src);
+  f[0] = v.x; f[1] = v.y;
 }
 
 __device__ __forceinline__ float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
@@ -72,251 +97,305 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Copies one row of `bytes` bytes (a multiple of 16) with the lanes of a warp.
+__device__ __forceinline__ unsigned long long warp_min64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = w < v ? w : v;
+  }
+  return v;
+}
+
+// Copies `bytes` (a multiple of 16) with the lanes of a warp.
 __device__ __forceinline__ void copy_row(void* dst, const void* src, int bytes, int lane) {
   for (int o = lane * 16; o < bytes; o += 32 * 16)
     *reinterpret_cast<uint4*>(static_cast<char*>(dst) + o) =
         *reinterpret_cast<const uint4*>(static_cast<const char*>(src) + o);
 }
 
-template <typename T, int D>
-__global__ void __launch_bounds__(kPartialThreads) decode_partial(const DecodeParams p) {
-  constexpr int U = D / 8;                         // 8-element pieces of a row
-  constexpr int KG = kPartialThreads / U;          // key groups of the P V phase
-  constexpr int KPG = kDecodeChunk / KG;           // keys per group
-  extern __shared__ __align__(16) float dsm[];
-  const int G = p.G;
-  float* qs = dsm;                                 // [G][D]
-  float* ps = qs + G * D;                          // [G][kDecodeChunk]
-  float* ored = ps + G * kDecodeChunk;             // [KG][G][D]
-  __shared__ float wred[kDecodeMaxG][kPartialThreads / 32];
-  __shared__ float hstat[kDecodeMaxG][2];          // chunk max, chunk sum
+template <typename T, int D, int G>
+struct PartialLayout {
+  static constexpr int KC = decode_chunk_keys(D, sizeof(T));
+  static constexpr int kRow = D * static_cast<int>(sizeof(T));
+  static constexpr int kK = 0;                          // [KC][D] T
+  static constexpr int kV = kK + KC * kRow;             // [KC][D] T
+  static constexpr int kX = kV + KC * kRow;             // [G][KC] float: logits, then P
+  static constexpr int kO = kX + G * KC * 4;            // [warps][G][D] float
+  static constexpr int kBytes = kO + kWarps * G * D * 4;
+};
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p) {
+  using L = PartialLayout<T, D, G>;
+  constexpr int KC = L::KC;
+  constexpr int E = D / 32;   // row elements per lane
+  constexpr int KB = 32 / G;  // keys per warp batch: 32 (key, head) pairs
+  extern __shared__ __align__(128) uint8_t dsm[];
+  uint8_t* sK = dsm + L::kK;
+  uint8_t* sV = dsm + L::kV;
+  float* xs = reinterpret_cast<float*>(dsm + L::kX);
+  float* ored = reinterpret_cast<float*>(dsm + L::kO);
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ int abort_flag;
+  __shared__ float hstat[G][2];  // chunk max, chunk sum
   // the merge kernel may start; it waits for this grid before reading
   griddep_launch_dependents();
 
   const int bg = blockIdx.y;
   const int b = bg / p.Hkv, g = bg % p.Hkv;
   const int chunk = blockIdx.x;
-  const int j0 = chunk * kDecodeChunk;
+  const int j0 = chunk * KC;
   const int nk = p.n + 1;
+  const int nkc = min(KC, nk - j0);           // keys of this chunk (>= 1)
+  const int rows = max(0, min(KC, p.n - j0));  // of them cache slots
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const T* q = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hkv * G + g * G) * D;
-  for (int i = tid; i < G * D; i += kPartialThreads) qs[i] = to_float(q[i]);
+  int* err = p.state + 2;
+  const uint32_t bK = smem_u32(&bars[0]), bV = smem_u32(&bars[1]);
+  if (tid == 0) {
+    mbar_init(bK, 1);
+    mbar_init(bV, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
   __syncthreads();
+  if (tid == 0 && rows > 0) {
+    const size_t off = (static_cast<size_t>(bg) * p.C + j0) * L::kRow;
+    const uint32_t bytes = static_cast<uint32_t>(rows) * L::kRow;
+    mbar_arrive_expect_tx(bK, bytes);
+    bulk_load(smem_u32(sK), static_cast<const uint8_t*>(p.k_cache) + off, bytes, bK);
+    mbar_arrive_expect_tx(bV, bytes);
+    bulk_load(smem_u32(sV), static_cast<const uint8_t*>(p.v_cache) + off, bytes, bV);
+  }
+  if (warp == 0 && nkc > rows) {  // the new token is key n, in this chunk
+    copy_row(sK + rows * L::kRow, static_cast<const uint8_t*>(p.k_new) + bg * L::kRow, L::kRow, lane);
+    copy_row(sV + rows * L::kRow, static_cast<const uint8_t*>(p.v_new) + bg * L::kRow, L::kRow, lane);
+  }
+  // this lane's slice of the G query rows
+  float qf[G][E];
+  {
+    const T* q = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hkv * G + g * G) * D;
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < E; ++e) qf[h][e] = to_float(q[h * D + lane * E + e]);
+  }
+  __syncthreads();  // the new token's rows are in place
+  bool ok = rows == 0 || mbar_wait(bK, 0, err, &abort_flag);
 
-  // ---- thread = key: logits of the G heads
-  const int j = j0 + tid;
-  const bool valid = j < nk;
-  float x[kDecodeMaxG];
+  // ---- logits: a warp batch is KB keys x G heads = 32 dot products
+  if (ok) {
+    float* lg = p.logits + static_cast<size_t>(bg) * G * (p.C + 1);
+    for (int k0 = warp * KB; k0 < nkc; k0 += kWarps * KB) {
+      float v[32];
 #pragma unroll
-  for (int h = 0; h < kDecodeMaxG; ++h) x[h] = 0.f;
-  if (valid) {
-    const T* krow = j < p.n
-                        ? static_cast<const T*>(p.k_cache) + (static_cast<size_t>(bg) * p.C + j) * D
-                        : static_cast<const T*>(p.k_new) + static_cast<size_t>(bg) * D;
-#pragma unroll 4
-    for (int d0 = 0; d0 < D; d0 += 8) {
-      float kf[8];
-      load8(krow + d0, kf);
+      for (int k = 0; k < KB; ++k) {
+        float kf[E];
+        lds_row<T, E>(sK + (k0 + k) * L::kRow + lane * E * sizeof(T), kf);
 #pragma unroll
-      for (int h = 0; h < kDecodeMaxG; ++h) {
-        if (h < G) {
-          const float4 qa = *reinterpret_cast<const float4*>(qs + h * D + d0);
-          const float4 qb = *reinterpret_cast<const float4*>(qs + h * D + d0 + 4);
-          float a = x[h];
-          a = fmaf(qa.x, kf[0], a);
-          a = fmaf(qa.y, kf[1], a);
-          a = fmaf(qa.z, kf[2], a);
-          a = fmaf(qa.w, kf[3], a);
-          a = fmaf(qb.x, kf[4], a);
-          a = fmaf(qb.y, kf[5], a);
-          a = fmaf(qb.z, kf[6], a);
-          a = fmaf(qb.w, kf[7], a);
-          x[h] = a;
+        for (int h = 0; h < G; ++h) {
+          float a = 0.f;
+#pragma unroll
+          for (int e = 0; e < E; ++e) a = fmaf(qf[h][e], kf[e], a);
+          v[k * G + h] = a;
         }
       }
-    }
-  }
-  float* lg = p.logits + static_cast<size_t>(bg) * G * (p.C + 1);
+      // transposing butterfly: after round r a lane keeps the half of its
+      // values whose index bit (4 - r) equals its own lane bit, and adds the
+      // partner's copy of them; at the end lane l holds pair l
 #pragma unroll
-  for (int h = 0; h < kDecodeMaxG; ++h) {
-    if (h < G) {
-      x[h] = valid ? x[h] * p.scale_log2 : -INFINITY;
-      if (valid) lg[static_cast<size_t>(h) * (p.C + 1) + j] = x[h];
-      const float m = warp_max(x[h]);
-      if (lane == 0) wred[h][warp] = m;
-    }
-  }
-  __syncthreads();
-  if (tid < G) {
-    float m = wred[tid][0];
-    for (int w = 1; w < kPartialThreads / 32; ++w) m = fmaxf(m, wred[tid][w]);
-    hstat[tid][0] = m;  // finite: every chunk holds at least one valid key
-  }
-  __syncthreads();
+      for (int r = 0; r < 5; ++r) {
+        const int off = 16 >> r;
+        const bool up = (lane & off) != 0;
 #pragma unroll
-  for (int h = 0; h < kDecodeMaxG; ++h) {
-    if (h < G) {
-      const float pw = valid ? ex2_approx(x[h] - hstat[h][0]) : 0.f;
-      ps[h * kDecodeChunk + tid] = pw;
-      const float s = warp_sum(pw);
-      if (lane == 0) wred[h][warp] = s;
+        for (int i = 0; i < off; ++i) {
+          const float send = up ? v[i] : v[i + off];
+          const float keep = up ? v[i + off] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      const int kl = k0 + lane / G, h = lane % G;
+      const bool valid = kl < nkc;  // rows past the chunk's keys hold stale data
+      if (kl < KC) xs[h * KC + kl] = valid ? v[0] * p.scale_log2 : -INFINITY;
+      if (valid) lg[static_cast<size_t>(h) * (p.C + 1) + j0 + kl] = v[0] * p.scale_log2;
     }
   }
   __syncthreads();
-  if (tid < G) {
-    float s = 0.f;
-    for (int w = 0; w < kPartialThreads / 32; ++w) s += wred[tid][w];
-    hstat[tid][1] = s;
+  // ---- chunk max and sum per head (one warp per head), P into xs
+  if (ok && warp < G) {
+    float m = -INFINITY;
+    for (int k = lane; k < nkc; k += 32) m = fmaxf(m, xs[warp * KC + k]);
+    m = warp_max(m);
+    float l = 0.f;
+    for (int k = lane; k < nkc; k += 32) {
+      const float pw = ex2_approx(xs[warp * KC + k] - m);
+      xs[warp * KC + k] = pw;
+      l += pw;
+    }
+    l = warp_sum(l);
+    if (lane == 0) {
+      hstat[warp][0] = m;
+      hstat[warp][1] = l;
+    }
   }
-
-  // ---- thread = (8 head-dim elements, key group): unnormalised P V
-  const int u = tid % U, kg = tid / U;
-  float o[kDecodeMaxG][8];
+  if (ok && rows > 0) ok = mbar_wait(bV, 0, err, &abort_flag);
+  __syncthreads();
+  // ---- P V: each lane its head-dim slice, warps over the keys
+  float o[G][E];
 #pragma unroll
-  for (int h = 0; h < kDecodeMaxG; ++h)
+  for (int h = 0; h < G; ++h)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) o[h][e] = 0.f;
-  for (int jj = 0; jj < KPG; ++jj) {
-    const int jl = kg * KPG + jj;
-    const int jv = j0 + jl;
-    if (jv >= nk) break;
-    const T* vrow = jv < p.n
-                        ? static_cast<const T*>(p.v_cache) + (static_cast<size_t>(bg) * p.C + jv) * D
-                        : static_cast<const T*>(p.v_new) + static_cast<size_t>(bg) * D;
-    float vf[8];
-    load8(vrow + u * 8, vf);
+    for (int e = 0; e < E; ++e) o[h][e] = 0.f;
+  if (ok) {
+    for (int k = warp; k < nkc; k += kWarps) {
+      float vf[E];
+      lds_row<T, E>(sV + k * L::kRow + lane * E * sizeof(T), vf);
 #pragma unroll
-    for (int h = 0; h < kDecodeMaxG; ++h) {
-      if (h < G) {
-        const float pw = ps[h * kDecodeChunk + jl];
+      for (int h = 0; h < G; ++h) {
+        const float pw = xs[h * KC + k];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[h][e] = fmaf(pw, vf[e], o[h][e]);
+        for (int e = 0; e < E; ++e) o[h][e] = fmaf(pw, vf[e], o[h][e]);
       }
     }
   }
 #pragma unroll
-  for (int h = 0; h < kDecodeMaxG; ++h) {
-    if (h < G) {
-      float4* dst = reinterpret_cast<float4*>(ored + (static_cast<size_t>(kg) * G + h) * D + u * 8);
-      dst[0] = make_float4(o[h][0], o[h][1], o[h][2], o[h][3]);
-      dst[1] = make_float4(o[h][4], o[h][5], o[h][6], o[h][7]);
-    }
-  }
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < E; ++e) ored[(warp * G + h) * D + lane * E + e] = o[h][e];
   __syncthreads();
-  float* part = p.part + (static_cast<size_t>(bg) * p.part_ld + chunk) * G * (D + 2);
-  for (int i = tid; i < G * D; i += kPartialThreads) {
-    float s = 0.f;
-    for (int k = 0; k < KG; ++k) s += ored[static_cast<size_t>(k) * G * D + i];
-    part[(i / D) * (D + 2) + (i % D)] = s;
-  }
-  if (tid < G) {
-    part[tid * (D + 2) + D] = hstat[tid][0];
-    part[tid * (D + 2) + D + 1] = hstat[tid][1];
+  if (ok) {
+    float* part = p.part + (static_cast<size_t>(bg) * p.part_ld + chunk) * G * (D + 2);
+    for (int i = tid; i < G * D; i += kThreads) {
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) s += ored[w * G * D + i];
+      part[(i / D) * (D + 2) + (i % D)] = s;
+    }
+    if (tid < G) {
+      part[tid * (D + 2) + D] = hstat[tid][0];
+      part[tid * (D + 2) + D + 1] = hstat[tid][1];
+    }
+  } else if (tid == 0 && rows > 0) {  // a wait gave up: let the copies land before exit
+    mbar_wait_drain(bK, 0, err);
+    mbar_wait_drain(bV, 0, err);
   }
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kFinishThreads) decode_finish(const DecodeParams p) {
-  __shared__ float fac[kDecodeMaxG][kMaxChunks];   // 2^(chunk max - head max)
-  __shared__ float psum[kDecodeMaxG][kMaxChunks];  // chunk sums
-  __shared__ float mh[kDecodeMaxG], lh[kDecodeMaxG], lse[kDecodeMaxG];
-  __shared__ unsigned long long wmin[kFinishThreads / 32];
+__global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) {
+  __shared__ float fac[kDecodeMaxG][kMaxChunks];  // 2^(chunk max - head max)
+  __shared__ float lse[kDecodeMaxG], lh[kDecodeMaxG];
+  __shared__ unsigned long long wmin[kWarps];
+  __shared__ int is_last;
   const int G = p.G;
-  const int bg = blockIdx.x;
+  const int slice = blockIdx.x;
+  const int bg = blockIdx.y;
   const int b = bg / p.Hkv, g = bg % p.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int NCk = p.n_chunks;
   const int C = p.C, n = p.n;
+  // the CTAs that merge O: all slices when there are few (cache, KV head)
+  // units (latency), else the first only (less repeated work)
+  const int o_slices = p.spread_o ? static_cast<int>(gridDim.x) : 1;
   griddep_wait();  // the partials come from the preceding kernel
   const float* part = p.part + static_cast<size_t>(bg) * p.part_ld * G * (D + 2);
   auto pidx = [&](int c, int h) { return (static_cast<size_t>(c) * G + h) * (D + 2); };
 
-  // ---- merge the chunks: chunk maxima and sums into shared memory, then
-  // one warp per head reduces them (fixed tree order)
-  for (int i = tid; i < NCk * G; i += kFinishThreads) {
-    const int c = i / G, h = i % G;
-    fac[h][c] = part[pidx(c, h) + D];       // chunk max, turned into the factor below
-    psum[h][c] = part[pidx(c, h) + D + 1];  // chunk sum
-  }
-  __syncthreads();
+  // ---- per-head log-sum-exp over the chunks (one warp per head)
   if (warp < G) {
     float m = -INFINITY;
-    for (int c = lane; c < NCk; c += 32) m = fmaxf(m, fac[warp][c]);
+    for (int c = lane; c < NCk; c += 32) m = fmaxf(m, part[pidx(c, warp) + D]);
     m = warp_max(m);
     float l = 0.f;
     for (int c = lane; c < NCk; c += 32) {
-      const float f = ex2_approx(fac[warp][c] - m);
-      fac[warp][c] = f;
-      l = fmaf(psum[warp][c], f, l);
+      const float f = ex2_approx(part[pidx(c, warp) + D] - m);
+      if (slice < o_slices) fac[warp][c] = f;
+      l = fmaf(part[pidx(c, warp) + D + 1], f, l);
     }
     l = warp_sum(l);
     if (lane == 0) {
-      mh[warp] = m;
       lh[warp] = l;
       lse[warp] = m + __log2f(l);
     }
   }
   __syncthreads();
-  T* out = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.Hkv * G + g * G) * D;
-  for (int i = tid; i < G * D; i += kFinishThreads) {
-    const int h = i / D, d = i % D;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < NCk; ++c) acc = fmaf(part[pidx(c, h) + d], fac[h][c], acc);
-    store(out + i, acc / lh[h]);
+  if (slice < o_slices) {  // O: this CTA's share of the G*D outputs, tpo lanes
+                          // per output (chunks strided over them, then a
+                          // fixed butterfly sum)
+    T* out = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.Hkv * G + g * G) * D;
+    const int GD = G * D;
+    const int per = (GD + o_slices - 1) / o_slices;
+    const int o_begin = slice * per, o_end = min(GD, o_begin + per);
+    int tpo = 1;
+    while (tpo < 32 && 2 * tpo * per <= kThreads) tpo *= 2;
+    const int cg = tid % tpo;
+    for (int base = o_begin; base < o_end; base += kThreads / tpo) {
+      const int i = base + tid / tpo;
+      const bool valid = i < o_end;
+      const int h = valid ? i / D : 0, d = valid ? i % D : 0;
+      float acc = 0.f;
+      if (valid) {
+#pragma unroll 4
+        for (int c = cg; c < NCk; c += tpo) acc = fmaf(part[pidx(c, h) + d], fac[h][c], acc);
+      }
+      for (int o = tpo / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (valid && cg == 0) store(out + i, acc / lh[h]);
+    }
   }
 
-  // ---- summed weights: slots, zeros up to C, the new key at C
+  // ---- summed weights of this slice's keys: slots, then the new key at C
   const float* lg = p.logits + static_cast<size_t>(bg) * G * (C + 1);
   float* cs = p.colsum + static_cast<size_t>(bg) * p.colsum_ld;
+  const int ja = slice * kDecodeSliceKeys;
+  const int jb = min(n + 1, ja + kDecodeSliceKeys);
 #pragma unroll 4
-  for (int j = tid; j <= n; j += kFinishThreads) {
+  for (int j = ja + tid; j < jb; j += kThreads) {
     float s = 0.f;
     for (int h = 0; h < G; ++h) s += ex2_approx(lg[static_cast<size_t>(h) * (C + 1) + j] - lse[h]);
     cs[j < n ? j : C] = s;
   }
-  for (int j = n + tid; j < C; j += kFinishThreads) cs[j] = 0.f;
+  const bool last_slice = slice == static_cast<int>(gridDim.x) - 1;
+  if (last_slice)  // empty slots received nothing
+    for (int j = n + tid; j < C; j += kThreads) cs[j] = 0.f;
   if (!p.evict) return;
 
-  // ---- eviction of one candidate
-  __syncthreads();  // the row of summed weights is complete
+  // ---- eviction
+  __syncthreads();  // this CTA's summed weights are written
+  const bool by_score = p.policy == kPolicyH2O;
+  const int sinks = p.policy == kPolicySLR ? p.sinks : 0;
   float* score = p.scores + static_cast<size_t>(bg) * C;
   int* pos = p.pos + static_cast<size_t>(bg) * C;
-  const float cnew = cs[C];
   const size_t row_bytes = static_cast<size_t>(D) * sizeof(T);
   char* kc = static_cast<char*>(p.k_cache) + static_cast<size_t>(bg) * C * row_bytes;
   char* vc = static_cast<char*>(p.v_cache) + static_cast<size_t>(bg) * C * row_bytes;
   const char* kn = static_cast<const char*>(p.k_new) + static_cast<size_t>(bg) * row_bytes;
   const char* vn = static_cast<const char*>(p.v_new) + static_cast<size_t>(bg) * row_bytes;
-  if (bg == 0 && tid == 0) {
+  if (bg == 0 && slice == 0 && tid == 0) {
     p.state[0] = min(C, n + 1);
     p.state[1] = p.t0 + 1;
   }
-  const bool by_score = p.policy == kPolicyH2O;
-  const int sinks = p.policy == kPolicySLR ? p.sinks : 0;
-  const float snew = by_score ? cnew : 0.f;  // the score-free policies keep none
-  if (n < C) {  // room left: the new token takes slot n
+  const int sa = ja, sb = min(jb, n);  // this slice's valid slots
+  if (n < C) {  // room left: the new token takes slot n (key n is in the last slice)
     if (by_score)
-      for (int s = tid; s < n; s += kFinishThreads) score[s] = __fadd_rn(score[s], cs[s]);
-    if (tid == 0) {
-      score[n] = snew;
-      pos[n] = p.t0;
-    }
-    if (warp == 0) {
-      copy_row(kc + n * row_bytes, kn, static_cast<int>(row_bytes), lane);
-      copy_row(vc + n * row_bytes, vn, static_cast<int>(row_bytes), lane);
+      for (int s = sa + tid; s < sb; s += kThreads) score[s] = __fadd_rn(score[s], cs[s]);
+    if (last_slice) {
+      if (tid == 0) {
+        score[n] = by_score ? cs[C] : 0.f;
+        pos[n] = p.t0;
+      }
+      if (warp == 0) {
+        copy_row(kc + n * row_bytes, kn, static_cast<int>(row_bytes), lane);
+        copy_row(vc + n * row_bytes, vn, static_cast<int>(row_bytes), lane);
+      }
     }
     return;
   }
-  // full: candidates with position < t0 + 1 - W (and, under SLR, >= the sink
-  // count) are unprotected; the one with the lowest rank value (then the
-  // highest index: slot s -> s, new token -> C) leaves.  The rank value is the
-  // score (>= 0, so its bit pattern orders like the value) or, for the
-  // score-free policies, the position.
+  // full: this slice's candidate.  Unprotected: position < t0 + 1 - W (and,
+  // under SLR, >= the sink count).  Key: rank value (score bits -- scores are
+  // >= 0 -- or position) then the inverted index, so that the minimum is the
+  // lowest value with the highest index.
   const long long limit = static_cast<long long>(p.t0) + 1 - p.W;
   unsigned long long best = ~0ull;
-  for (int s = tid; s < C; s += kFinishThreads) {
+  for (int s = sa + tid; s < sb; s += kThreads) {
     const int ps = pos[s];
     uint32_t rank;
     if (by_score) {
@@ -331,58 +410,74 @@ __global__ void __launch_bounds__(kFinishThreads) decode_finish(const DecodePara
       best = key < best ? key : best;
     }
   }
-  if (tid == 0 && p.t0 < limit && p.t0 >= sinks) {  // W = 0: the new token competes too
-    const uint32_t rank = by_score ? __float_as_uint(cnew) : static_cast<uint32_t>(p.t0);
+  if (last_slice && tid == 0 && p.t0 < limit && p.t0 >= sinks) {  // W = 0: the new token competes
+    const uint32_t rank = by_score ? __float_as_uint(cs[C]) : static_cast<uint32_t>(p.t0);
     const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - C);
     best = key < best ? key : best;
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-    best = other < best ? other : best;
-  }
+  best = warp_min64(best);
   if (lane == 0) wmin[warp] = best;
   __syncthreads();
-  if (warp == 0) {
-    best = lane < kFinishThreads / 32 ? wmin[lane] : ~0ull;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-      best = other < best ? other : best;
-    }
-    if (best == ~0ull) {  // cannot happen: W <= C leaves an unprotected candidate
-      if (lane == 0) atomicOr(&p.state[2], kDevErrPlan);
-      return;
-    }
-    const int e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(best & 0xffffffffu));
-    if (e < C) {  // an old slot leaves; the new token takes it
-      if (lane == 0) {
-        score[e] = snew;
-        pos[e] = p.t0;
-      }
-      copy_row(kc + static_cast<size_t>(e) * row_bytes, kn, static_cast<int>(row_bytes), lane);
-      copy_row(vc + static_cast<size_t>(e) * row_bytes, vn, static_cast<int>(row_bytes), lane);
-    }
+  if (tid == 0) {
+    unsigned long long m = wmin[0];
+    for (int w = 1; w < kWarps; ++w) m = wmin[w] < m ? wmin[w] : m;
+    p.best[static_cast<size_t>(bg) * p.slices_ld + slice] = m;
+    __threadfence();  // candidate, scores and summed weights before the ticket
+    is_last = atomicAdd(&p.ticket[bg], 1) == static_cast<int>(gridDim.x) - 1;
   }
+  __syncthreads();
+  if (!is_last || warp != 0) return;
+  // the last CTA of this (cache, KV head): every slice's writes are visible
+  __threadfence();
+  unsigned long long m = ~0ull;
+  for (int sl = lane; sl < static_cast<int>(gridDim.x); sl += 32) {
+    const unsigned long long v = __ldcg(&p.best[static_cast<size_t>(bg) * p.slices_ld + sl]);
+    m = v < m ? v : m;
+  }
+  m = warp_min64(m);
+  if (lane == 0) p.ticket[bg] = 0;  // ready for the next step
+  if (m == ~0ull) {  // cannot happen: W + sinks <= C leaves an unprotected candidate
+    if (lane == 0) atomicOr(&p.state[2], kDevErrPlan);
+    return;
+  }
+  const int e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(m & 0xffffffffu));
+  if (e < C) {  // an old slot leaves; the new token takes it
+    if (lane == 0) {
+      score[e] = by_score ? __ldcg(&cs[C]) : 0.f;
+      pos[e] = p.t0;
+    }
+    copy_row(kc + static_cast<size_t>(e) * row_bytes, kn, static_cast<int>(row_bytes), lane);
+    copy_row(vc + static_cast<size_t>(e) * row_bytes, vn, static_cast<int>(row_bytes), lane);
+  }
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_partial(const DecodeParams& p, cudaStream_t st) {
+  using L = PartialLayout<T, D, G>;
+  static int attr_bits[2] = {0, 0};
+  if (!smem_attr_done(reinterpret_cast<const void*>(decode_partial<T, D, G>), attr_bits)) {
+    cudaError_t e = cudaFuncSetAttribute(decode_partial<T, D, G>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+    if (e != cudaSuccess) return e;
+  }
+  decode_partial<T, D, G><<<dim3(p.n_chunks, p.B * p.Hkv), kThreads, L::kBytes, st>>>(p);
+  return cudaGetLastError();
 }
 
 template <typename T, int D>
 cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
-  constexpr int U = D / 8, KG = kPartialThreads / U;
-  const size_t smem = static_cast<size_t>(p.G) * (D + kDecodeChunk + KG * D) * sizeof(float);
-  static int attr_bits[2] = {0, 0};
-  if (!smem_attr_done(reinterpret_cast<const void*>(decode_partial<T, D>), attr_bits)) {
-    const int most = kDecodeMaxG * (D + kDecodeChunk + KG * D) * static_cast<int>(sizeof(float));
-    cudaError_t e = cudaFuncSetAttribute(decode_partial<T, D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, most);
-    if (e != cudaSuccess) return e;
+  cudaError_t e;
+  switch (p.G) {
+    case 1: e = launch_partial<T, D, 1>(p, st); break;
+    case 2: e = launch_partial<T, D, 2>(p, st); break;
+    case 4: e = launch_partial<T, D, 4>(p, st); break;
+    case 8: e = launch_partial<T, D, 8>(p, st); break;
+    default: return cudaErrorInvalidValue;
   }
-  decode_partial<T, D><<<dim3(p.n_chunks, p.B * p.Hkv), kPartialThreads, smem, st>>>(p);
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.B * p.Hkv);
-  cfg.blockDim = dim3(kFinishThreads);
+  cfg.gridDim = dim3(p.n_slices, p.B * p.Hkv);
+  cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -395,8 +490,11 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
 
 }  // namespace
 
+bool decode_supported(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
+
 cudaError_t launch_decode(const DecodeParams& p, int esize, int head_dim, cudaStream_t st) {
-  if (p.n_chunks > kMaxChunks || p.G > kDecodeMaxG) return cudaErrorInvalidValue;
+  if (p.n_chunks > kMaxChunks || !decode_supported(p.G) || p.n_slices > p.slices_ld)
+    return cudaErrorInvalidValue;
   if (esize == 2)
     return head_dim == 128 ? launch<__nv_bfloat16, 128>(p, st) : launch<__nv_bfloat16, 64>(p, st);
   return head_dim == 128 ? launch<float, 128>(p, st) : launch<float, 64>(p, st);

@@ -38,6 +38,9 @@ struct h2o_cache {
   float* dec_logits = nullptr;  // decode: [B*Hkv, G, C + 1]
   float* dec_part = nullptr;    // decode: [B*Hkv, dec_part_ld, G, d + 2]
   int dec_part_ld = 0;
+  unsigned long long* dec_best = nullptr;  // decode: [B*Hkv, dec_slices_ld]
+  int* dec_ticket = nullptr;               // decode: [B*Hkv], zero between steps
+  int dec_slices_ld = 0;
   // h2o_chunk_step_host: two staging sets, used by alternate calls, so the
   // copies of one call overlap the kernels of its neighbours.  The copies run
   // on two internal streams (one per direction); events order them with the
@@ -67,8 +70,9 @@ size_t esize_of(h2o_dtype t) { return t == H2O_BF16 ? 2 : 4; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct Layout {
-  size_t lse, colsum, slots, tokens, count, dlog, dpart, sq[2], skn[2], svn[2], sout[2], total;
-  int nq_pad, colsum_ld, dpart_ld;
+  size_t lse, colsum, slots, tokens, count, dlog, dpart, dbest, dticket, sq[2], skn[2], svn[2],
+      sout[2], total;
+  int nq_pad, colsum_ld, dpart_ld, dslices_ld;
 };
 
 Layout workspace_layout(const h2o_config& c) {
@@ -90,10 +94,13 @@ Layout workspace_layout(const h2o_config& c) {
   L.count = take(BHkv * 4);
   // decode steps (n_q = 1): stored logits and the split-KV partials
   const size_t G = static_cast<size_t>(c.n_q_heads / c.n_kv_heads);
-  L.dpart_ld = cdiv(c.capacity + 1, kDecodeChunk);
-  const bool dec = G <= static_cast<size_t>(kDecodeMaxG);
+  L.dpart_ld = cdiv(c.capacity + 1, decode_chunk_keys(c.head_dim, static_cast<int>(esize_of(c.dtype))));
+  L.dslices_ld = cdiv(c.capacity + 1, kDecodeSliceKeys);
+  const bool dec = decode_supported(static_cast<int>(G));
   L.dlog = take(dec ? BHkv * G * (static_cast<size_t>(c.capacity) + 1) * 4 : 0);
   L.dpart = take(dec ? BHkv * L.dpart_ld * G * (c.head_dim + 2) * 4 : 0);
+  L.dbest = take(dec ? BHkv * L.dslices_ld * 8 : 0);
+  L.dticket = take(dec ? BHkv * 4 : 0);
   const size_t rows = static_cast<size_t>(c.batch) * c.max_chunk * c.head_dim * e;
   for (int i = 0; i < 2; ++i) {
     L.sq[i] = take(rows * c.n_q_heads);
@@ -296,7 +303,7 @@ h2o_status run_evict(h2o_cache* c, const float* colsum, int ld, const void* kn, 
 }
 
 bool decode_path(const h2o_cache* c, int nq) {
-  return nq == 1 && c->cfg.n_q_heads / c->cfg.n_kv_heads <= kDecodeMaxG;
+  return nq == 1 && decode_supported(c->cfg.n_q_heads / c->cfg.n_kv_heads);
 }
 
 // The step for one new token per cache (decode.cu): split-KV attention with
@@ -313,8 +320,18 @@ h2o_status run_decode(h2o_cache* c, const void* q, const void* kn, const void* v
   d.n = c->n;
   d.t0 = c->t0;
   d.W = g.recent_window;
-  d.n_chunks = cdiv(c->n + 1, kDecodeChunk);
+  d.n_chunks = cdiv(c->n + 1, decode_chunk_keys(g.head_dim, static_cast<int>(esize_of(g.dtype))));
   d.part_ld = c->dec_part_ld;
+  d.n_slices = cdiv(c->n + 1, kDecodeSliceKeys);
+  d.slices_ld = c->dec_slices_ld;
+  d.best = c->dec_best;
+  d.ticket = c->dec_ticket;
+  // few (cache, KV head) units leave SMs idle: then every merge CTA takes
+  // part of O, else only the first of each unit does
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  d.spread_o = g.batch * g.n_kv_heads < sms ? 1 : 0;
   const float scale = g.softmax_scale > 0.f ? g.softmax_scale : 1.f / sqrtf((float)g.head_dim);
   d.scale_log2 = scale * 1.4426950408889634f;
   d.q = q;
@@ -431,6 +448,9 @@ h2o_status h2o_cache_create(const h2o_config* cfg, const h2o_buffers* bufs, void
   c->dec_logits = reinterpret_cast<float*>(ws + L.dlog);
   c->dec_part = reinterpret_cast<float*>(ws + L.dpart);
   c->dec_part_ld = L.dpart_ld;
+  c->dec_best = reinterpret_cast<unsigned long long*>(ws + L.dbest);
+  c->dec_ticket = reinterpret_cast<int*>(ws + L.dticket);
+  c->dec_slices_ld = L.dslices_ld;
   for (int i = 0; i < 2; ++i) {
     c->stage_q[i] = ws + L.sq[i];
     c->stage_kn[i] = ws + L.skn[i];
@@ -450,6 +470,9 @@ h2o_status h2o_cache_create(const h2o_config* cfg, const h2o_buffers* bufs, void
   if (e == cudaSuccess) e = cudaMemsetAsync(bufs->scores, 0, sz.scores_bytes, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(bufs->pos, 0xFF, sz.pos_bytes, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(bufs->state, 0, sz.state_bytes, st);
+  // the decode merge's completion tickets start at zero (each step leaves them so)
+  if (e == cudaSuccess && decode_supported(cfg->n_q_heads / cfg->n_kv_heads))
+    e = cudaMemsetAsync(ws + L.dticket, 0, static_cast<size_t>(cfg->batch) * cfg->n_kv_heads * 4, st);
   if (e != cudaSuccess) {
     delete c;
     return H2O_ERR_CUDA;
