@@ -112,6 +112,55 @@ def attention_one_cache(q: np.ndarray, kc: np.ndarray, vc: np.ndarray, n: int,
     return o, colsum, lse
 
 
+def attention_backward_one_cache(q: np.ndarray, kc: np.ndarray, vc: np.ndarray, n: int,
+                                 kn: np.ndarray, vn: np.ndarray, do: np.ndarray,
+                                 scale: float):
+    """Gradients of the attention output O of ``attention_one_cache`` with
+    respect to its inputs, for one cache, given dO = dL/dO [n_q, H_q, d].
+
+    The cache contents and the visibility are held fixed: the eviction that
+    follows the attention in a step is a discrete decision and is not
+    differentiated (the paper trains through the cache with its policy in
+    place, summary page, Tables 1 and 6).  For query head h of KV head g, over
+    its visible keys:  P = softmax(scale q k^T);  dV_g += P^T dO_h;
+    dP = dO_h V^T;  dS = P * (dP - rowsum(P * dP)) (the softmax Jacobian);
+    dq_h = scale dS K;  dK_g += scale dS^T q_h.
+
+    Returns (dq [n_q, H_q, d], dkc [H_kv, C, d], dvc [H_kv, C, d],
+    dkn [n_q, H_kv, d], dvn [n_q, H_kv, d]); rows of dkc, dvc past the n
+    valid slots are 0.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    n_q, H_q, d = q.shape
+    H_kv, C, _ = kc.shape
+    G = H_q // H_kv
+    dq = np.zeros_like(q)
+    dkc = np.zeros((H_kv, C, d))
+    dvc = np.zeros((H_kv, C, d))
+    dkn = np.zeros((n_q, H_kv, d))
+    dvn = np.zeros((n_q, H_kv, d))
+    vis = visible_mask(n, n_q)
+    for h in range(H_q):
+        g = kv_head_of(h, G)
+        keys = np.concatenate([kc[g, :n], kn[:, g]], axis=0)       # [n + n_q, d]
+        vals = np.concatenate([vc[g, :n], vn[:, g]], axis=0)
+        s = scale * (q[:, h, :] @ keys.T)
+        s = np.where(vis, s, -np.inf)
+        e = np.exp(s - s.max(axis=1, keepdims=True))
+        p = e / e.sum(axis=1, keepdims=True)                       # [n_q, n + n_q]
+        dv = p.T @ do[:, h, :]
+        dp = do[:, h, :] @ vals.T
+        ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+        dq[:, h, :] = scale * (ds @ keys)
+        dk = scale * (ds.T @ q[:, h, :])
+        dkc[g, :n] += dk[:n]
+        dvc[g, :n] += dv[:n]
+        dkn[:, g] += dk[n:]
+        dvn[:, g] += dv[n:]
+    return dq, dkc, dvc, dkn, dvn
+
+
 # --------------------------------------------------------------------------
 # score accumulation, selection and placement (one cache, one KV head)
 # --------------------------------------------------------------------------
@@ -238,6 +287,22 @@ class OracleCache:
             O[b], colsum[b], lse[b] = attention_one_cache(
                 Q[b], self.K[b], self.V[b], self.n, Kn[b], Vn[b], self.scale)
         return O, colsum, lse
+
+    def attention_backward(self, Q, Kn, Vn, dO):
+        """Gradients of ``attention``'s O for the current state (before the
+        eviction of the same step): (dQ, dK_cache, dV_cache, dK_new, dV_new)
+        with the layouts of Q [B, n_q, H_q, d], the cache [B, H_kv, C, d] and
+        Kn [B, n_q, H_kv, d]."""
+        Q, Kn, Vn, dO = (np.asarray(x, dtype=np.float64) for x in (Q, Kn, Vn, dO))
+        B = Q.shape[0]
+        outs = [np.zeros_like(Q), np.zeros_like(self.K), np.zeros_like(self.V),
+                np.zeros_like(Kn), np.zeros_like(Vn)]
+        for b in range(B):
+            r = attention_backward_one_cache(Q[b], self.K[b], self.V[b], self.n, Kn[b], Vn[b],
+                                             dO[b], self.scale)
+            for o, x in zip(outs, r):
+                o[b] = x
+        return tuple(outs)
 
     def evict(self, colsum32, Kn, Vn):
         """Apply the score update, selection and placement with the given fp32
