@@ -186,6 +186,26 @@ H2O_API h2o_status h2o_attention(h2o_cache* c, const void* q, const void* k_new,
                          const void* v_new, int32_t n_q, void* out,
                          float* colsum_out, void* stream);
 
+/* Backward of h2o_attention for fine-tuning through the cache: the
+ * gradients of O with respect to q, the cache's K and V and the chunk's
+ * k_new and v_new, with the cache contents and visibility held fixed (the
+ * eviction that follows is a discrete decision and is not differentiated).
+ * Call it after h2o_attention with the same q, k_new, v_new, n_q and before
+ * anything changes the cache (h2o_evict, a step, h2o_cache_write); it reads
+ * that call's row statistics from the workspace (else H2O_ERR_STATE).
+ * out, d_out: device [batch, n_q, H_q, d] bf16 (O of that call and dL/dO).
+ * Outputs, device float32, 16-byte aligned: dq [batch, n_q, H_q, d];
+ * dk_cache, dv_cache [batch, H_kv, C, d] (rows of slots >= n are zero);
+ * dk_new, dv_new [batch, n_q, H_kv, d].  BF16 caches only (else
+ * H2O_ERR_DTYPE); n_q >= 2 (a one-token h2o_attention runs the decode
+ * kernels, which keep no row statistics).  Deterministic (fixed reduction
+ * order). */
+H2O_API h2o_status h2o_attention_backward(h2o_cache* c, const void* q, const void* k_new,
+                                          const void* v_new, int32_t n_q, const void* out,
+                                          const void* d_out, float* dq, float* dk_cache,
+                                          float* dv_cache, float* dk_new, float* dv_new,
+                                          void* stream);
+
 /* Steps 3-5 only, with caller-supplied summed weights `colsum` (device,
  * colsum layout for this n_q, float32).  Advances n and t0. */
 H2O_API h2o_status h2o_evict(h2o_cache* c, const float* colsum, const void* k_new,

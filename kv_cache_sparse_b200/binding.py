@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "H2O_OK", 1: "H2O_ERR_INVALID_ARG", 2: "H2O_ERR_SHAPE", 3: "H
                 4: "H2O_ERR_ALIGN", 5: "H2O_ERR_CUDA", 6: "H2O_ERR_TIMEOUT", 7: "H2O_ERR_STATE"}
 
 EXPORTED = ["h2o_required_bytes", "h2o_cache_create", "h2o_chunk_step", "h2o_chunk_step_host",
-            "h2o_cache_host_join", "h2o_attention", "h2o_evict", "h2o_cache_read", "h2o_cache_write",
+            "h2o_cache_host_join", "h2o_attention", "h2o_attention_backward", "h2o_evict", "h2o_cache_read", "h2o_cache_write",
             "h2o_cache_check", "h2o_cache_info", "h2o_cache_set_timing", "h2o_cache_kernel_ms",
             "h2o_cache_destroy", "h2o_status_string"]
 
@@ -237,6 +237,25 @@ class H2OCache:
             self._h, _ptr(q), _ptr(k_new), _ptr(v_new), n_q, _ptr(out), _ptr(colsum),
             _stream(stream)))
         return out, colsum
+
+    def attention_backward(self, q, k_new, v_new, out, d_out, stream=None):
+        """Gradients of ``attention``'s O (call it right after ``attention``
+        with the same inputs, before the cache changes): returns float32
+        (dq, dk_cache, dv_cache, dk_new, dv_new)."""
+        n_q = self._check_inputs(q, k_new, v_new)
+        s = self.shape
+        f = dict(dtype=torch.float32, device=self.device)
+        dq = torch.empty(s.batch, n_q, s.n_q_heads, s.head_dim, **f)
+        dkc = torch.empty(s.batch, s.n_kv_heads, s.capacity, s.head_dim, **f)
+        dvc = torch.empty_like(dkc)
+        dkn = torch.empty(s.batch, n_q, s.n_kv_heads, s.head_dim, **f)
+        dvn = torch.empty_like(dkn)
+        out = out.contiguous()
+        d_out = d_out.to(device=self.device, dtype=s.dtype).contiguous()
+        _check("h2o_attention_backward", lib().h2o_attention_backward(
+            self._h, _ptr(q), _ptr(k_new), _ptr(v_new), n_q, _ptr(out), _ptr(d_out), _ptr(dq),
+            _ptr(dkc), _ptr(dvc), _ptr(dkn), _ptr(dvn), _stream(stream)))
+        return dq, dkc, dvc, dkn, dvn
 
     def evict(self, colsum, k_new, v_new, stream=None):
         n_q = k_new.shape[1]

@@ -17,6 +17,11 @@ struct AttnMaps {
   CUtensorMap vn;
 };
 
+// TMA descriptors of a backward call: AttnMaps plus dO (layout of q).
+struct BwdMaps {
+  CUtensorMap q, dout, kc, vc, kn, vn;
+};
+
 // Records that a kernel's shared-memory opt-in was set on the current device.
 bool smem_attr_done(const void* fn, int* slot_bits);
 
@@ -37,6 +42,11 @@ cudaError_t launch_attn_f32(int head_dim, const float* q, const float* kc, const
 cudaError_t launch_decode(const DecodeParams& p, int esize, int head_dim, cudaStream_t st);
 // Group sizes the decode kernels take (a warp batch holds 32 / G keys).
 bool decode_supported(int G);
+
+// Backward of the attention (bf16, head_dim 64 or 128): D_i, then dK/dV and
+// dQ; out and dout are [B, nq, Hq, d] bf16.
+cudaError_t launch_attn_bwd_bf16(int head_dim, const BwdMaps& m, const BwdParams& p,
+                                 const void* out, const void* dout, cudaStream_t st);
 
 // K3 (with the K/V scatter fused): score update, selection, placement.
 cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st);

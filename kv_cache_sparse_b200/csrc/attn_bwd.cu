@@ -1,0 +1,607 @@
+// attn_bwd.cu -- backward of the chunk step's attention on sm_100a tensor
+// cores: dQ, dK and dV for the cache slots and the chunk's keys, with the
+// eviction decision held fixed ("Learning how to Forget", §1: fine-tuning
+// through the KV cache with the policy in place; summary page, Tables 1 and
+// 6: training with each cache policy).
+//
+// With P = softmax(scale Q K^T) over the visible keys (the forward's row
+// statistic lse2 rebuilds it: P = 2^(x - lse2), x = scale*log2(e)*<q, k>),
+//   dV = P^T dO,  dP = dO V^T,  dS = P (dP - D) with D_i = <dO_i, O_i>,
+//   dQ = scale dS K,  dK = scale dS^T Q,
+// dK and dV summed over the G query heads of a KV head.  Three kernels:
+//   bwd_rowdot   D_i for every (cache, head, query): one warp per row.
+//   bwd_dkdv     key-stationary, like the column-sum kernel: one CTA per
+//                (cache, KV head, 128 keys), looping over the (head, query
+//                tile) units that see its keys.  The MMAs compute
+//                S^T = K Q^T and dP^T = V dO^T with the keys on the TMEM
+//                lanes; one thread per key turns its rows into P^T and
+//                scale*dS^T (bf16, written back over the first columns of S^T
+//                and dP^T), and the MMAs accumulate dV += P^T dO and
+//                dK += dS^T Q in TMEM (A operand from TMEM, B the dO / Q tile
+//                as an MN-major operand).
+//   bwd_dq       query-stationary, like the forward: one CTA per (cache,
+//                head, 128 queries), looping over the key tiles it sees:
+//                S = Q K^T, dP = dO V^T, one thread per query row forms
+//                scale*dS (bf16, over S), and dQ += dS K accumulates in TMEM.
+// Every reduction has a fixed order (no atomics): the results are
+// deterministic.  Roles in the two tensor-core kernels: warp 0 TMA producer,
+// warp 1 TMEM allocation and the MMA-issuing thread, warps 2..5 the rows.
+#include <cuda_bf16.h>
+
+#include "attn.h"
+#include "sm100.cuh"
+
+namespace h2o {
+
+// ---------------------------------------------------------------- D_i
+
+__global__ void bwd_rowdot(const __nv_bfloat16* __restrict__ out,
+                           const __nv_bfloat16* __restrict__ dout, const BwdParams p, int d) {
+  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);  // (b, i, h)
+  const int lane = threadIdx.x & 31;
+  const int rows = p.B * p.nq * p.Hq;
+  if (row >= rows) return;
+  const __nv_bfloat16* o = out + static_cast<size_t>(row) * d;
+  const __nv_bfloat16* g = dout + static_cast<size_t>(row) * d;
+  float s = 0.f;
+  for (int e = lane; e < d; e += 32) s = fmaf(__bfloat162float(o[e]), __bfloat162float(g[e]), s);
+#pragma unroll
+  for (int o2 = 16; o2 > 0; o2 >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o2);
+  if (lane == 0) {
+    const int h = row % p.Hq;
+    const int i = (row / p.Hq) % p.nq;
+    const int b = row / (p.Hq * p.nq);
+    p.dsum[(static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + i] = s;
+  }
+}
+
+// ---------------------------------------------------------------- dK, dV
+
+template <int D>
+struct DkdvLayout {
+  static constexpr int kRegions = D / 64;
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kStages = 2;  // units in flight (Q, dO, lse2, D)
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kKOff + kTileBytes;
+  static constexpr int kQOff = kVOff + kTileBytes;                  // [stage]
+  static constexpr int kDOOff = kQOff + kStages * kTileBytes;       // [stage]
+  static constexpr int kRowOff = kDOOff + kStages * kTileBytes;     // [stage][2][128] float
+  static constexpr int kBarOff = kRowOff + kStages * 1024;
+  // kv_full, u_full[S], u_empty[S], s_full, p_full, o_done, drain
+  static constexpr int kNumBars = 1 + 2 * kStages + 4;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr int kThreads = 192;
+};
+
+// Row arithmetic shared by the two kernels: from 32 logits s and 32 dP
+// values of one row (or one key), the bf16 pairs of P and of scale * dS.
+// nls[c] = -lse2 of the query of column c (or of the row), dv[c] = its D.
+template <bool kMask>
+__device__ __forceinline__ void p_ds_32(const uint32_t (&s)[32], const uint32_t (&dp)[32],
+                                        const float* nls, const float* dv, float c, float scale,
+                                        int first_valid, int last_valid, uint32_t (&pp)[16],
+                                        uint32_t (&dd)[16]) {
+#pragma unroll
+  for (int k = 0; k < 32; k += 2) {
+    float p0 = ex2_approx(fmaf(__uint_as_float(s[k]), c, nls[k]));
+    float p1 = ex2_approx(fmaf(__uint_as_float(s[k + 1]), c, nls[k + 1]));
+    if (kMask) {
+      p0 = (k >= first_valid && k <= last_valid) ? p0 : 0.f;
+      p1 = (k + 1 >= first_valid && k + 1 <= last_valid) ? p1 : 0.f;
+    }
+    // P = 0 (masked, padding or underflow) gives dS = 0 whatever D holds
+    const float d0 = p0 != 0.f ? p0 * (__uint_as_float(dp[k]) - dv[k]) * scale : 0.f;
+    const float d1 = p1 != 0.f ? p1 * (__uint_as_float(dp[k + 1]) - dv[k + 1]) * scale : 0.f;
+    pp[k >> 1] = pack_bf16x2(p0, p1);
+    dd[k >> 1] = pack_bf16x2(d0, d1);
+  }
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    bwd_dkdv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+             const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
+             const __grid_constant__ CUtensorMap tm_kn, const __grid_constant__ CUtensorMap tm_vn,
+             const BwdParams p) {
+  using L = DkdvLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bg = blockIdx.y;
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  const int NCTC = cdiv(p.C, 128);
+  const int NQT = cdiv(p.nq, 128);
+  const bool is_chunk = static_cast<int>(blockIdx.x) >= NCTC;
+  const int kt = is_chunk ? blockIdx.x - NCTC : blockIdx.x;
+  const int j0 = kt * 128;
+  const size_t row_stride = static_cast<size_t>(D);
+  if (!is_chunk && j0 >= p.n) {
+    // slots past the valid ones have no gradient
+    for (int r = threadIdx.x; r < min(128, p.C - j0) * D; r += blockDim.x) {
+      const size_t at = (static_cast<size_t>(bg) * p.C + j0) * row_stride + r;
+      p.dk_cache[at] = 0.f;
+      p.dv_cache[at] = 0.f;
+    }
+    return;
+  }
+  const int qt_min = is_chunk ? kt : 0;
+  const int span = NQT - qt_min;
+  const int R = p.G * span;
+
+  const uint32_t bar_kv = sbase + L::kBarOff;
+  const uint32_t bar_full0 = bar_kv + 8;
+  const uint32_t bar_empty0 = bar_full0 + 8 * L::kStages;
+  const uint32_t bar_s = bar_empty0 + 8 * L::kStages;
+  const uint32_t bar_p = bar_s + 8;
+  const uint32_t bar_o = bar_p + 8;
+  const uint32_t bar_drain = bar_o + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  if (threadIdx.x == 0) {
+    mbar_init(bar_kv, 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar_full0 + 8 * s, 1);
+      mbar_init(bar_empty0 + 8 * s, 1);
+    }
+    mbar_init(bar_s, 1);
+    mbar_init(bar_p, 128);
+    mbar_init(bar_o, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM columns: S^T [0,128), dP^T [128,256), dV [256, 256+D), dK [384, 384+D)
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_kv, 2 * L::kTileBytes);
+      for (int r = 0; r < L::kRegions; ++r) {
+        if (is_chunk) {
+          tma_load_4d(sbase + L::kKOff + r * 16384, &tm_kn, bar_kv, r * 64, g, j0, b);
+          tma_load_4d(sbase + L::kVOff + r * 16384, &tm_vn, bar_kv, r * 64, g, j0, b);
+        } else {
+          tma_load_3d(sbase + L::kKOff + r * 16384, &tm_kc, bar_kv, r * 64, j0, bg);
+          tma_load_3d(sbase + L::kVOff + r * 16384, &tm_vc, bar_kv, r * 64, j0, bg);
+        }
+      }
+      int issued = 0;
+      for (int u = 0; u < R; ++u) {
+        const int h = g * p.G + u / span;
+        const int qt = qt_min + u % span;
+        const int s = u % L::kStages;
+        if (u >= L::kStages &&
+            !mbar_wait(bar_empty0 + 8 * s, ((u / L::kStages) + 1) & 1, p.err, abort_flag))
+          break;
+        const uint32_t full = bar_full0 + 8 * s;
+        mbar_arrive_expect_tx(full, 2 * L::kTileBytes + 1024);
+        for (int r = 0; r < L::kRegions; ++r) {
+          tma_load_4d(sbase + L::kQOff + s * L::kTileBytes + r * 16384, &tm_q, full, r * 64, h,
+                      qt * 128, b);
+          tma_load_4d(sbase + L::kDOOff + s * L::kTileBytes + r * 16384, &tm_do, full, r * 64, h,
+                      qt * 128, b);
+        }
+        const size_t roff = (static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + qt * 128;
+        bulk_load(sbase + L::kRowOff + s * 1024, p.nlse2 + roff, 512, full);
+        bulk_load(sbase + L::kRowOff + s * 1024 + 512, p.dsum + roff, 512, full);
+        issued = u + 1;
+      }
+      mbar_wait_drain(bar_kv, 0, p.err);
+      for (int u = (issued > L::kStages ? issued - L::kStages : 0); u < issued; ++u)
+        mbar_wait_drain(bar_full0 + 8 * (u % L::kStages), (u / L::kStages) & 1, p.err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, false, true);
+      bool ok = mbar_wait(bar_kv, 0, p.err, abort_flag);
+      for (int u = 0; u < R && ok; ++u) {
+        const int s = u % L::kStages;
+        ok = mbar_wait(bar_full0 + 8 * s, (u / L::kStages) & 1, p.err, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t qb = sbase + L::kQOff + s * L::kTileBytes;
+        const uint32_t db = sbase + L::kDOOff + s * L::kTileBytes;
+        // S^T = K Q^T, dP^T = V dO^T (contraction over the head dim)
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_bf16_ss(tmem, sw128_desc(sbase + L::kKOff + off, 16, 1024), sw128_desc(qb + off, 16, 1024),
+                      kIdescS, ks > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_bf16_ss(tmem + 128, sw128_desc(sbase + L::kVOff + off, 16, 1024),
+                      sw128_desc(db + off, 16, 1024), kIdescS, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_s);
+        ok = mbar_wait(bar_p, u & 1, p.err, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        // dV += P^T dO and dK += (scale dS)^T Q (contraction over the 128
+        // queries, 16 per MMA = 8 TMEM columns of bf16 pairs)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          mma_bf16_ts(tmem + 256, tmem + 8 * ks, sw128_desc(db + ks * 2048, 16384, 1024), kIdescAcc,
+                      (u > 0 || ks > 0) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          mma_bf16_ts(tmem + 384, tmem + 128 + 8 * ks, sw128_desc(qb + ks * 2048, 16384, 1024),
+                      kIdescAcc, (u > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(bar_empty0 + 8 * s);
+      }
+      mma_commit(bar_o);
+      mma_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0, p.err);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;  // key j0 + row
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const float c = p.scale_log2, scale = p.scale;
+    bool ok = true;
+    for (int u = 0; u < R; ++u) {
+      const int s = u % L::kStages;
+      ok = mbar_wait(bar_s, u & 1, p.err, abort_flag);
+      if (ok) ok = mbar_wait(bar_full0 + 8 * s, (u / L::kStages) & 1, p.err, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const float* nls = reinterpret_cast<const float*>(smem + L::kRowOff + s * 1024);
+      const float* dvv = nls + 128;
+      const int qt = qt_min + u % span;
+      const bool diag = is_chunk && qt == kt;  // query col sees key row iff row <= col
+#pragma unroll
+      for (int q32 = 0; q32 < 4; ++q32) {
+        uint32_t sv[32], dp[32], pp[16], dd[16];
+        tmem_ld32(lane_base + 32 * q32, sv);
+        tmem_ld32(lane_base + 128 + 32 * q32, dp);
+        tmem_wait_ld();
+        if (diag)
+          p_ds_32<true>(sv, dp, nls + 32 * q32, dvv + 32 * q32, c, scale, row - 32 * q32, 1 << 30,
+                        pp, dd);
+        else
+          p_ds_32<false>(sv, dp, nls + 32 * q32, dvv + 32 * q32, c, scale, 0, 0, pp, dd);
+        // bf16 pairs over the first columns: queries [32 q32, +32) -> [16 q32, +16)
+        tmem_st16(lane_base + 16 * q32, pp);
+        tmem_st16(lane_base + 128 + 16 * q32, dd);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p);
+    }
+    if (ok) {
+      ok = mbar_wait(bar_o, 0, p.err, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const int key = j0 + row;
+      float* dkr = nullptr;
+      float* dvr = nullptr;
+      if (is_chunk) {
+        if (key < p.nq) {
+          const size_t at = ((static_cast<size_t>(b) * p.nq + key) * p.Hkv + g) * row_stride;
+          dkr = p.dk_new + at;
+          dvr = p.dv_new + at;
+        }
+      } else if (key < p.C) {
+        const size_t at = (static_cast<size_t>(bg) * p.C + key) * row_stride;
+        dkr = p.dk_cache + at;
+        dvr = p.dv_cache + at;
+      }
+      const bool valid = is_chunk ? key < p.nq : key < p.n;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t kv[32], vv[32];
+        tmem_ld32(lane_base + 384 + c0, kv);
+        tmem_ld32(lane_base + 256 + c0, vv);
+        tmem_wait_ld();
+        if (dkr) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 k4 = valid ? make_float4(__uint_as_float(kv[e]), __uint_as_float(kv[e + 1]),
+                                                  __uint_as_float(kv[e + 2]), __uint_as_float(kv[e + 3]))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 v4 = valid ? make_float4(__uint_as_float(vv[e]), __uint_as_float(vv[e + 1]),
+                                                  __uint_as_float(vv[e + 2]), __uint_as_float(vv[e + 3]))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4*>(dkr + c0 + e) = k4;
+            *reinterpret_cast<float4*>(dvr + c0 + e) = v4;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- dQ
+
+template <int D>
+struct DqLayout {
+  static constexpr int kRegions = D / 64;
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kStages = 2;
+  static constexpr int kQOff = 0;
+  static constexpr int kDOOff = kQOff + kTileBytes;
+  static constexpr int kKOff = kDOOff + kTileBytes;            // [stage]
+  static constexpr int kVOff = kKOff + kStages * kTileBytes;   // [stage]
+  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  // qd_full, kv_full[S], kv_empty[S], s_full, p_full, o_done, drain
+  static constexpr int kNumBars = 1 + 2 * kStages + 4;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+           const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
+           const __grid_constant__ CUtensorMap tm_kn, const __grid_constant__ CUtensorMap tm_vn,
+           const BwdParams p) {
+  using L = DqLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NQT = cdiv(p.nq, 128);
+  const int qt = blockIdx.x % NQT;
+  const int bh = blockIdx.x / NQT;
+  const int b = bh / p.Hq, h = bh % p.Hq, g = h / p.G;
+  const int NCT = cdiv(p.n, 128);
+  const int T = NCT + qt + 1;  // cache tiles, then chunk tiles 0..qt
+
+  const uint32_t bar_qd = sbase + L::kBarOff;
+  const uint32_t bar_full0 = bar_qd + 8;
+  const uint32_t bar_empty0 = bar_full0 + 8 * L::kStages;
+  const uint32_t bar_s = bar_empty0 + 8 * L::kStages;
+  const uint32_t bar_p = bar_s + 8;
+  const uint32_t bar_o = bar_p + 8;
+  const uint32_t bar_drain = bar_o + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  if (threadIdx.x == 0) {
+    mbar_init(bar_qd, 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar_full0 + 8 * s, 1);
+      mbar_init(bar_empty0 + 8 * s, 1);
+    }
+    mbar_init(bar_s, 1);
+    mbar_init(bar_p, 128);
+    mbar_init(bar_o, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM columns: S [0,128) (then scale*dS as bf16), dP [128,256), dQ [256, 256+D)
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_qd, 2 * L::kTileBytes);
+      for (int r = 0; r < L::kRegions; ++r) {
+        tma_load_4d(sbase + L::kQOff + r * 16384, &tm_q, bar_qd, r * 64, h, qt * 128, b);
+        tma_load_4d(sbase + L::kDOOff + r * 16384, &tm_do, bar_qd, r * 64, h, qt * 128, b);
+      }
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const bool chunk = t >= NCT;
+        const int j0 = (chunk ? t - NCT : t) * 128;
+        const int s = t % L::kStages;
+        if (t >= L::kStages &&
+            !mbar_wait(bar_empty0 + 8 * s, ((t / L::kStages) + 1) & 1, p.err, abort_flag))
+          break;
+        const uint32_t full = bar_full0 + 8 * s;
+        mbar_arrive_expect_tx(full, 2 * L::kTileBytes);
+        for (int r = 0; r < L::kRegions; ++r) {
+          const uint32_t kd = sbase + L::kKOff + s * L::kTileBytes + r * 16384;
+          const uint32_t vd = sbase + L::kVOff + s * L::kTileBytes + r * 16384;
+          if (chunk) {
+            tma_load_4d(kd, &tm_kn, full, r * 64, g, j0, b);
+            tma_load_4d(vd, &tm_vn, full, r * 64, g, j0, b);
+          } else {
+            tma_load_3d(kd, &tm_kc, full, r * 64, j0, b * p.Hkv + g);
+            tma_load_3d(vd, &tm_vc, full, r * 64, j0, b * p.Hkv + g);
+          }
+        }
+        issued = t + 1;
+      }
+      mbar_wait_drain(bar_qd, 0, p.err);
+      for (int t = (issued > L::kStages ? issued - L::kStages : 0); t < issued; ++t)
+        mbar_wait_drain(bar_full0 + 8 * (t % L::kStages), (t / L::kStages) & 1, p.err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, false, true);
+      bool ok = mbar_wait(bar_qd, 0, p.err, abort_flag);
+      for (int t = 0; t < T && ok; ++t) {
+        const int s = t % L::kStages;
+        ok = mbar_wait(bar_full0 + 8 * s, (t / L::kStages) & 1, p.err, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kb = sbase + L::kKOff + s * L::kTileBytes;
+        const uint32_t vb = sbase + L::kVOff + s * L::kTileBytes;
+        // S = Q K^T, dP = dO V^T
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_bf16_ss(tmem, sw128_desc(sbase + L::kQOff + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
+                      kIdescS, ks > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_bf16_ss(tmem + 128, sw128_desc(sbase + L::kDOOff + off, 16, 1024),
+                      sw128_desc(vb + off, 16, 1024), kIdescS, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_s);
+        ok = mbar_wait(bar_p, t & 1, p.err, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        // dQ += (scale dS) K (contraction over the 128 keys)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          mma_bf16_ts(tmem + 256, tmem + 8 * ks, sw128_desc(kb + ks * 2048, 16384, 1024), kIdescAcc,
+                      (t > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(bar_empty0 + 8 * s);
+      }
+      mma_commit(bar_o);
+      mma_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0, p.err);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;  // query qt*128 + row
+    const int i = qt * 128 + row;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const float c = p.scale_log2, scale = p.scale;
+    const size_t ridx = (static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + i;
+    const float nl = p.nlse2[ridx];  // -inf for padding rows: P = 0
+    const float dsum = i < p.nq ? p.dsum[ridx] : 0.f;
+    float nls[32], dvv[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      nls[k] = nl;
+      dvv[k] = dsum;
+    }
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      ok = mbar_wait(bar_s, t & 1, p.err, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      // visible keys of this tile for this row
+      int last = 127;
+      bool masked = false;
+      if (t < NCT) {
+        if (t == NCT - 1 && p.n - t * 128 < 128) {
+          masked = true;
+          last = p.n - t * 128 - 1;
+        }
+      } else if (t - NCT == qt) {
+        masked = true;
+        last = row;
+      }
+#pragma unroll
+      for (int q32 = 0; q32 < 4; ++q32) {
+        uint32_t sv[32], dp[32], pp[16], dd[16];
+        tmem_ld32(lane_base + 32 * q32, sv);
+        tmem_ld32(lane_base + 128 + 32 * q32, dp);
+        tmem_wait_ld();
+        if (masked)
+          p_ds_32<true>(sv, dp, nls, dvv, c, scale, 0, last - 32 * q32, pp, dd);
+        else
+          p_ds_32<false>(sv, dp, nls, dvv, c, scale, 0, 0, pp, dd);
+        tmem_st16(lane_base + 16 * q32, dd);  // scale*dS over S: keys [32 q32, +32)
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p);
+    }
+    if (ok) {
+      ok = mbar_wait(bar_o, 0, p.err, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      float* dqr = p.dq + ((static_cast<size_t>(b) * p.nq + i) * p.Hq + h) * D;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t qv[32];
+        tmem_ld32(lane_base + 256 + c0, qv);
+        tmem_wait_ld();
+        if (i < p.nq) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dqr + c0 + e) =
+                make_float4(__uint_as_float(qv[e]), __uint_as_float(qv[e + 1]),
+                            __uint_as_float(qv[e + 2]), __uint_as_float(qv[e + 3]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- launch
+
+template <int D>
+static cudaError_t launch_bwd_d(const BwdMaps& m, const BwdParams& p, const void* out,
+                                const void* dout, cudaStream_t st) {
+  const int rows = p.B * p.nq * p.Hq;
+  bwd_rowdot<<<cdiv(rows, 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(out),
+                                            static_cast<const __nv_bfloat16*>(dout), p, D);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  static int bits_a[2] = {0, 0}, bits_b[2] = {0, 0};
+  if (!smem_attr_done(reinterpret_cast<const void*>(bwd_dkdv<D>), bits_a)) {
+    e = cudaFuncSetAttribute(bwd_dkdv<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DkdvLayout<D>::kAlloc);
+    if (e != cudaSuccess) return e;
+  }
+  if (!smem_attr_done(reinterpret_cast<const void*>(bwd_dq<D>), bits_b)) {
+    e = cudaFuncSetAttribute(bwd_dq<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DqLayout<D>::kAlloc);
+    if (e != cudaSuccess) return e;
+  }
+  bwd_dkdv<D><<<dim3(cdiv(p.C, 128) + cdiv(p.nq, 128), p.B * p.Hkv), 192, DkdvLayout<D>::kAlloc,
+                st>>>(m.q, m.dout, m.kc, m.vc, m.kn, m.vn, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bwd_dq<D><<<p.B * p.Hq * cdiv(p.nq, 128), 192, DqLayout<D>::kAlloc, st>>>(m.q, m.dout, m.kc, m.vc,
+                                                                           m.kn, m.vn, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_bwd_bf16(int head_dim, const BwdMaps& m, const BwdParams& p,
+                                 const void* out, const void* dout, cudaStream_t st) {
+  return head_dim == 128 ? launch_bwd_d<128>(m, p, out, dout, st)
+                         : launch_bwd_d<64>(m, p, out, dout, st);
+}
+
+}  // namespace h2o

@@ -44,6 +44,21 @@ struct AttnParams {
   int* err;             // device error word (state + 2)
 };
 
+// Arguments of the backward kernels (attn_bwd.cu).
+struct BwdParams {
+  int B, Hq, Hkv, G, nq, n, C, nq_pad;
+  float scale;            // softmax scale (natural)
+  float scale_log2;       // scale * log2(e)
+  const float* nlse2;     // [B, Hq, nq_pad]: the forward's -lse2 (-inf for padding rows)
+  float* dsum;            // [B, Hq, nq_pad]: D_i = <dO_i, O_i>
+  float* dq;              // [B, nq, Hq, d]
+  float* dk_cache;        // [B, Hkv, C, d]
+  float* dv_cache;
+  float* dk_new;          // [B, nq, Hkv, d]
+  float* dv_new;
+  int* err;               // device error word (state + 2)
+};
+
 // ---------------------------------------------------------------- eviction
 
 constexpr int kPolicyH2O = 0;

@@ -38,6 +38,9 @@ struct h2o_cache {
   float* dec_logits = nullptr;  // decode: [B*Hkv, G, C + 1]
   float* dec_part = nullptr;    // decode: [B*Hkv, dec_part_ld, G, d + 2]
   int dec_part_ld = 0;
+  float* dsum = nullptr;  // backward: D_i = <dO_i, O_i>, [B, Hq, nq_pad]
+  int fwd_nq = 0;         // n_q of the last attention whose row statistics are
+  int fwd_n = -1;         // in the workspace, and the valid slots it saw
   unsigned long long* dec_best = nullptr;  // decode: [B*Hkv, dec_slices_ld]
   int* dec_ticket = nullptr;               // decode: [B*Hkv], zero between steps
   int dec_slices_ld = 0;
@@ -70,8 +73,8 @@ size_t esize_of(h2o_dtype t) { return t == H2O_BF16 ? 2 : 4; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct Layout {
-  size_t lse, colsum, slots, tokens, count, dlog, dpart, dbest, dticket, sq[2], skn[2], svn[2],
-      sout[2], total;
+  size_t lse, dsum, colsum, slots, tokens, count, dlog, dpart, dbest, dticket, sq[2], skn[2],
+      svn[2], sout[2], total;
   int nq_pad, colsum_ld, dpart_ld, dslices_ld;
 };
 
@@ -88,6 +91,7 @@ Layout workspace_layout(const h2o_config& c) {
     return at;
   };
   L.lse = take(static_cast<size_t>(c.batch) * c.n_q_heads * L.nq_pad * 4);
+  L.dsum = take(static_cast<size_t>(c.batch) * c.n_q_heads * L.nq_pad * 4);
   L.colsum = take(BHkv * L.colsum_ld * 4);
   L.slots = take(BHkv * c.max_chunk * 4);
   L.tokens = take(BHkv * c.max_chunk * 4);
@@ -250,6 +254,8 @@ h2o_status run_attention(h2o_cache* c, const void* q, const void* kn, const void
   cudaError_t e = launch_attn_fwd_bf16(g.head_dim, m, p, st);
   if (e != cudaSuccess) return H2O_ERR_CUDA;
   c->launches += 1;
+  c->fwd_nq = nq;  // the row statistics of this call stay for a backward
+  c->fwd_n = c->n;
   mark(c, 1, st);
   if (with_colsum) {
     e = launch_attn_colsum_bf16(g.head_dim, m, p, st);
@@ -295,6 +301,7 @@ h2o_status run_evict(h2o_cache* c, const float* colsum, int ld, const void* kn, 
   }
   cudaError_t err = launch_evict(e, g.max_chunk, st);
   if (err != cudaSuccess) return H2O_ERR_CUDA;
+  c->fwd_nq = 0;  // the cache changes: no backward of the earlier attention
   c->launches += 1;
   mark(c, 3, st);
   c->n = c->n + nq < g.capacity ? c->n + nq : g.capacity;
@@ -354,6 +361,7 @@ h2o_status run_decode(h2o_cache* c, const void* q, const void* kn, const void* v
   mark(c, 0, st);
   if (launch_decode(d, static_cast<int>(esize_of(g.dtype)), g.head_dim, st) != cudaSuccess)
     return H2O_ERR_CUDA;
+  c->fwd_nq = 0;  // the decode path keeps no row statistics
   c->launches += 2;
   mark(c, 1, st);  // both kernels are reported as the first part
   mark(c, 2, st);
@@ -441,6 +449,7 @@ h2o_status h2o_cache_create(const h2o_config* cfg, const h2o_buffers* bufs, void
   c->nq_pad = L.nq_pad;
   c->colsum_ld = L.colsum_ld;
   c->lse2 = reinterpret_cast<float*>(ws + L.lse);
+  c->dsum = reinterpret_cast<float*>(ws + L.dsum);
   c->colsum = reinterpret_cast<float*>(ws + L.colsum);
   c->plan_slots = reinterpret_cast<int*>(ws + L.slots);
   c->plan_tokens = reinterpret_cast<int*>(ws + L.tokens);
@@ -490,6 +499,55 @@ h2o_status h2o_attention(h2o_cache* c, const void* q, const void* k_new, const v
                           : run_attention(c, q, k_new, v_new, n_q, out, st);
   if (s == H2O_OK && colsum_out) s = copy_colsum(c, colsum_out, n_q, st);
   return s;
+}
+
+h2o_status h2o_attention_backward(h2o_cache* c, const void* q, const void* k_new,
+                                  const void* v_new, int32_t n_q, const void* out,
+                                  const void* d_out, float* dq, float* dk_cache, float* dv_cache,
+                                  float* dk_new, float* dv_new, void* stream) {
+  h2o_status s = check_step_args(c, q, k_new, v_new, n_q, out);
+  if (s != H2O_OK || n_q == 0) return s;
+  const h2o_config& g = c->cfg;
+  if (g.dtype != H2O_BF16) return H2O_ERR_DTYPE;
+  if (!d_out || !dq || !dk_cache || !dv_cache || !dk_new || !dv_new) return H2O_ERR_INVALID_ARG;
+  if (!aligned(d_out, 16) || !aligned(dq, 16) || !aligned(dk_cache, 16) ||
+      !aligned(dv_cache, 16) || !aligned(dk_new, 16) || !aligned(dv_new, 16))
+    return H2O_ERR_ALIGN;
+  // the row statistics must be those of h2o_attention on this state and n_q
+  if (c->fwd_nq != n_q || c->fwd_n != c->n) return H2O_ERR_STATE;
+  BwdParams p;
+  p.B = g.batch;
+  p.Hq = g.n_q_heads;
+  p.Hkv = g.n_kv_heads;
+  p.G = g.n_q_heads / g.n_kv_heads;
+  p.nq = n_q;
+  p.n = c->n;
+  p.C = g.capacity;
+  p.nq_pad = c->nq_pad;
+  p.scale = g.softmax_scale > 0.f ? g.softmax_scale : 1.f / sqrtf((float)g.head_dim);
+  p.scale_log2 = p.scale * 1.4426950408889634f;
+  p.nlse2 = c->lse2;
+  p.dsum = c->dsum;
+  p.dq = dq;
+  p.dk_cache = dk_cache;
+  p.dv_cache = dv_cache;
+  p.dk_new = dk_new;
+  p.dv_new = dv_new;
+  p.err = c->buf.state + 2;
+  BwdMaps m;
+  const int BH = g.batch * g.n_kv_heads;
+  if (!encode_chunk(&m.q, q, g.batch, n_q, g.n_q_heads, g.head_dim) ||
+      !encode_chunk(&m.dout, d_out, g.batch, n_q, g.n_q_heads, g.head_dim) ||
+      !encode_chunk(&m.kn, k_new, g.batch, n_q, g.n_kv_heads, g.head_dim) ||
+      !encode_chunk(&m.vn, v_new, g.batch, n_q, g.n_kv_heads, g.head_dim) ||
+      !encode_cache(&m.kc, c->buf.k, BH, c->n, g.capacity, g.head_dim) ||
+      !encode_cache(&m.vc, c->buf.v, BH, c->n, g.capacity, g.head_dim))
+    return H2O_ERR_CUDA;
+  if (launch_attn_bwd_bf16(g.head_dim, m, p, out, d_out, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return H2O_ERR_CUDA;
+  c->launches += 3;
+  return H2O_OK;
 }
 
 h2o_status h2o_evict(h2o_cache* c, const float* colsum, const void* k_new, const void* v_new,
@@ -610,6 +668,7 @@ h2o_status h2o_cache_write(h2o_cache* c, const void* k, const void* v, const flo
   if (e != cudaSuccess) return H2O_ERR_CUDA;
   c->n = n_t0[0];
   c->t0 = n_t0[1];
+  c->fwd_nq = 0;
   return H2O_OK;
 }
 
