@@ -366,6 +366,33 @@ def run_ours(args, world, rank, local):
     h2d = sum(t.numel() * t.element_size() for t in hq[0])
     d2h = hout[0].numel() * hout[0].element_size()
 
+    # ---- backward of the attention (fine-tuning through the cache): the
+    # gradients of O for the steady-state cache, timed on their own
+    bwd = None
+    if not decode and wl.dtype == "bf16":
+        nb = min(K, 8)
+        b_s = [torch.cuda.Event(enable_timing=True) for _ in range(nb)]
+        b_e = [torch.cuda.Event(enable_timing=True) for _ in range(nb)]
+        for k in range(nb + 2):
+            q, kn, vn = chunks[W + k % K]
+            O, _ = cache.attention(q, kn, vn)
+            dO = torch.randn_like(O)
+            flush.zero_()
+            if k >= 2:
+                b_s[k - 2].record(stream)
+            cache.attention_backward(q, kn, vn, O, dO)
+            if k >= 2:
+                b_e[k - 2].record(stream)
+        torch.cuda.synchronize(dev)
+        if cache.check() != 0:
+            raise SystemExit("device error during the backward")
+        b_ms = float(np.mean([s_.elapsed_time(e_) for s_, e_ in zip(b_s, b_e)]))
+        bflops = 2 * attention_flops(wl, cache.info()["n"], wl.chunk)
+        bwd = {"ms": round(b_ms, 5), "tflops": round(bflops / (b_ms * 1e-3) / 1e12, 2),
+               "frac": round(bflops / (b_ms * 1e-3) / 1e12 / load_peaks()[0]["bf16_tflops"], 4),
+               "per_call": f"{bflops:.4e} FLOP (dV, dP, dQ, dK over visible pairs: 8*d per "
+                           f"(head, query, key)); 3 launches (row dots, dK/dV, dQ)"}
+
     # ---- roofline of the dominant kernel
     peaks, peaks_kind = load_peaks()
     avg = kern.mean(axis=0)
@@ -449,6 +476,8 @@ def run_ours(args, world, rank, local):
         "clocks": clocks.summary(),
     }
     line.update(extra)
+    if bwd is not None:
+        line["backward"] = bwd
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_steps)
     return line
