@@ -44,8 +44,10 @@ The readings taken here, where the sources are silent:
 Parity status: attention output, summed weights and the selection are pinned
 by brute force, a library routine (torch SDPA in fp64), closed forms and
 invariants in ``tests/test_oracle_*.py``.  The multi-step trajectory is pinned
-by an independent token-centric re-implementation.  No worked numeric example
-exists in the sources.
+by an independent token-centric re-implementation.  The backward is pinned by
+torch fp64 autograd, central finite differences and closed forms; the
+score-free policies by the closed form of the positions they keep.  No worked
+numeric example exists in the sources.
 """
 from __future__ import annotations
 
