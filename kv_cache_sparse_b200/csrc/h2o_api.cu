@@ -1,15 +1,18 @@
 // h2o_api.cu -- host side of the C ABI declared in include/h2o.h.
 //
 // Validates arguments, lays out the caller's workspace, encodes the TMA
-// descriptors of each call and launches the four kernels of a step on the
-// caller's stream (three kernels; the K/V scatter is fused into K3):
+// descriptors of each call and launches the kernels of a step on the
+// caller's stream (three; the K/V scatter is fused into K3):
 //   K1 attention forward + row statistics   (attn_fwd.cu, tcgen05)
 //   K2 summed attention weights per key     (attn_colsum.cu, tcgen05)
 //   K3 score update + top-C selection + K/V scatter into the freed slots
 //                                           (evict.cu)
 // Float32 caches use the fp32 kernels of attn_f32.cu for K1/K2.  A call with
-// n_q = 1 (a decode step) runs the two split-KV kernels of decode.cu instead,
-// when the group has at most kDecodeMaxG query heads.
+// n_q = 1 (a decode step) runs the two split-KV kernels of decode.cu instead
+// when the group has 1, 2, 4 or 8 query heads.  The score-free policies skip
+// K2 unless the caller asks for the summed weights.  The backward of the
+// attention (attn_bwd.cu) runs on the row statistics K1 left in the
+// workspace.
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
@@ -266,7 +269,8 @@ h2o_status run_attention(h2o_cache* c, const void* q, const void* kn, const void
   return H2O_OK;
 }
 
-// K3 + K4 with summed weights `colsum` (row stride ld); advances n and t0.
+// K3 (selection and the fused K/V scatter) with summed weights `colsum` (row
+// stride ld); advances n and t0.
 h2o_status run_evict(h2o_cache* c, const float* colsum, int ld, const void* kn, const void* vn,
                      int nq, cudaStream_t st) {
   const h2o_config& g = c->cfg;
