@@ -96,7 +96,11 @@ def traffic(path, kernel, source):
     rows = list(csv.reader(out.splitlines()))
     hdr, units = rows[0], rows[1]
     scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
-    r = rows[2]
+    name_col = hdr.index("Kernel Name")
+    mine = [r for r in rows[2:] if kernel in r[name_col]]
+    if not mine:
+        raise SystemExit(f"no launch of {kernel} in {path}")
+    r = mine[0]
     total = 0.0
     for k in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
         i = hdr.index(k)
