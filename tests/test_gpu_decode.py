@@ -143,3 +143,26 @@ def test_decode_full_size_qwen_cache():
     gh.assert_attention_close(O, cs, O_ref, cs_ref, 1, 4, "C 8192 decode")
     ref.evict(gh.np64(cs).astype(np.float32), gh.np64(kn), gh.np64(vn))
     gh.assert_state_equal(gpu.read(), ref, torch.bfloat16, "C 8192 decode")
+
+
+def test_one_token_step_with_unsupported_group_runs_the_chunk_kernels():
+    """G = 3 is not a decode-kernel group size: a one-token step takes the
+    chunk kernels (three launches) and still matches the oracle."""
+    B, Hq, Hkv, d, C, n = 1, 6, 2, 128, 300, 300
+    shape = gh.shape_of(B, Hq, Hkv, d, C, 4, 8)
+    gpu = binding.H2OCache(shape)
+    ref = gh.oracle_for(shape)
+    rng = np.random.default_rng(33)
+    K, V, sc, pos = gh.random_state(shape, n, n + 20, rng)
+    gh.install_state(gpu, ref, K, V, sc, pos, n, n + 20)
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(B, 1, Hq, d, generator=g).to(torch.bfloat16)
+    kn = torch.randn(B, 1, Hkv, d, generator=g).to(torch.bfloat16)
+    vn = torch.randn(B, 1, Hkv, d, generator=g).to(torch.bfloat16)
+    launches0 = gpu.info()["kernel_launches"]
+    O, cs = gpu.step(q.cuda(), kn.cuda(), vn.cuda(), return_colsum=True)
+    assert gpu.info()["kernel_launches"] - launches0 == 3
+    O_ref, cs_ref, _ = ref.attention(gh.np64(q), gh.np64(kn), gh.np64(vn))
+    gh.assert_attention_close(O, cs, O_ref, cs_ref, 1, 3, "G = 3 one-token step")
+    ref.evict(gh.np64(cs).astype(np.float32), gh.np64(kn), gh.np64(vn))
+    gh.assert_state_equal(gpu.read(), ref, torch.bfloat16, "G = 3 one-token step")

@@ -110,3 +110,17 @@ def test_policy_with_summed_weights_requested():
             gh.assert_state_equal(gpu.read(), ref, shape.dtype, "lr with colsum")
     assert np.array_equal(out["h2o"][0], out["lr"][0])
     assert np.array_equal(out["h2o"][1], out["lr"][1])
+
+
+def test_policy_with_float_inputs():
+    """The fp32 path (FMA attention kernels) under SLR: chunk steps past the
+    capacity, then decode steps; the state equals the oracle's each step."""
+    B, Hq, Hkv, d, C, W, sinks = 1, 4, 2, 64, 192, 4, 2
+    shape, gpu, ref = _pair(B, Hq, Hkv, d, C, 64, W, "slr", sinks, dt=torch.float32)
+    g = torch.Generator().manual_seed(8)
+    for step, nq in enumerate([64] * 4 + [1] * 6):
+        q, kn, vn = _inputs(B, nq, Hq, Hkv, d, g, dt=torch.float32)
+        O = gpu.step(q.cuda(), kn.cuda(), vn.cuda())
+        O_ref, _ = ref.step(gh.np64(q), gh.np64(kn), gh.np64(vn))
+        assert float(np.max(np.abs(gh.np64(O) - O_ref))) <= gh.O_TOL
+        gh.assert_state_equal(gpu.read(), ref, torch.float32, f"fp32 slr step {step}")
