@@ -25,7 +25,11 @@
 //                scale*dS (bf16, over S), and dQ += dS K accumulates in TMEM.
 // Every reduction has a fixed order (no atomics): the results are
 // deterministic.  Roles in the two tensor-core kernels: warp 0 TMA producer,
-// warp 1 TMEM allocation and the MMA-issuing thread, warps 2..5 the rows.
+// warp 1 TMEM allocation and the MMA-issuing thread, warps 2..9 the rows in
+// two warpgroups, one per half of the 128 columns of S (queries in bwd_dkdv,
+// keys in bwd_dq).  Each half has its own ready barriers, so the tensor core
+// accumulates one half and computes the next unit's first half while the
+// other warpgroup still works on the second.
 #include <cuda_bf16.h>
 
 #include "attn.h"
@@ -68,13 +72,16 @@ struct DkdvLayout {
   static constexpr int kDOOff = kQOff + kStages * kTileBytes;       // [stage]
   static constexpr int kRowOff = kDOOff + kStages * kTileBytes;     // [stage][2][128] float
   static constexpr int kBarOff = kRowOff + kStages * 1024;
-  // kv_full, u_full[S], u_empty[S], s_full, p_full, o_done, drain
-  static constexpr int kNumBars = 1 + 2 * kStages + 4;
+  // kv_full, u_full[S], u_empty[S], s_full[2], p_full[2], o_done, drain
+  static constexpr int kNumBars = 1 + 2 * kStages + 6;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
-  static constexpr int kThreads = 192;
 };
+
+// Both tensor-core kernels: warp 0 TMA, warp 1 TMEM + MMA, then two
+// warpgroups of row threads, one per half of the 128 columns of S.
+constexpr int kBwdThreads = 64 + 2 * 128;
 
 // Row arithmetic shared by the two kernels: from 32 logits s and 32 dP
 // values of one row (or one key), the bf16 pairs of P and of scale * dS.
@@ -111,7 +118,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
              const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
              const __grid_constant__ CUtensorMap tm_kn, const __grid_constant__ CUtensorMap tm_vn,
@@ -145,9 +152,9 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t bar_kv = sbase + L::kBarOff;
   const uint32_t bar_full0 = bar_kv + 8;
   const uint32_t bar_empty0 = bar_full0 + 8 * L::kStages;
-  const uint32_t bar_s = bar_empty0 + 8 * L::kStages;
-  const uint32_t bar_p = bar_s + 8;
-  const uint32_t bar_o = bar_p + 8;
+  const uint32_t bar_s0 = bar_empty0 + 8 * L::kStages;  // [half]
+  const uint32_t bar_p0 = bar_s0 + 16;                  // [half]
+  const uint32_t bar_o = bar_p0 + 16;
   const uint32_t bar_drain = bar_o + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -157,8 +164,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(bar_full0 + 8 * s, 1);
       mbar_init(bar_empty0 + 8 * s, 1);
     }
-    mbar_init(bar_s, 1);
-    mbar_init(bar_p, 128);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(bar_s0 + 8 * h, 1);
+      mbar_init(bar_p0 + 8 * h, 128);
+    }
     mbar_init(bar_o, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -172,7 +181,10 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns: S^T [0,128), dP^T [128,256), dV [256, 256+D), dK [384, 384+D)
+  // TMEM columns: S^T [0,128), dP^T [128,256), dV [256, 256+D), dK [384, 384+D).
+  // Half hf of a unit is its queries [64 hf, +64): S^T columns [64 hf, +64),
+  // dP^T columns [128 + 64 hf, +64); its P^T and scale*dS^T (bf16 pairs) go
+  // over the first 32 of those columns.
 
   if (warp == 0) {
     if (lane == 0) {
@@ -213,52 +225,81 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, false, true);
-      bool ok = mbar_wait(bar_kv, 0, p.err, abort_flag);
-      for (int u = 0; u < R && ok; ++u) {
-        const int s = u % L::kStages;
-        ok = mbar_wait(bar_full0 + 8 * s, (u / L::kStages) & 1, p.err, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t qb = sbase + L::kQOff + s * L::kTileBytes;
-        const uint32_t db = sbase + L::kDOOff + s * L::kTileBytes;
-        // S^T = K Q^T, dP^T = V dO^T (contraction over the head dim)
+      // S^T and dP^T of one half of unit u (stage s): contraction over the
+      // head dim, the half's 64 query rows of the Q / dO tiles as B
+      auto issue_s = [&](int s, int hf) {
+        const uint32_t qb = sbase + L::kQOff + s * L::kTileBytes + hf * 8192;
+        const uint32_t db = sbase + L::kDOOff + s * L::kTileBytes + hf * 8192;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_bf16_ss(tmem, sw128_desc(sbase + L::kKOff + off, 16, 1024), sw128_desc(qb + off, 16, 1024),
-                      kIdescS, ks > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + 64 * hf, sw128_desc(sbase + L::kKOff + off, 16, 1024),
+                      sw128_desc(qb + off, 16, 1024), kIdescS, ks > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_bf16_ss(tmem + 128, sw128_desc(sbase + L::kVOff + off, 16, 1024),
+          mma_bf16_ss(tmem + 128 + 64 * hf, sw128_desc(sbase + L::kVOff + off, 16, 1024),
                       sw128_desc(db + off, 16, 1024), kIdescS, ks > 0 ? 1u : 0u);
         }
-        mma_commit(bar_s);
-        ok = mbar_wait(bar_p, u & 1, p.err, abort_flag);
+        mma_commit(bar_s0 + 8 * hf);
+      };
+      // dV += P^T dO and dK += (scale dS)^T Q over the half's 64 queries (16
+      // per MMA = 8 TMEM columns of bf16 pairs; B the dO / Q rows MN-major)
+      auto issue_acc = [&](int s, int hf, bool first) {
+        const uint32_t qb = sbase + L::kQOff + s * L::kTileBytes;
+        const uint32_t db = sbase + L::kDOOff + s * L::kTileBytes;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          mma_bf16_ts(tmem + 256, tmem + 64 * hf + 8 * ks,
+                      sw128_desc(db + (4 * hf + ks) * 2048, 16384, 1024), kIdescAcc,
+                      (first && ks == 0) ? 0u : 1u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          mma_bf16_ts(tmem + 384, tmem + 128 + 64 * hf + 8 * ks,
+                      sw128_desc(qb + (4 * hf + ks) * 2048, 16384, 1024), kIdescAcc,
+                      (first && ks == 0) ? 0u : 1u);
+        }
+      };
+      bool ok = mbar_wait(bar_kv, 0, p.err, abort_flag);
+      if (ok && R > 0) ok = mbar_wait(bar_full0, 0, p.err, abort_flag);
+      if (ok && R > 0) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(0, 1);
+      }
+      // per unit: the accumulation of half 0 and the next unit's half-0 S^T
+      // run on the tensor core while the row threads work on half 1
+      for (int u = 0; u < R && ok; ++u) {
+        const int s = u % L::kStages;
+        const bool more = u + 1 < R;
+        const int s1 = (u + 1) % L::kStages;
+        ok = mbar_wait(bar_p0, u & 1, p.err, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        // dV += P^T dO and dK += (scale dS)^T Q (contraction over the 128
-        // queries, 16 per MMA = 8 TMEM columns of bf16 pairs)
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          mma_bf16_ts(tmem + 256, tmem + 8 * ks, sw128_desc(db + ks * 2048, 16384, 1024), kIdescAcc,
-                      (u > 0 || ks > 0) ? 1u : 0u);
+        issue_acc(s, 0, u == 0);
+        if (more) {
+          ok = mbar_wait(bar_full0 + 8 * s1, ((u + 1) / L::kStages) & 1, p.err, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(s1, 0);
         }
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          mma_bf16_ts(tmem + 384, tmem + 128 + 8 * ks, sw128_desc(qb + ks * 2048, 16384, 1024),
-                      kIdescAcc, (u > 0 || ks > 0) ? 1u : 0u);
-        }
+        ok = mbar_wait(bar_p0 + 8, u & 1, p.err, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_acc(s, 1, false);
         mma_commit(bar_empty0 + 8 * s);
+        if (more) issue_s(s1, 1);
       }
       mma_commit(bar_o);
       mma_commit(bar_drain);
       mbar_wait_drain(bar_drain, 0, p.err);
     }
   } else {
+    const int hf = (warp - 2) >> 2;  // half of the unit's queries
     const int quad = warp & 3;
     const int row = quad * 32 + lane;  // key j0 + row
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
@@ -266,7 +307,7 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = true;
     for (int u = 0; u < R; ++u) {
       const int s = u % L::kStages;
-      ok = mbar_wait(bar_s, u & 1, p.err, abort_flag);
+      ok = mbar_wait(bar_s0 + 8 * hf, u & 1, p.err, abort_flag);
       if (ok) ok = mbar_wait(bar_full0 + 8 * s, (u / L::kStages) & 1, p.err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -276,7 +317,8 @@ __global__ void __launch_bounds__(192, 1)
       const int qt = qt_min + u % span;
       const bool diag = is_chunk && qt == kt;  // query col sees key row iff row <= col
 #pragma unroll
-      for (int q32 = 0; q32 < 4; ++q32) {
+      for (int q2 = 0; q2 < 2; ++q2) {
+        const int q32 = 2 * hf + q2;
         uint32_t sv[32], dp[32], pp[16], dd[16];
         tmem_ld32(lane_base + 32 * q32, sv);
         tmem_ld32(lane_base + 128 + 32 * q32, dp);
@@ -286,52 +328,45 @@ __global__ void __launch_bounds__(192, 1)
                         pp, dd);
         else
           p_ds_32<false>(sv, dp, nls + 32 * q32, dvv + 32 * q32, c, scale, 0, 0, pp, dd);
-        // bf16 pairs over the first columns: queries [32 q32, +32) -> [16 q32, +16)
-        tmem_st16(lane_base + 16 * q32, pp);
-        tmem_st16(lane_base + 128 + 16 * q32, dd);
+        // bf16 pairs over the half's first columns: queries [32 q32, +32) ->
+        // columns [64 hf + 16 q2, +16)
+        tmem_st16(lane_base + 64 * hf + 16 * q2, pp);
+        tmem_st16(lane_base + 128 + 64 * hf + 16 * q2, dd);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_p);
+      mbar_arrive(bar_p0 + 8 * hf);
     }
     if (ok) {
       ok = mbar_wait(bar_o, 0, p.err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
+      // half 0 writes dK, half 1 dV
       tc_fence_after();
       const int key = j0 + row;
-      float* dkr = nullptr;
-      float* dvr = nullptr;
+      float* dst = nullptr;
       if (is_chunk) {
-        if (key < p.nq) {
-          const size_t at = ((static_cast<size_t>(b) * p.nq + key) * p.Hkv + g) * row_stride;
-          dkr = p.dk_new + at;
-          dvr = p.dv_new + at;
-        }
+        if (key < p.nq)
+          dst = (hf == 0 ? p.dk_new : p.dv_new) +
+                ((static_cast<size_t>(b) * p.nq + key) * p.Hkv + g) * row_stride;
       } else if (key < p.C) {
-        const size_t at = (static_cast<size_t>(bg) * p.C + key) * row_stride;
-        dkr = p.dk_cache + at;
-        dvr = p.dv_cache + at;
+        dst = (hf == 0 ? p.dk_cache : p.dv_cache) + (static_cast<size_t>(bg) * p.C + key) * row_stride;
       }
       const bool valid = is_chunk ? key < p.nq : key < p.n;
+      const uint32_t col = hf == 0 ? 384 : 256;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t kv[32], vv[32];
-        tmem_ld32(lane_base + 384 + c0, kv);
-        tmem_ld32(lane_base + 256 + c0, vv);
+        uint32_t v[32];
+        tmem_ld32(lane_base + col + c0, v);
         tmem_wait_ld();
-        if (dkr) {
+        if (dst) {
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
-            const float4 k4 = valid ? make_float4(__uint_as_float(kv[e]), __uint_as_float(kv[e + 1]),
-                                                  __uint_as_float(kv[e + 2]), __uint_as_float(kv[e + 3]))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float4 v4 = valid ? make_float4(__uint_as_float(vv[e]), __uint_as_float(vv[e + 1]),
-                                                  __uint_as_float(vv[e + 2]), __uint_as_float(vv[e + 3]))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<float4*>(dkr + c0 + e) = k4;
-            *reinterpret_cast<float4*>(dvr + c0 + e) = v4;
+            const float4 x = valid ? make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                                 __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4*>(dst + c0 + e) = x;
           }
         }
       }
@@ -357,15 +392,15 @@ struct DqLayout {
   static constexpr int kKOff = kDOOff + kTileBytes;            // [stage]
   static constexpr int kVOff = kKOff + kStages * kTileBytes;   // [stage]
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-  // qd_full, kv_full[S], kv_empty[S], s_full, p_full, o_done, drain
-  static constexpr int kNumBars = 1 + 2 * kStages + 4;
+  // qd_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, drain
+  static constexpr int kNumBars = 1 + 2 * kStages + 6;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
            const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
            const __grid_constant__ CUtensorMap tm_kn, const __grid_constant__ CUtensorMap tm_vn,
@@ -385,9 +420,9 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t bar_qd = sbase + L::kBarOff;
   const uint32_t bar_full0 = bar_qd + 8;
   const uint32_t bar_empty0 = bar_full0 + 8 * L::kStages;
-  const uint32_t bar_s = bar_empty0 + 8 * L::kStages;
-  const uint32_t bar_p = bar_s + 8;
-  const uint32_t bar_o = bar_p + 8;
+  const uint32_t bar_s0 = bar_empty0 + 8 * L::kStages;  // [half]
+  const uint32_t bar_p0 = bar_s0 + 16;                  // [half]
+  const uint32_t bar_o = bar_p0 + 16;
   const uint32_t bar_drain = bar_o + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -397,8 +432,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(bar_full0 + 8 * s, 1);
       mbar_init(bar_empty0 + 8 * s, 1);
     }
-    mbar_init(bar_s, 1);
-    mbar_init(bar_p, 128);
+    for (int hf = 0; hf < 2; ++hf) {
+      mbar_init(bar_s0 + 8 * hf, 1);
+      mbar_init(bar_p0 + 8 * hf, 128);
+    }
     mbar_init(bar_o, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -412,7 +449,10 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns: S [0,128) (then scale*dS as bf16), dP [128,256), dQ [256, 256+D)
+  // TMEM columns: S [0,128), dP [128,256), dQ [256, 256+D).  Half hf of a
+  // key tile is its keys [64 hf, +64): S columns [64 hf, +64), dP columns
+  // [128 + 64 hf, +64); its scale*dS (bf16 pairs) goes over the first 32 S
+  // columns of the half.
 
   if (warp == 0) {
     if (lane == 0) {
@@ -450,46 +490,71 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdescS = idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, false, true);
-      bool ok = mbar_wait(bar_qd, 0, p.err, abort_flag);
-      for (int t = 0; t < T && ok; ++t) {
-        const int s = t % L::kStages;
-        ok = mbar_wait(bar_full0 + 8 * s, (t / L::kStages) & 1, p.err, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t kb = sbase + L::kKOff + s * L::kTileBytes;
-        const uint32_t vb = sbase + L::kVOff + s * L::kTileBytes;
-        // S = Q K^T, dP = dO V^T
+      // S = Q K^T and dP = dO V^T for one half of key tile t (stage s): the
+      // half's 64 key rows of the K / V tiles as B
+      auto issue_s = [&](int s, int hf) {
+        const uint32_t kb = sbase + L::kKOff + s * L::kTileBytes + hf * 8192;
+        const uint32_t vb = sbase + L::kVOff + s * L::kTileBytes + hf * 8192;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_bf16_ss(tmem, sw128_desc(sbase + L::kQOff + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
-                      kIdescS, ks > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + 64 * hf, sw128_desc(sbase + L::kQOff + off, 16, 1024),
+                      sw128_desc(kb + off, 16, 1024), kIdescS, ks > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_bf16_ss(tmem + 128, sw128_desc(sbase + L::kDOOff + off, 16, 1024),
+          mma_bf16_ss(tmem + 128 + 64 * hf, sw128_desc(sbase + L::kDOOff + off, 16, 1024),
                       sw128_desc(vb + off, 16, 1024), kIdescS, ks > 0 ? 1u : 0u);
         }
-        mma_commit(bar_s);
-        ok = mbar_wait(bar_p, t & 1, p.err, abort_flag);
+        mma_commit(bar_s0 + 8 * hf);
+      };
+      // dQ += (scale dS) K over the half's 64 keys (B the K rows, MN-major)
+      auto issue_acc = [&](int s, int hf, bool first) {
+        const uint32_t kb = sbase + L::kKOff + s * L::kTileBytes;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          mma_bf16_ts(tmem + 256, tmem + 64 * hf + 8 * ks,
+                      sw128_desc(kb + (4 * hf + ks) * 2048, 16384, 1024), kIdescAcc,
+                      (first && ks == 0) ? 0u : 1u);
+        }
+      };
+      bool ok = mbar_wait(bar_qd, 0, p.err, abort_flag);
+      if (ok) ok = mbar_wait(bar_full0, 0, p.err, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(0, 1);
+      }
+      for (int t = 0; t < T && ok; ++t) {
+        const int s = t % L::kStages;
+        const bool more = t + 1 < T;
+        const int s1 = (t + 1) % L::kStages;
+        ok = mbar_wait(bar_p0, t & 1, p.err, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        // dQ += (scale dS) K (contraction over the 128 keys)
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          mma_bf16_ts(tmem + 256, tmem + 8 * ks, sw128_desc(kb + ks * 2048, 16384, 1024), kIdescAcc,
-                      (t > 0 || ks > 0) ? 1u : 0u);
+        issue_acc(s, 0, t == 0);
+        if (more) {
+          ok = mbar_wait(bar_full0 + 8 * s1, ((t + 1) / L::kStages) & 1, p.err, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(s1, 0);
         }
+        ok = mbar_wait(bar_p0 + 8, t & 1, p.err, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_acc(s, 1, false);
         mma_commit(bar_empty0 + 8 * s);
+        if (more) issue_s(s1, 1);
       }
       mma_commit(bar_o);
       mma_commit(bar_drain);
       mbar_wait_drain(bar_drain, 0, p.err);
     }
   } else {
+    const int hf = (warp - 2) >> 2;  // half of each key tile
     const int quad = warp & 3;
     const int row = quad * 32 + lane;  // query qt*128 + row
     const int i = qt * 128 + row;
@@ -506,7 +571,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     bool ok = true;
     for (int t = 0; t < T; ++t) {
-      ok = mbar_wait(bar_s, t & 1, p.err, abort_flag);
+      ok = mbar_wait(bar_s0 + 8 * hf, t & 1, p.err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -523,7 +588,8 @@ __global__ void __launch_bounds__(192, 1)
         last = row;
       }
 #pragma unroll
-      for (int q32 = 0; q32 < 4; ++q32) {
+      for (int q2 = 0; q2 < 2; ++q2) {
+        const int q32 = 2 * hf + q2;
         uint32_t sv[32], dp[32], pp[16], dd[16];
         tmem_ld32(lane_base + 32 * q32, sv);
         tmem_ld32(lane_base + 128 + 32 * q32, dp);
@@ -532,21 +598,23 @@ __global__ void __launch_bounds__(192, 1)
           p_ds_32<true>(sv, dp, nls, dvv, c, scale, 0, last - 32 * q32, pp, dd);
         else
           p_ds_32<false>(sv, dp, nls, dvv, c, scale, 0, 0, pp, dd);
-        tmem_st16(lane_base + 16 * q32, dd);  // scale*dS over S: keys [32 q32, +32)
+        // scale*dS over S: keys [32 q32, +32) -> columns [64 hf + 16 q2, +16)
+        tmem_st16(lane_base + 64 * hf + 16 * q2, dd);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_p);
+      mbar_arrive(bar_p0 + 8 * hf);
     }
     if (ok) {
       ok = mbar_wait(bar_o, 0, p.err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
+      // each half writes D/2 of the row's dQ columns
       tc_fence_after();
       float* dqr = p.dq + ((static_cast<size_t>(b) * p.nq + i) * p.Hq + h) * D;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = hf * (D / 2); c0 < (hf + 1) * (D / 2); c0 += 32) {
         uint32_t qv[32];
         tmem_ld32(lane_base + 256 + c0, qv);
         tmem_wait_ld();
@@ -589,11 +657,11 @@ static cudaError_t launch_bwd_d(const BwdMaps& m, const BwdParams& p, const void
                              DqLayout<D>::kAlloc);
     if (e != cudaSuccess) return e;
   }
-  bwd_dkdv<D><<<dim3(cdiv(p.C, 128) + cdiv(p.nq, 128), p.B * p.Hkv), 192, DkdvLayout<D>::kAlloc,
-                st>>>(m.q, m.dout, m.kc, m.vc, m.kn, m.vn, p);
+  bwd_dkdv<D><<<dim3(cdiv(p.C, 128) + cdiv(p.nq, 128), p.B * p.Hkv), kBwdThreads,
+                DkdvLayout<D>::kAlloc, st>>>(m.q, m.dout, m.kc, m.vc, m.kn, m.vn, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dq<D><<<p.B * p.Hq * cdiv(p.nq, 128), 192, DqLayout<D>::kAlloc, st>>>(m.q, m.dout, m.kc, m.vc,
+  bwd_dq<D><<<p.B * p.Hq * cdiv(p.nq, 128), kBwdThreads, DqLayout<D>::kAlloc, st>>>(m.q, m.dout, m.kc, m.vc,
                                                                            m.kn, m.vn, p);
   return cudaGetLastError();
 }
