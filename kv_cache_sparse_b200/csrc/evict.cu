@@ -20,12 +20,12 @@
 //      candidate index (slot s -> s, new token i -> n + i; same order as the
 //      C + i numbering).  So exactly C candidates stay, ties go to the lower
 //      index, and the protected ones always stay (there are at most W <= C).
-//   4. Ordered compaction (block scans over contiguous per-thread ranges)
+//   4. Ordered compaction (one block scan over contiguous per-thread ranges)
 //      lists the free slots (evicted or empty) and the kept new tokens in
 //      ascending order; the k-th kept token goes to the k-th free slot.  The
 //      CTA writes the score and position of the placed tokens and the plan,
-//      then copies their K and V rows into the slots (one warp per token,
-//      16-byte vector loads and stores).
+//      then copies their K and V rows into the slots (16-byte vector loads
+//      and stores, whole rows per warp, several loads in flight per thread).
 #include "attn.h"
 #include "sm100.cuh"
 
@@ -38,51 +38,82 @@ __device__ __forceinline__ uint32_t score_key(float s) {
   return u == 0x80000000u ? 0u : u;  // -0 orders as +0
 }
 
-// Exclusive scan of one value per thread over the block; returns the prefix,
-// writes the block total to *total.  All threads must call it.
+// Exclusive scan of one 64-bit value per thread over the block (four packed
+// 16-bit counters: no field carries into the next while every block total
+// stays below 2^16); returns the prefix, writes the block total to *total.
 template <int NT>
-__device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total) {
+__device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t* warp_sums,
+                                                      uint64_t* total) {
   constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int x = v;
+  uint64_t x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
   __syncthreads();
   if (lane == 31) warp_sums[w] = x;
   __syncthreads();
   if (w == 0) {
-    int s = lane < NW ? warp_sums[lane] : 0;
+    uint64_t s = lane < NW ? warp_sums[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, s, o);
+      const uint64_t y = __shfl_up_sync(0xffffffffu, s, o);
       if (lane >= o) s += y;
     }
     if (lane < NW) warp_sums[lane] = s;  // inclusive
   }
   __syncthreads();
-  const int before = (w > 0 ? warp_sums[w - 1] : 0) + x - v;
+  const uint64_t before = (w > 0 ? warp_sums[w - 1] : 0) + x - v;
   *total = warp_sums[NW - 1];
   return before;
 }
 
-// Copies the K and V rows of new token `tok` into slot `slot`: one warp, one
-// 16-byte vector per lane and pass (K vectors first, then V vectors).
-__device__ __forceinline__ void move_rows(const EvictParams& e, int b, int g, int slot, int tok,
-                                          int lane) {
+// Copies the K and V rows of the placed tokens: the k-th token tok_of(k)
+// goes to slot slot_of(k), k < count.  The block walks the 16-byte vectors
+// of all rows (token-major: the K vectors, then the V vectors of a token), so
+// a warp reads and writes whole rows; each thread keeps kCopyBatch loads in
+// flight before it stores.
+constexpr int kCopyBatch = 8;
+
+template <int NT, class SlotOf, class TokOf>
+__device__ __forceinline__ void copy_rows(const EvictParams& e, int b, int g, int count,
+                                          SlotOf slot_of, TokOf tok_of) {
   const int vpr = e.d * e.esize / 16;  // vectors per row
-  const size_t row_bytes = static_cast<size_t>(e.d) * e.esize;
-  const size_t src_off = ((static_cast<size_t>(b) * e.nq + tok) * e.Hkv + g) * row_bytes;
-  const size_t dst_off = ((static_cast<size_t>(b) * e.Hkv + g) * e.C + slot) * row_bytes;
-  for (int v = lane; v < 2 * vpr; v += 32) {
-    const bool is_v = v >= vpr;
-    const int vv = is_v ? v - vpr : v;
-    const uint4* src =
-        reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(is_v ? e.v_new : e.k_new) + src_off);
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(is_v ? e.v_cache : e.k_cache) + dst_off);
-    dst[vv] = __ldg(src + vv);
+  const int per_tok = 2 * vpr;
+  const int total = count * per_tok;
+  const size_t row_vecs = static_cast<size_t>(vpr);
+  const uint4* kn = static_cast<const uint4*>(e.k_new);
+  const uint4* vn = static_cast<const uint4*>(e.v_new);
+  uint4* kc = static_cast<uint4*>(e.k_cache);
+  uint4* vc = static_cast<uint4*>(e.v_cache);
+  const size_t head_row0 = (static_cast<size_t>(b) * e.Hkv + g) * e.C;
+  for (int v0 = threadIdx.x; v0 < total; v0 += kCopyBatch * NT) {
+    uint4 buf[kCopyBatch];
+    int to[kCopyBatch];  // (slot << 7) | vector within the token (per_tok <= 64), or -1
+#pragma unroll
+    for (int u = 0; u < kCopyBatch; ++u) {
+      const int v = v0 + u * NT;
+      to[u] = -1;
+      if (v < total) {
+        const int q = v / per_tok, r = v - q * per_tok;
+        const bool is_v = r >= vpr;
+        const int c = is_v ? r - vpr : r;
+        const size_t src = ((static_cast<size_t>(b) * e.nq + tok_of(q)) * e.Hkv + g) * row_vecs + c;
+        buf[u] = __ldg((is_v ? vn : kn) + src);
+        to[u] = (slot_of(q) << 7) | r;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyBatch; ++u) {
+      if (to[u] >= 0) {
+        const int r = to[u] & 127;
+        const bool is_v = r >= vpr;
+        const size_t at = (head_row0 + (to[u] >> 7)) * row_vecs + (is_v ? r - vpr : r);
+        (is_v ? vc : kc)[at] = buf[u];
+      }
+    }
   }
 }
 
@@ -90,12 +121,12 @@ constexpr int kLoadBatch = 8;  // global loads in flight per thread in the first
 constexpr int kBins = 256;     // radix passes of 8 bits, most significant first
 
 template <int NT>
-__global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1)) h2o_select(const EvictParams e) {
-  constexpr int NW = NT / 32;
+__global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
+    h2o_select(const EvictParams e, int plan_smem) {
   constexpr int kSub = (NT == 1024) ? 8 : 2;  // sub-histograms spread the first passes' atomics
-  extern __shared__ uint32_t keys[];          // [n + nq]
+  extern __shared__ uint32_t keys[];          // [n + nq], then (plan_smem) the plan [2][nq]
   __shared__ int hist[kSub][kBins];           // warp w counts into hist[w % kSub]
-  __shared__ int warp_sums[32];
+  __shared__ uint64_t warp_sums[32];
   __shared__ int sel_bin, sel_above;
 
   const int bg = blockIdx.x;
@@ -186,7 +217,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1)) h2o_select(const Evic
       pos[n + i] = e.t0 + i;
     }
     if (tid == 0) e.plan_count[bg] = nq;
-    for (int q = warp; q < nq; q += NW) move_rows(e, b, g, n + q, q, lane);
+    copy_rows<NT>(e, b, g, nq, [n](int q) { return n + q; }, [](int q) { return q; });
     return;
   }
   __syncthreads();
@@ -256,28 +287,40 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1)) h2o_select(const Evic
   }
   const uint32_t T = prefix;  // C-th largest key; keep the first k keys equal to T
 
-  // 3. ordered pass over contiguous ranges: rank the T-keys by index, then
-  //    count freed old slots and kept new tokens (one packed scan)
+  // 3. ordered pass over contiguous ranges.  Keys above T stay, keys below
+  //    go, and of the keys equal to T the first k in candidate-index order
+  //    stay.  One scan of four counters per thread (freed old slots and kept
+  //    new tokens among the keys != T, keys == T, keys == T that are old
+  //    slots) places every thread's output: old slots precede new tokens in
+  //    index order, so the kept T-keys before a range are the first
+  //    min(eq, k) of them, and the old ones among those min(eq_old, k).
   const int per = (NC + NT - 1) / NT;
   const int lo = min(NC, tid * per), hi = min(NC, lo + per);
-  int n_eq = 0;
-  for (int x = lo; x < hi; ++x) n_eq += (keys[x] == T);
-  int tot;
-  int eq_before = block_excl_scan<NT>(n_eq, warp_sums, &tot);
-  int free_old = 0, n_new = 0;
+  int fo_s = 0, nn_s = 0, eq = 0, eq_old = 0;
   for (int x = lo; x < hi; ++x) {
     const uint32_t key = keys[x];
-    bool kept = key > T;
-    if (key == T) kept = (eq_before++ < k);
-    if (x < n) free_old += !kept;
-    else n_new += kept;
-    keys[x] = kept ? 1u : 0u;  // from here on: kept flag
+    if (key == T) {
+      ++eq;
+      eq_old += x < n;
+    } else if (key > T) {
+      nn_s += x >= n;
+    } else {
+      fo_s += x < n;
+    }
   }
   // counts and totals stay below 2^16 (candidates <= kMaxCandidates)
-  int pk_tot;
-  const int pk_before = block_excl_scan<NT>(free_old | (n_new << 16), warp_sums, &pk_tot);
-  const int fo_before = pk_before & 0xFFFF, nw_before = pk_before >> 16;
-  const int tot_free_old = pk_tot & 0xFFFF, tot_new = pk_tot >> 16;
+  uint64_t pk_tot;
+  const uint64_t pk_before = block_excl_scan64<NT>(
+      static_cast<uint64_t>(fo_s) | (static_cast<uint64_t>(nn_s) << 16) |
+          (static_cast<uint64_t>(eq) << 32) | (static_cast<uint64_t>(eq_old) << 48),
+      warp_sums, &pk_tot);
+  auto field = [](uint64_t v, int f) { return static_cast<int>((v >> (16 * f)) & 0xFFFF); };
+  const int eq_b = field(pk_before, 2), eqo_b = field(pk_before, 3);
+  const int fo_before = field(pk_before, 0) + eqo_b - min(eqo_b, k);
+  const int nw_before = field(pk_before, 1) + min(eq_b, k) - min(eqo_b, k);
+  const int eq_t = field(pk_tot, 2), eqo_t = field(pk_tot, 3);
+  const int tot_free_old = field(pk_tot, 0) + eqo_t - min(eqo_t, k);
+  const int tot_new = field(pk_tot, 1) + min(eq_t, k) - min(eqo_t, k);
   // empty slots n .. C-1 are free too: thread t takes a fixed share, in order
   const int empty = C - n;
   const int e_per = (empty + NT - 1) / NT;
@@ -289,50 +332,66 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1)) h2o_select(const Evic
     }
     return;
   }
-  // free slots in order: evicted old slots (< n) first, then the empty ones
-  int fo = fo_before, nw = nw_before;
+  // free slots in order (evicted old slots (< n) first, then the empty ones)
+  // and kept new tokens in order; in shared memory when it has room
+  int* p_slots = plan_smem ? reinterpret_cast<int*>(keys + NC) : slots;
+  int* p_toks = plan_smem ? p_slots + nq : toks;
+  int fo = fo_before, nw = nw_before, eq_rank = eq_b;
   for (int x = lo; x < hi; ++x) {
+    const uint32_t key = keys[x];
+    bool kept = key > T;
+    if (key == T) kept = eq_rank++ < k;
     if (x < n) {
-      if (!keys[x]) slots[fo++] = x;
-    } else if (keys[x]) {
-      toks[nw++] = x - n;
+      if (!kept) p_slots[fo++] = x;
+    } else if (kept) {
+      p_toks[nw++] = x - n;
     }
   }
   int em = tot_free_old + (e_lo - n);
-  for (int s = e_lo; s < e_hi; ++s) slots[em++] = s;
+  for (int s = e_lo; s < e_hi; ++s) p_slots[em++] = s;
   __syncthreads();
-  // 4. scores and positions of the placed tokens, then their K/V rows
+  // 4. scores and positions of the placed tokens (and the plan, when it was
+  //    built in shared memory), then their K/V rows
   for (int q = tid; q < tot_new; q += NT) {
-    const int s = slots[q], i = toks[q];
+    const int s = p_slots[q], i = p_toks[q];
     score[s] = by_score ? cs[C + i] : 0.f;
     pos[s] = e.t0 + i;
-  }
-  if (tid == 0) e.plan_count[bg] = tot_new;
-  // K/V rows: warp w moves rows w, w + NW, ...; lane L first fetches the
-  // (slot, token) of the warp's L-th row, so that the copies do not wait on
-  // one another's plan reads
-  for (int q0 = warp; q0 < tot_new; q0 += NW * 32) {
-    const int q = q0 + lane * NW;
-    const int my_slot = q < tot_new ? slots[q] : 0;
-    const int my_tok = q < tot_new ? toks[q] : 0;
-    const int rows = min(32, (tot_new - q0 + NW - 1) / NW);
-#pragma unroll 4
-    for (int r = 0; r < rows; ++r) {
-      const int sl = __shfl_sync(0xffffffffu, my_slot, r);
-      const int tk = __shfl_sync(0xffffffffu, my_tok, r);
-      move_rows(e, b, g, sl, tk, lane);
+    if (plan_smem) {
+      slots[q] = s;
+      toks[q] = i;
     }
   }
+  if (tid == 0) e.plan_count[bg] = tot_new;
+  copy_rows<NT>(e, b, g, tot_new, [p_slots](int q) { return p_slots[q]; },
+                [p_toks](int q) { return p_toks[q]; });
+}
+
+// Dynamic shared memory the selection kernel can take next to its static
+// arrays (histograms, scan sums).
+template <int NT>
+static size_t select_dyn_limit() {
+  static const size_t limit = [] {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, h2o_select<NT>) != cudaSuccess) return size_t{0};
+    return static_cast<size_t>(kMaxDynSmem) - fa.sharedSizeBytes;
+  }();
+  return limit;
 }
 
 template <int NT>
 static cudaError_t launch_select(const EvictParams& e, cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(e.n + e.nq) * sizeof(uint32_t);
+  const size_t limit = select_dyn_limit<NT>();
+  if (limit < static_cast<size_t>(kMaxCandidates) * sizeof(uint32_t)) return cudaErrorInvalidValue;
+  // the keys, then the plan when it fits next to them
+  const size_t keys_bytes = static_cast<size_t>(e.n + e.nq) * sizeof(uint32_t);
+  const size_t plan_bytes = static_cast<size_t>(2) * e.nq * sizeof(int);
+  const int plan_smem = keys_bytes + plan_bytes <= limit ? 1 : 0;
+  const size_t smem = keys_bytes + (plan_smem ? plan_bytes : 0);
   static int attr_bits[2] = {0, 0};
   if (!smem_attr_done(reinterpret_cast<const void*>(h2o_select<NT>), attr_bits)) {
     cudaError_t err = cudaFuncSetAttribute(h2o_select<NT>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           kMaxCandidates * 4);
+                                           static_cast<int>(limit));
     if (err != cudaSuccess) return err;
   }
   cudaLaunchConfig_t cfg = {};
@@ -345,7 +404,7 @@ static cudaError_t launch_select(const EvictParams& e, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, h2o_select<NT>, e);
+  return cudaLaunchKernelEx(&cfg, h2o_select<NT>, e, plan_smem);
 }
 
 cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st) {
