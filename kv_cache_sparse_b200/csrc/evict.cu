@@ -71,10 +71,11 @@ __device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t* warp
 }
 
 // Copies the K and V rows of the placed tokens: the k-th token tok_of(k)
-// goes to slot slot_of(k), k < count.  The block walks the 16-byte vectors
-// of all rows (token-major: the K vectors, then the V vectors of a token), so
-// a warp reads and writes whole rows; each thread keeps kCopyBatch loads in
-// flight before it stores.
+// goes to slot slot_of(k), k < count.  A token's K row and V row are
+// per_tok = 2 * (16-byte vectors per row) consecutive vectors; thread t always
+// moves vector t % per_tok of tokens t / per_tok, + NT / per_tok, ... (per_tok
+// is 16, 32 or 64 and divides NT), so a warp reads and writes whole rows and
+// each thread keeps kCopyBatch loads in flight before it stores.
 constexpr int kCopyBatch = 8;
 
 template <int NT, class SlotOf, class TokOf>
@@ -82,37 +83,28 @@ __device__ __forceinline__ void copy_rows(const EvictParams& e, int b, int g, in
                                           SlotOf slot_of, TokOf tok_of) {
   const int vpr = e.d * e.esize / 16;  // vectors per row
   const int per_tok = 2 * vpr;
-  const int total = count * per_tok;
-  const size_t row_vecs = static_cast<size_t>(vpr);
-  const uint4* kn = static_cast<const uint4*>(e.k_new);
-  const uint4* vn = static_cast<const uint4*>(e.v_new);
-  uint4* kc = static_cast<uint4*>(e.k_cache);
-  uint4* vc = static_cast<uint4*>(e.v_cache);
-  const size_t head_row0 = (static_cast<size_t>(b) * e.Hkv + g) * e.C;
-  for (int v0 = threadIdx.x; v0 < total; v0 += kCopyBatch * NT) {
+  const int r = static_cast<int>(threadIdx.x) % per_tok;
+  const int tok_step = NT / per_tok;
+  const bool is_v = r >= vpr;
+  const int c = is_v ? r - vpr : r;
+  const size_t vpr_s = static_cast<size_t>(vpr);
+  // this thread's vector of new token 0 of (b, g), and of slot 0 of (b, g)
+  const uint4* src0 = static_cast<const uint4*>(is_v ? e.v_new : e.k_new) +
+                      (static_cast<size_t>(b) * e.nq * e.Hkv + g) * vpr_s + c;
+  uint4* dst0 = static_cast<uint4*>(is_v ? e.v_cache : e.k_cache) +
+                (static_cast<size_t>(b) * e.Hkv + g) * e.C * vpr_s + c;
+  const size_t src_tok = static_cast<size_t>(e.Hkv) * vpr_s;  // vectors between new tokens
+  for (int q0 = static_cast<int>(threadIdx.x) / per_tok; q0 < count; q0 += kCopyBatch * tok_step) {
     uint4 buf[kCopyBatch];
-    int to[kCopyBatch];  // (slot << 7) | vector within the token (per_tok <= 64), or -1
 #pragma unroll
     for (int u = 0; u < kCopyBatch; ++u) {
-      const int v = v0 + u * NT;
-      to[u] = -1;
-      if (v < total) {
-        const int q = v / per_tok, r = v - q * per_tok;
-        const bool is_v = r >= vpr;
-        const int c = is_v ? r - vpr : r;
-        const size_t src = ((static_cast<size_t>(b) * e.nq + tok_of(q)) * e.Hkv + g) * row_vecs + c;
-        buf[u] = __ldg((is_v ? vn : kn) + src);
-        to[u] = (slot_of(q) << 7) | r;
-      }
+      const int q = q0 + u * tok_step;
+      if (q < count) buf[u] = __ldg(src0 + static_cast<size_t>(tok_of(q)) * src_tok);
     }
 #pragma unroll
     for (int u = 0; u < kCopyBatch; ++u) {
-      if (to[u] >= 0) {
-        const int r = to[u] & 127;
-        const bool is_v = r >= vpr;
-        const size_t at = (head_row0 + (to[u] >> 7)) * row_vecs + (is_v ? r - vpr : r);
-        (is_v ? vc : kc)[at] = buf[u];
-      }
+      const int q = q0 + u * tok_step;
+      if (q < count) dst0[static_cast<size_t>(slot_of(q)) * vpr_s] = buf[u];
     }
   }
 }
