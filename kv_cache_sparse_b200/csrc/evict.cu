@@ -112,6 +112,106 @@ __device__ __forceinline__ void copy_rows(const EvictParams& e, int b, int g, in
 constexpr int kLoadBatch = 8;  // global loads in flight per thread in the first pass
 constexpr int kBins = 256;     // radix passes of 8 bits, most significant first
 
+// What the selection of one (cache, KV head) needs to know.
+struct SelectCtx {
+  float* score;        // [C] of this (cache, KV head)
+  const int* pos;      // [C]
+  const float* cs;     // summed weights: [n] cache slots, then [C + i] new token i
+  int n, nq, C, t0, sinks;
+  long long limit;     // positions >= limit are in the protected window
+  bool evict, by_score, old_protectable, need_pos;
+};
+
+// Step 1 for the candidates x in [x_lo, x_hi) (cache slot x < n, new token
+// x - n otherwise): accumulates the slots' scores and writes each
+// candidate's key to keys[x - x_lo].  kLoadBatch loads in flight per thread.
+template <int NT>
+__device__ __forceinline__ void build_keys(const SelectCtx& s, int x_lo, int x_hi,
+                                           uint32_t* keys) {
+  const int o_hi = min(x_hi, s.n);
+  for (int x0 = x_lo + static_cast<int>(threadIdx.x); x0 < o_hi; x0 += kLoadBatch * NT) {
+    float sc[kLoadBatch], cv[kLoadBatch];
+    int ps[kLoadBatch];
+#pragma unroll
+    for (int k = 0; k < kLoadBatch; ++k) {
+      const int x = x0 + k * NT;
+      sc[k] = 0.f;
+      cv[k] = 0.f;
+      ps[k] = -1;
+      if (x < o_hi) {
+        if (s.by_score) {
+          sc[k] = s.score[x];
+          cv[k] = s.cs[x];
+        }
+        if (s.need_pos) ps[k] = s.pos[x];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kLoadBatch; ++k) {
+      const int x = x0 + k * NT;
+      if (x < o_hi) {
+        const bool prot = s.old_protectable && (ps[k] >= s.limit || ps[k] < s.sinks);
+        uint32_t key;
+        if (s.by_score) {
+          const float v = sc[k] + cv[k];
+          s.score[x] = v;
+          key = score_key(v);
+        } else {
+          key = static_cast<uint32_t>(ps[k]);  // the most recent rank highest
+        }
+        keys[x - x_lo] = prot ? kProtectedKey : key;
+      }
+    }
+  }
+  for (int x0 = max(x_lo, s.n) + static_cast<int>(threadIdx.x); x0 < x_hi; x0 += kLoadBatch * NT) {
+    float cv[kLoadBatch];
+#pragma unroll
+    for (int k = 0; k < kLoadBatch; ++k) {
+      const int x = x0 + k * NT;
+      cv[k] = (s.by_score && x < x_hi) ? s.cs[s.C + (x - s.n)] : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < kLoadBatch; ++k) {
+      const int x = x0 + k * NT;
+      if (x < x_hi) {
+        const long long p = static_cast<long long>(s.t0) + (x - s.n);
+        const bool prot = s.evict && (p >= s.limit || p < s.sinks);
+        keys[x - x_lo] = prot ? kProtectedKey
+                              : (s.by_score ? score_key(cv[k]) : static_cast<uint32_t>(p));
+      }
+    }
+  }
+}
+
+// Warp 0 of the CTA: the bin of histogram h (scanned from the top) that holds
+// the k-th largest key, and the count of keys in the bins above it.
+__device__ __forceinline__ void find_bin(const int* h, int k, int lane, int* sel_bin,
+                                         int* sel_above) {
+  constexpr int per = kBins / 32;  // lane L looks at bins 255-8L .. 248-8L
+  int loc = 0;
+#pragma unroll
+  for (int e8 = 0; e8 < per; ++e8) loc += h[kBins - 1 - lane * per - e8];
+  int inc = loc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  int run = inc - loc;  // keys in higher bins than this lane's
+  if (run < k && run + loc >= k) {
+    for (int e8 = 0; e8 < per; ++e8) {
+      const int bin = kBins - 1 - lane * per - e8;
+      const int cnt = h[bin];
+      if (run + cnt >= k) {
+        *sel_bin = bin;
+        *sel_above = run;
+        break;
+      }
+      run += cnt;
+    }
+  }
+}
+
 template <int NT>
 __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
     h2o_select(const EvictParams e, int plan_smem) {
@@ -245,32 +345,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
       }
       __syncthreads();
     }
-    if (warp == 0) {
-      // lane L looks at bins nb-1-L*per .. nb-per-L*per (descending)
-      constexpr int per = nb / 32;
-      int loc = 0;
-#pragma unroll
-      for (int e8 = 0; e8 < per; ++e8) loc += hist[0][nb - 1 - lane * per - e8];
-      int inc = loc;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += y;
-      }
-      int run = inc - loc;  // keys in higher bins than this lane's
-      if (run < k && run + loc >= k) {
-        for (int e8 = 0; e8 < per; ++e8) {
-          const int bin = nb - 1 - lane * per - e8;
-          const int cnt = hist[0][bin];
-          if (run + cnt >= k) {
-            sel_bin = bin;
-            sel_above = run;
-            break;
-          }
-          run += cnt;
-        }
-      }
-    }
+    if (warp == 0) find_bin(hist[0], k, lane, &sel_bin, &sel_above);
     __syncthreads();
     prefix |= static_cast<uint32_t>(sel_bin) << shift;
     pmask |= static_cast<uint32_t>(nb - 1) << shift;
@@ -358,6 +433,211 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
                 [p_toks](int q) { return p_toks[q]; });
 }
 
+// h2o_select_cluster: the same selection for few (cache, KV head) units,
+// spread over a cluster of CL CTAs each, so that one unit's work runs on CL
+// SMs.  CTA r of the cluster holds the keys of candidates [r*share,
+// (r+1)*share).  Each radix pass counts into the CTA's own histogram (two
+// buffers, alternating between passes, so that one cluster barrier per pass
+// suffices), then every CTA sums the CL histograms through distributed shared
+// memory and finds the same digit.  The ordered compaction scans each CTA's
+// range, exchanges the CTA totals the same way and writes the plan to global
+// memory; after a cluster barrier (release / acquire) each CTA places its
+// share of the kept tokens.  Every CTA takes the same cluster barriers; none
+// leaves before the last one, after which no CTA reads another's memory.
+template <int NT, int CL>
+__global__ void __launch_bounds__(NT, 1) h2o_select_cluster(const EvictParams e) {
+  extern __shared__ uint32_t keys[];  // [share]: this CTA's candidates
+  __shared__ int hist[2][kBins];      // this CTA's counts, alternating buffers
+  __shared__ int tot[kBins];          // the cluster's counts of the current pass
+  __shared__ uint64_t warp_sums[32];
+  __shared__ uint64_t cta_total;      // this CTA's packed counters, read by the cluster
+  __shared__ uint64_t cl_before, cl_total;
+  __shared__ int sel_bin, sel_above;
+
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int bg = blockIdx.x / CL;
+  const int b = bg / e.Hkv, g = bg % e.Hkv;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int n = e.n, nq = e.nq, C = e.C;
+  const int NC = n + nq;
+  float* __restrict__ score = e.scores + static_cast<size_t>(bg) * C;
+  int* __restrict__ pos = e.pos + static_cast<size_t>(bg) * C;
+  const float* __restrict__ cs = e.colsum + static_cast<size_t>(bg) * e.colsum_ld;
+  int* __restrict__ slots = e.plan_slots + static_cast<size_t>(bg) * e.plan_ld;
+  int* __restrict__ toks = e.plan_tokens + static_cast<size_t>(bg) * e.plan_ld;
+  SelectCtx sx;
+  sx.score = score;
+  sx.pos = pos;
+  sx.cs = cs;
+  sx.n = n;
+  sx.nq = nq;
+  sx.C = C;
+  sx.t0 = e.t0;
+  sx.evict = NC > C;
+  sx.by_score = e.policy == kPolicyH2O;
+  sx.sinks = e.policy == kPolicySLR ? e.sinks : 0;
+  sx.limit = static_cast<long long>(e.t0) + nq - e.W;
+  sx.old_protectable = sx.evict && (e.W > nq || sx.sinks > 0);
+  sx.need_pos = sx.old_protectable || !sx.by_score;
+  const int share = (NC + CL - 1) / CL;
+  const int x_lo = min(NC, rank * share), x_hi = min(NC, x_lo + share);
+  const int len = x_hi - x_lo;
+  griddep_wait();  // the summed weights come from the preceding kernel
+  if (bg == 0 && rank == 0 && tid == 0) {
+    e.state[0] = min(C, n + nq);
+    e.state[1] = e.t0 + nq;
+  }
+
+  // 1. scores and keys of this CTA's candidates
+  build_keys<NT>(sx, x_lo, x_hi, keys);
+  if (!sx.evict) {
+    // fill phase: new token i goes to slot n + i; CTA r takes the tokens of
+    // its own share (no cluster barrier on this path)
+    const int qs = (nq + CL - 1) / CL;
+    const int i_lo = min(nq, rank * qs), i_hi = min(nq, i_lo + qs);
+    for (int i = i_lo + tid; i < i_hi; i += NT) {
+      slots[i] = n + i;
+      toks[i] = i;
+      score[n + i] = sx.by_score ? cs[C + i] : 0.f;
+      pos[n + i] = e.t0 + i;
+    }
+    if (rank == 0 && tid == 0) e.plan_count[bg] = nq;
+    copy_rows<NT>(e, b, g, i_hi - i_lo, [n, i_lo](int q) { return n + i_lo + q; },
+                  [i_lo](int q) { return i_lo + q; });
+    return;
+  }
+  __syncthreads();
+
+  // 2. radix select of the C-th largest key over the whole cluster
+  uint32_t prefix = 0, pmask = 0;
+  int k = C;  // rank (1-based, descending) still to locate
+  const int iters = (len + NT - 1) / NT;
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    int* my_hist = hist[pass & 1];
+    for (int i = tid; i < kBins; i += NT) my_hist[i] = 0;
+    __syncthreads();
+    for (int it = 0; it < iters; ++it) {
+      const int x = it * NT + tid;
+      int bin = -1;
+      if (x < len) {
+        const uint32_t key = keys[x];
+        if ((key & pmask) == prefix) bin = static_cast<int>((key >> shift) & (kBins - 1));
+      }
+      const unsigned same = __match_any_sync(0xffffffffu, bin);
+      if (bin >= 0 && (__ffs(same) - 1) == lane) atomicAdd(&my_hist[bin], __popc(same));
+    }
+    cluster_sync_all();  // every CTA's counts of this pass are complete
+    for (int i = tid; i < kBins; i += NT) {
+      const uint32_t a = smem_u32(&my_hist[i]);
+      int t = 0;
+#pragma unroll
+      for (int r = 0; r < CL; ++r) t += static_cast<int>(ld_dsmem_u32(dsmem_map(a, r)));
+      tot[i] = t;
+    }
+    __syncthreads();
+    if (warp == 0) find_bin(tot, k, lane, &sel_bin, &sel_above);
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(sel_bin) << shift;
+    pmask |= static_cast<uint32_t>(kBins - 1) << shift;
+    k -= sel_above;
+    // the buffer read above is cleared again two passes later, after the
+    // next pass's cluster barrier: every CTA has finished reading it by then
+  }
+  const uint32_t T = prefix;  // C-th largest key; keep the first k keys equal to T
+
+  // 3. ordered compaction (the packed counters of the single-CTA kernel),
+  //    first within the CTA, then across the cluster in rank order
+  const int per = (len + NT - 1) / NT;
+  const int lo = min(len, tid * per), hi = min(len, lo + per);
+  int fo_s = 0, nn_s = 0, eq = 0, eq_old = 0;
+  for (int j = lo; j < hi; ++j) {
+    const uint32_t key = keys[j];
+    const int x = x_lo + j;
+    if (key == T) {
+      ++eq;
+      eq_old += x < n;
+    } else if (key > T) {
+      nn_s += x >= n;
+    } else {
+      fo_s += x < n;
+    }
+  }
+  uint64_t cta_sum;
+  const uint64_t in_cta = block_excl_scan64<NT>(
+      static_cast<uint64_t>(fo_s) | (static_cast<uint64_t>(nn_s) << 16) |
+          (static_cast<uint64_t>(eq) << 32) | (static_cast<uint64_t>(eq_old) << 48),
+      warp_sums, &cta_sum);
+  if (tid == 0) cta_total = cta_sum;
+  cluster_sync_all();  // every CTA's total is published
+  if (warp == 0) {
+    const uint64_t v = lane < CL ? ld_dsmem_u64(dsmem_map(smem_u32(&cta_total), lane)) : 0;
+    uint64_t before = 0, all = 0;
+#pragma unroll
+    for (int r = 0; r < CL; ++r) {
+      const uint64_t t = __shfl_sync(0xffffffffu, v, r);
+      all += t;
+      if (r < rank) before += t;
+    }
+    if (lane == 0) {
+      cl_before = before;
+      cl_total = all;
+    }
+  }
+  __syncthreads();
+  auto field = [](uint64_t v, int f) { return static_cast<int>((v >> (16 * f)) & 0xFFFF); };
+  const uint64_t pk_before = cl_before + in_cta, pk_tot = cl_total;
+  const int eq_b = field(pk_before, 2), eqo_b = field(pk_before, 3);
+  const int fo_before = field(pk_before, 0) + eqo_b - min(eqo_b, k);
+  const int nw_before = field(pk_before, 1) + min(eq_b, k) - min(eqo_b, k);
+  const int eq_t = field(pk_tot, 2), eqo_t = field(pk_tot, 3);
+  const int tot_free_old = field(pk_tot, 0) + eqo_t - min(eqo_t, k);
+  const int tot_new = field(pk_tot, 1) + min(eq_t, k) - min(eqo_t, k);
+  // empty slots n .. C-1 are free too: the cluster's threads take fixed shares
+  const int empty = C - n;
+  const int gt = rank * NT + tid;
+  const int e_per = (empty + CL * NT - 1) / (CL * NT);
+  const int e_lo = n + min(empty, gt * e_per), e_hi = n + min(empty, (gt + 1) * e_per);
+  const bool bad = tot_free_old + empty != tot_new;  // the same in every CTA
+  if (!bad) {
+    int fo = fo_before, nw = nw_before, eq_rank = eq_b;
+    for (int j = lo; j < hi; ++j) {
+      const uint32_t key = keys[j];
+      const int x = x_lo + j;
+      bool kept = key > T;
+      if (key == T) kept = eq_rank++ < k;
+      if (x < n) {
+        if (!kept) slots[fo++] = x;
+      } else if (kept) {
+        toks[nw++] = x - n;
+      }
+    }
+    int em = tot_free_old + (e_lo - n);
+    for (int s2 = e_lo; s2 < e_hi; ++s2) slots[em++] = s2;
+  }
+  cluster_sync_all();  // the plan is complete; no CTA reads another's shared memory after this
+  if (bad) {
+    if (rank == 0 && tid == 0) {
+      atomicOr(e.state + 2, kDevErrPlan);
+      e.plan_count[bg] = 0;
+    }
+    return;
+  }
+  // 4. this CTA's share of the placed tokens: scores, positions, K/V rows
+  const int qs = (tot_new + CL - 1) / CL;
+  const int q_lo = min(tot_new, rank * qs), q_hi = min(tot_new, q_lo + qs);
+  for (int q = q_lo + tid; q < q_hi; q += NT) {
+    const int s2 = slots[q], i = toks[q];
+    score[s2] = sx.by_score ? cs[C + i] : 0.f;
+    pos[s2] = e.t0 + i;
+  }
+  if (rank == 0 && tid == 0) e.plan_count[bg] = tot_new;
+  copy_rows<NT>(e, b, g, q_hi - q_lo, [slots, q_lo](int q) { return slots[q_lo + q]; },
+                [toks, q_lo](int q) { return toks[q_lo + q]; });
+}
+
 // Dynamic shared memory the selection kernel can take next to its static
 // arrays (histograms, scan sums).
 template <int NT>
@@ -399,10 +679,38 @@ static cudaError_t launch_select(const EvictParams& e, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, h2o_select<NT>, e, plan_smem);
 }
 
+// Cluster variant: kClusterCtas CTAs of kClusterThreads per (cache, KV head),
+// used while the units fill at most kClusterUnits * kClusterCtas SMs.
+constexpr int kClusterCtas = 8;
+constexpr int kClusterThreads = 512;
+constexpr int kClusterUnits = 16;
+
+static cudaError_t launch_select_cluster(const EvictParams& e, cudaStream_t st) {
+  constexpr int CL = kClusterCtas, NT = kClusterThreads;
+  const int share = (e.n + e.nq + CL - 1) / CL;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(e.B * e.Hkv * CL);
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = static_cast<size_t>(share) * sizeof(uint32_t);  // <= 25 KiB
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, h2o_select_cluster<NT, CL>, e);
+}
+
 cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st) {
   (void)max_chunk;
-  // few (cache, KV head) units: one large CTA each, to cut the latency of
-  // each selection; many units: smaller CTAs, several per SM
+  // few (cache, KV head) units: a cluster of CTAs each, so that a unit's
+  // selection runs on several SMs; many units: one CTA each (smaller CTAs,
+  // several per SM, once the units outnumber the SMs twice)
+  if (e.B * e.Hkv <= kClusterUnits) return launch_select_cluster(e, st);
   if (e.B * e.Hkv >= 2 * 148) return launch_select<256>(e, st);
   return launch_select<1024>(e, st);
 }

@@ -28,6 +28,9 @@ CASES = [
     (1, 8, 128, 8192, 8192, 1024, 256, None, torch.bfloat16),  # full-size shape
     (1, 2, 64, 256, 256, 64, 0, None, torch.float32),    # fp32 cache
     (4, 2, 64, 33, 20, 20, 5, 3, torch.float32),         # tiny, odd sizes
+    (1, 1, 64, 5, 5, 1, 0, None, torch.bfloat16),        # 6 candidates: some cluster CTAs hold none
+    (4, 8, 128, 512, 512, 128, 16, None, torch.bfloat16),  # 32 units: one 1024-thread CTA each
+    (3, 8, 64, 300, 250, 100, 120, 3, torch.bfloat16),   # 24 units, partial fill, W > nq, ties
     (40, 8, 64, 96, 96, 32, 8, 3, torch.bfloat16),       # 320 units: the many-cache variant
     (40, 8, 64, 300, 250, 100, 120, None, torch.bfloat16),  # many units, partial fill, W > nq
 ]
