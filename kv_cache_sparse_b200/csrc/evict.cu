@@ -4,8 +4,10 @@
 // evicts when it is full; summary page glossary "H2O": entries are scored by
 // the attention they accumulated and the less important ones evicted.
 //
-// h2o_select (one 1024-thread CTA per (cache, KV head); candidates in shared
-// memory):
+// Per (cache, KV head), with the candidates' keys in shared memory -- one
+// CTA (h2o_select: 1024 threads, or 256 when the units outnumber the SMs
+// twice) or, for up to 16 units, a cluster of 8 CTAs (h2o_select_cluster,
+// below) -- the selection runs these steps:
 //   1. score[s] <- fl32(score[s] + colsum[s]) for the n valid slots; new token
 //      i's candidate score is colsum[C + i].  The score-free policies (LR,
 //      SLR) rank by position instead: a candidate's key is its position, no
