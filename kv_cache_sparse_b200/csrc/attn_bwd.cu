@@ -143,6 +143,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       p.dk_cache[at] = 0.f;
       p.dv_cache[at] = 0.f;
     }
+    griddep_wait();  // see the end of the kernel
     return;
   }
   const int qt_min = is_chunk ? kt : 0;
@@ -378,6 +379,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // this grid may overlap the dQ grid before it (programmatic launch: they
+  // share no data); it completes only after that grid has, so the stream's
+  // later work sees both
+  griddep_wait();
 }
 
 // ---------------------------------------------------------------- dQ
@@ -416,6 +421,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int b = bh / p.Hq, h = bh % p.Hq, g = h / p.G;
   const int NCT = cdiv(p.n, 128);
   const int T = NCT + qt + 1;  // cache tiles, then chunk tiles 0..qt
+  // the dK/dV grid (launched next, programmatically) may fill the SMs this
+  // grid's last wave leaves idle
+  griddep_launch_dependents();
 
   const uint32_t bar_qd = sbase + L::kBarOff;
   const uint32_t bar_full0 = bar_qd + 8;
@@ -657,13 +665,24 @@ static cudaError_t launch_bwd_d(const BwdMaps& m, const BwdParams& p, const void
                              DqLayout<D>::kAlloc);
     if (e != cudaSuccess) return e;
   }
-  bwd_dkdv<D><<<dim3(cdiv(p.C, 128) + cdiv(p.nq, 128), p.B * p.Hkv), kBwdThreads,
-                DkdvLayout<D>::kAlloc, st>>>(m.q, m.dout, m.kc, m.vc, m.kn, m.vn, p);
+  // dQ first (256 CTAs on the headline cache: 1.7 waves), then dK/dV, which
+  // needs nothing from dQ and starts its CTAs on the SMs dQ's last wave
+  // leaves idle
+  bwd_dq<D><<<p.B * p.Hq * cdiv(p.nq, 128), kBwdThreads, DqLayout<D>::kAlloc, st>>>(
+      m.q, m.dout, m.kc, m.vc, m.kn, m.vn, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dq<D><<<p.B * p.Hq * cdiv(p.nq, 128), kBwdThreads, DqLayout<D>::kAlloc, st>>>(m.q, m.dout, m.kc, m.vc,
-                                                                           m.kn, m.vn, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cdiv(p.C, 128) + cdiv(p.nq, 128), p.B * p.Hkv);
+  cfg.blockDim = dim3(kBwdThreads);
+  cfg.dynamicSmemBytes = DkdvLayout<D>::kAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, bwd_dkdv<D>, m.q, m.dout, m.kc, m.vc, m.kn, m.vn, p);
 }
 
 cudaError_t launch_attn_bwd_bf16(int head_dim, const BwdMaps& m, const BwdParams& p,
