@@ -78,3 +78,26 @@ def test_null_arguments_rejected(lib):
     assert lib.h2o_chunk_step(None, None, None, None, 1, None, None, None) == 1
     assert lib.h2o_cache_check(None, None) == 1
     assert lib.h2o_status_string(6) == b"device wait timed out"
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """No silent fallback: without the built library the binding raises."""
+    with pytest.raises(ImportError, match="is missing"):
+        binding.load_library(str(tmp_path / "libh2o.so"))
+
+
+def test_product_package_does_not_import_the_oracle():
+    """The oracle is test infrastructure: importing the package and its
+    binding, workloads and build modules loads nothing from oracle/."""
+    import subprocess
+    import sys
+    code = ("import sys, kv_cache_sparse_b200, kv_cache_sparse_b200.binding, "
+            "kv_cache_sparse_b200.workloads, kv_cache_sparse_b200.build; "
+            "bad = [m for m in sys.modules if m == 'oracle' or m.startswith('oracle.')]; "
+            "sys.exit(1 if bad else 0)")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    for name in os.listdir(os.path.join(ROOT, "kv_cache_sparse_b200")):
+        if name.endswith(".py"):
+            text = open(os.path.join(ROOT, "kv_cache_sparse_b200", name)).read()
+            assert not re.search(r"^\s*(from|import)\s+oracle\b", text, flags=re.M), name
