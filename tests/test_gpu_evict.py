@@ -31,6 +31,7 @@ CASES = [
     (1, 1, 64, 5, 5, 1, 0, None, torch.bfloat16),        # 6 candidates: some cluster CTAs hold none
     (4, 8, 128, 512, 512, 128, 16, None, torch.bfloat16),  # 32 units: one 1024-thread CTA each
     (3, 8, 64, 300, 250, 100, 120, 3, torch.bfloat16),   # 24 units, partial fill, W > nq, ties
+    (1, 1, 64, 49152, 49152, 1024, 64, None, torch.bfloat16),  # the most candidates a cache takes (C + nq = 50176)
     (40, 8, 64, 96, 96, 32, 8, 3, torch.bfloat16),       # 320 units: the many-cache variant
     (40, 8, 64, 300, 250, 100, 120, None, torch.bfloat16),  # many units, partial fill, W > nq
 ]
