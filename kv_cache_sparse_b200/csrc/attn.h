@@ -22,7 +22,9 @@ struct BwdMaps {
   CUtensorMap q, dout, kc, vc, kn, vn;
 };
 
-// Records that a kernel's shared-memory opt-in was set on the current device.
+// One-time function attributes per device: returns true when the caller's
+// bit for the current device was already set, else sets it (atomically) and
+// returns false, so that the caller sets the attribute.
 bool smem_attr_done(const void* fn, int* slot_bits);
 
 // K1: attention forward + row statistics (tcgen05), head_dim 64 or 128.

@@ -410,9 +410,9 @@ bool smem_attr_done(const void* fn, int* slot_bits) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   const int w = dev / 32, bit = 1 << (dev % 32);
-  if (slot_bits[w] & bit) return true;
-  slot_bits[w] |= bit;
-  return false;
+  // atomic: handles may be used from different host threads at once (setting
+  // a function attribute twice is harmless)
+  return (__atomic_fetch_or(&slot_bits[w], bit, __ATOMIC_ACQ_REL) & bit) != 0;
 }
 }  // namespace h2o
 
