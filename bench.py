@@ -476,6 +476,12 @@ def run_ours(args, world, rank, local):
         "clocks": clocks.summary(),
     }
     line.update(extra)
+    if wl.layers > 1:
+        # a model step advances every layer's cache by one chunk: the rate of
+        # one sequence batch through all the model's layers
+        line["model_tokens_per_s"] = {
+            "value": round(value / wl.layers, 1), "unit": "tokens/s",
+            "per": f"{wl.seqs} sequences x {wl.layers} layers (chunk-tokens/s / {wl.layers})"}
     if bwd is not None:
         line["backward"] = bwd
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
