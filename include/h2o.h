@@ -258,21 +258,33 @@ H2O_API h2o_status h2o_cache_kernel_ms(h2o_cache* c, float* ms4);
  * n valid slots, q, k_new, v_new (device, chunk layouts).  Outputs (device):
  * out, and colsum_out in the colsum layout for this n_q (required).
  * The first call on a device looks up the array's device address on the
- * current device (cudaGetSymbolAddress); make that first call before any
- * stream capture.  All calls on a device share the array and it keeps the
- * last call's contents (nothing in it needs clearing between calls), so
- * calls that overlap on the GPU race on it: serialise them. */
+ * current device (cudaGetSymbolAddress; safe if several host threads make
+ * it at once); make that first call before any stream capture.  All calls
+ * on a device share the array and it keeps the last call's contents
+ * (nothing in it needs clearing between calls), so calls that overlap on
+ * the GPU race on it: serialise them.  A static error word beside it is
+ * cleared at the start of every call (cudaMemsetAsync on `stream`) and
+ * latches an expired bounded wait of that call's kernels, in which case out
+ * and colsum_out are incomplete: h2o_static_scratch_check reports it. */
 H2O_API h2o_status h2o_attention_static_scratch(const h2o_config* cfg, const void* k_cache,
                                                 const void* v_cache, int32_t n, const void* q,
                                                 const void* k_new, const void* v_new,
                                                 int32_t n_q, void* out, float* colsum_out,
                                                 void* stream);
 
+/* Status of the last h2o_attention_static_scratch call on the current
+ * device: synchronises `stream` (the stream of that call), then returns
+ * H2O_ERR_TIMEOUT if one of its kernels' bounded waits expired (its outputs
+ * are then incomplete), H2O_OK otherwise (or H2O_ERR_CUDA).  No counterpart
+ * in the paper; allocates nothing. */
+H2O_API h2o_status h2o_static_scratch_check(void* stream);
+
 /* Diagnostic of the failure path: one warp waits, with the same bounded
  * wait the kernels use, on a barrier nothing completes.  After limit_us
  * (1 .. 2,000,000) the wait gives up, ORs the timeout bit (1) into
- * *err_word (device int32) and the kernel returns; the context stays
- * usable.  No trap, no hang. */
+ * *err_word (device int32; NULL selects the error word that
+ * h2o_static_scratch_check reports) and the kernel returns; the context
+ * stays usable.  No trap, no hang. */
 H2O_API h2o_status h2o_selftest_wait_timeout(int32_t* err_word, uint32_t limit_us,
                                              void* stream);
 

@@ -23,9 +23,11 @@ STATUS_NAMES = {0: "H2O_OK", 1: "H2O_ERR_INVALID_ARG", 2: "H2O_ERR_SHAPE", 3: "H
                 4: "H2O_ERR_ALIGN", 5: "H2O_ERR_CUDA", 6: "H2O_ERR_TIMEOUT", 7: "H2O_ERR_STATE"}
 
 EXPORTED = ["h2o_required_bytes", "h2o_cache_create", "h2o_chunk_step", "h2o_chunk_step_host",
-            "h2o_cache_host_join", "h2o_attention", "h2o_attention_backward", "h2o_evict", "h2o_cache_read", "h2o_cache_write",
-            "h2o_cache_check", "h2o_cache_info", "h2o_cache_set_timing", "h2o_cache_kernel_ms",
-            "h2o_cache_destroy", "h2o_status_string"]
+            "h2o_cache_host_join", "h2o_attention", "h2o_attention_backward", "h2o_evict",
+            "h2o_cache_read", "h2o_cache_write", "h2o_cache_check", "h2o_cache_info",
+            "h2o_cache_set_timing", "h2o_cache_kernel_ms", "h2o_attention_static_scratch",
+            "h2o_static_scratch_check", "h2o_selftest_wait_timeout", "h2o_cache_destroy",
+            "h2o_status_string"]
 
 
 class H2OError(RuntimeError):
@@ -65,6 +67,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                      ctypes.POINTER(P)]
     for name in ("h2o_chunk_step", "h2o_chunk_step_host", "h2o_attention"):
         getattr(lib, name).argtypes = [P, P, P, P, I, P, P, P]
+    lib.h2o_cache_host_join.argtypes = [P, P]
+    lib.h2o_attention_backward.argtypes = [P, P, P, P, I, P, P, P, P, P, P, P, P]
+    lib.h2o_attention_static_scratch.argtypes = [ctypes.POINTER(Config), P, P, I, P, P, P, I, P,
+                                                 P, P]
+    lib.h2o_static_scratch_check.argtypes = [P]
+    lib.h2o_selftest_wait_timeout.argtypes = [P, ctypes.c_uint32, P]
     lib.h2o_evict.argtypes = [P, P, P, P, I, P]
     lib.h2o_cache_read.argtypes = [P, P, P, P, P, P, P]
     lib.h2o_cache_write.argtypes = [P, P, P, P, P, P, P]

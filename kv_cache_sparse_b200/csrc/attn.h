@@ -22,10 +22,12 @@ struct BwdMaps {
   CUtensorMap q, dout, kc, vc, kn, vn;
 };
 
-// One-time function attributes per device: returns true when the caller's
-// bit for the current device was already set, else sets it (atomically) and
-// returns false, so that the caller sets the attribute.
-bool smem_attr_done(const void* fn, int* slot_bits);
+// Raises the kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per device.  The device's bit in slot_bits is set only after
+// cudaFuncSetAttribute succeeded, so a thread that sees it set may launch;
+// threads that see it clear all make the (idempotent) call themselves, and
+// a failed call is retried by the next launch.
+cudaError_t ensure_smem_attr(const void* fn, int bytes, int* slot_bits);
 
 // K1: attention forward + row statistics (tcgen05), head_dim 64 or 128.
 cudaError_t launch_attn_fwd_bf16(int head_dim, const AttnMaps& m, const AttnParams& p,
@@ -49,6 +51,10 @@ bool decode_supported(int G);
 // dQ; out and dout are [B, nq, Hq, d] bf16.
 cudaError_t launch_attn_bwd_bf16(int head_dim, const BwdMaps& m, const BwdParams& p,
                                  const void* out, const void* dout, cudaStream_t st);
+
+// Device address of the error word of h2o_attention_static_scratch on the
+// current device (null if it cannot be resolved).
+int* static_scratch_error_word();
 
 // K3 (with the K/V scatter fused): score update, selection, placement.
 cudaError_t launch_evict(const EvictParams& e, int max_chunk, cudaStream_t st);

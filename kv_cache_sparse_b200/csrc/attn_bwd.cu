@@ -655,16 +655,10 @@ static cudaError_t launch_bwd_d(const BwdMaps& m, const BwdParams& p, const void
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   static int bits_a[2] = {0, 0}, bits_b[2] = {0, 0};
-  if (!smem_attr_done(reinterpret_cast<const void*>(bwd_dkdv<D>), bits_a)) {
-    e = cudaFuncSetAttribute(bwd_dkdv<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DkdvLayout<D>::kAlloc);
-    if (e != cudaSuccess) return e;
-  }
-  if (!smem_attr_done(reinterpret_cast<const void*>(bwd_dq<D>), bits_b)) {
-    e = cudaFuncSetAttribute(bwd_dq<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DqLayout<D>::kAlloc);
-    if (e != cudaSuccess) return e;
-  }
+  e = ensure_smem_attr(reinterpret_cast<const void*>(bwd_dkdv<D>), DkdvLayout<D>::kAlloc, bits_a);
+  if (e != cudaSuccess) return e;
+  e = ensure_smem_attr(reinterpret_cast<const void*>(bwd_dq<D>), DqLayout<D>::kAlloc, bits_b);
+  if (e != cudaSuccess) return e;
   // dQ first (256 CTAs on the headline cache: 1.7 waves), then dK/dV, which
   // needs nothing from dQ and starts its CTAs on the SMs dQ's last wave
   // leaves idle

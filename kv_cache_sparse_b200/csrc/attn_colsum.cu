@@ -292,11 +292,9 @@ template <int D>
 static cudaError_t launch_colsum(const AttnMaps& m, const AttnParams& p, cudaStream_t st) {
   using L = ColLayout<D>;
   static int attr_bits[2] = {0, 0};
-  if (!smem_attr_done(reinterpret_cast<const void*>(attn_colsum_kernel<D>), attr_bits)) {
-    cudaError_t e = cudaFuncSetAttribute(attn_colsum_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-    if (e != cudaSuccess) return e;
-  }
+  cudaError_t e =
+      ensure_smem_attr(reinterpret_cast<const void*>(attn_colsum_kernel<D>), L::kAlloc, attr_bits);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cdiv(p.C, 128) + cdiv(p.nq, 128), p.B * p.Hkv);
   cfg.blockDim = dim3(L::kThreads);

@@ -388,11 +388,9 @@ template <int D>
 static cudaError_t launch_fwd(const AttnMaps& m, const AttnParams& p, cudaStream_t st) {
   using L = FwdLayout<D>;
   static int attr_bits[2] = {0, 0};
-  if (!smem_attr_done(reinterpret_cast<const void*>(attn_fwd_kernel<D>), attr_bits)) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-    if (e != cudaSuccess) return e;
-  }
+  cudaError_t e =
+      ensure_smem_attr(reinterpret_cast<const void*>(attn_fwd_kernel<D>), L::kAlloc, attr_bits);
+  if (e != cudaSuccess) return e;
   const int pairs = cdiv(p.G * cdiv(p.nq, 128), 2);
   const int grid = p.B * p.Hkv * pairs;
   attn_fwd_kernel<D><<<grid, L::kThreads, L::kAlloc, st>>>(m.q, m.kc, m.vc, m.kn, m.vn, p);

@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <stdint.h>
+#include <string.h>
 
 namespace h2o {
 
@@ -24,6 +25,18 @@ constexpr int kTileKeys = 128;  // keys per attention tile
 constexpr int kMaxCandidates = 50176;
 
 __host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// A 32-bit key that orders like the fp32 value, negative values included:
+// non-negative values get the sign bit set, negative ones all bits flipped;
+// -0 is +0.  The largest key (0xFFFFFFFF) is left free for the selection's
+// "protected" mark (only a NaN pattern would map there).
+__host__ __device__ inline uint32_t ordered_key(float v) {
+  uint32_t u;
+  memcpy(&u, &v, sizeof(u));
+  if (u == 0x80000000u) u = 0u;
+  const uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return k == 0xFFFFFFFFu ? 0xFFFFFFFEu : k;
+}
 
 // ---------------------------------------------------------------- attention
 

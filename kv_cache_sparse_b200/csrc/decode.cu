@@ -390,9 +390,9 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
     return;
   }
   // full: this slice's candidate.  Unprotected: position < t0 + 1 - W (and,
-  // under SLR, >= the sink count).  Key: rank value (score bits -- scores are
-  // >= 0 -- or position) then the inverted index, so that the minimum is the
-  // lowest value with the highest index.
+  // under SLR, >= the sink count).  Key: rank value (the score as an
+  // order-preserving key, or the position) then the inverted index, so that
+  // the minimum is the lowest value with the highest index.
   const long long limit = static_cast<long long>(p.t0) + 1 - p.W;
   unsigned long long best = ~0ull;
   for (int s = sa + tid; s < sb; s += kThreads) {
@@ -401,7 +401,7 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
     if (by_score) {
       const float sc = __fadd_rn(score[s], cs[s]);
       score[s] = sc;
-      rank = __float_as_uint(sc);
+      rank = ordered_key(sc);
     } else {
       rank = static_cast<uint32_t>(ps);
     }
@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
     }
   }
   if (last_slice && tid == 0 && p.t0 < limit && p.t0 >= sinks) {  // W = 0: the new token competes
-    const uint32_t rank = by_score ? __float_as_uint(cs[C]) : static_cast<uint32_t>(p.t0);
+    const uint32_t rank = by_score ? ordered_key(cs[C]) : static_cast<uint32_t>(p.t0);
     const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - C);
     best = key < best ? key : best;
   }
@@ -455,11 +455,9 @@ template <typename T, int D, int G>
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t st) {
   using L = PartialLayout<T, D, G>;
   static int attr_bits[2] = {0, 0};
-  if (!smem_attr_done(reinterpret_cast<const void*>(decode_partial<T, D, G>), attr_bits)) {
-    cudaError_t e = cudaFuncSetAttribute(decode_partial<T, D, G>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
-    if (e != cudaSuccess) return e;
-  }
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(decode_partial<T, D, G>),
+                                   L::kBytes, attr_bits);
+  if (e != cudaSuccess) return e;
   decode_partial<T, D, G><<<dim3(p.n_chunks, p.B * p.Hkv), kThreads, L::kBytes, st>>>(p);
   return cudaGetLastError();
 }

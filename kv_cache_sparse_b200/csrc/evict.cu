@@ -15,8 +15,9 @@
 //      positions below the sink count.
 //   2. If n + nq <= C every new token is kept and goes to slot n + i.
 //   3. Otherwise a candidate at position >= t0 + nq - W is protected.  Each
-//      candidate gets a 32-bit key: 0xFFFFFFFF when protected, else the bit
-//      pattern of its (non-negative) fp32 score, which orders like the score.
+//      candidate gets a 32-bit key: 0xFFFFFFFF when protected, else its fp32
+//      score mapped to a key that orders like the score (negative scores
+//      included), or its position for LR / SLR.
 //      A 4 x 8-bit MSB-first radix select finds the C-th largest key T and
 //      how many keys equal to T are kept; those are the ones of lowest
 //      candidate index (slot s -> s, new token i -> n + i; same order as the
@@ -35,10 +36,7 @@ namespace h2o {
 
 constexpr uint32_t kProtectedKey = 0xFFFFFFFFu;
 
-__device__ __forceinline__ uint32_t score_key(float s) {
-  uint32_t u = __float_as_uint(s);
-  return u == 0x80000000u ? 0u : u;  // -0 orders as +0
-}
+__device__ __forceinline__ uint32_t score_key(float s) { return ordered_key(s); }
 
 // Exclusive scan of one 64-bit value per thread over the block (four packed
 // 16-bit counters: no field carries into the next while every block total
@@ -662,12 +660,9 @@ static cudaError_t launch_select(const EvictParams& e, cudaStream_t st) {
   const int plan_smem = keys_bytes + plan_bytes <= limit ? 1 : 0;
   const size_t smem = keys_bytes + (plan_smem ? plan_bytes : 0);
   static int attr_bits[2] = {0, 0};
-  if (!smem_attr_done(reinterpret_cast<const void*>(h2o_select<NT>), attr_bits)) {
-    cudaError_t err = cudaFuncSetAttribute(h2o_select<NT>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(limit));
-    if (err != cudaSuccess) return err;
-  }
+  cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(h2o_select<NT>),
+                                     static_cast<int>(limit), attr_bits);
+  if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(e.B * e.Hkv);
   cfg.blockDim = dim3(NT);

@@ -19,6 +19,8 @@
 
 #include <new>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/h2o.h"
 #include "attn.h"
 
@@ -70,6 +72,16 @@ struct h2o_cache {
 namespace {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// NVTX range around the host-side launch of one kernel (or kernel pair), so
+// that a profiler's timeline names each part of the step; costs a pointer
+// check when no tool is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 size_t esize_of(h2o_dtype t) { return t == H2O_BF16 ? 2 : 4; }
 
@@ -237,12 +249,14 @@ h2o_status run_attention(h2o_cache* c, const void* q, const void* kn, const void
   for (int i = 0; i < 5; ++i) c->ev_used[i] = false;
   mark(c, 0, st);
   if (g.dtype == H2O_F32) {
+    NvtxRange r("h2o attention f32 (K1+K2)");
     cudaError_t e = launch_attn_f32(g.head_dim, static_cast<const float*>(q),
                                     static_cast<const float*>(c->buf.k),
                                     static_cast<const float*>(c->buf.v),
                                     static_cast<const float*>(kn), static_cast<const float*>(vn),
                                     p, st);
     c->launches += (c->n < g.capacity) ? 3 : 2;
+    mark(c, 1, st);  // the fp32 kernels are reported together as the first part
     mark(c, 2, st);
     return cuda_status(e);
   }
@@ -254,13 +268,18 @@ h2o_status run_attention(h2o_cache* c, const void* q, const void* kn, const void
       !encode_cache(&m.kc, c->buf.k, BH, c->n, g.capacity, g.head_dim) ||
       !encode_cache(&m.vc, c->buf.v, BH, c->n, g.capacity, g.head_dim))
     return H2O_ERR_CUDA;
-  cudaError_t e = launch_attn_fwd_bf16(g.head_dim, m, p, st);
+  cudaError_t e;
+  {
+    NvtxRange r("h2o K1 attention forward");
+    e = launch_attn_fwd_bf16(g.head_dim, m, p, st);
+  }
   if (e != cudaSuccess) return H2O_ERR_CUDA;
   c->launches += 1;
   c->fwd_nq = nq;  // the row statistics of this call stay for a backward
   c->fwd_n = c->n;
   mark(c, 1, st);
   if (with_colsum) {
+    NvtxRange r("h2o K2 summed weights");
     e = launch_attn_colsum_bf16(g.head_dim, m, p, st);
     if (e != cudaSuccess) return H2O_ERR_CUDA;
     c->launches += 1;
@@ -303,7 +322,11 @@ h2o_status run_evict(h2o_cache* c, const float* colsum, int ld, const void* kn, 
     for (int i = 0; i < 5; ++i) c->ev_used[i] = false;
     mark(c, 2, st);
   }
-  cudaError_t err = launch_evict(e, g.max_chunk, st);
+  cudaError_t err;
+  {
+    NvtxRange r("h2o K3 score update + selection + scatter");
+    err = launch_evict(e, g.max_chunk, st);
+  }
   if (err != cudaSuccess) return H2O_ERR_CUDA;
   c->fwd_nq = 0;  // the cache changes: no backward of the earlier attention
   c->launches += 1;
@@ -363,8 +386,11 @@ h2o_status run_decode(h2o_cache* c, const void* q, const void* kn, const void* v
   d.sinks = g.sink_tokens;
   for (int i = 0; i < 5; ++i) c->ev_used[i] = false;
   mark(c, 0, st);
-  if (launch_decode(d, static_cast<int>(esize_of(g.dtype)), g.head_dim, st) != cudaSuccess)
-    return H2O_ERR_CUDA;
+  {
+    NvtxRange r("h2o decode step (split-KV attention, merge, eviction)");
+    if (launch_decode(d, static_cast<int>(esize_of(g.dtype)), g.head_dim, st) != cudaSuccess)
+      return H2O_ERR_CUDA;
+  }
   c->fwd_nq = 0;  // the decode path keeps no row statistics
   c->launches += 2;
   mark(c, 1, st);  // both kernels are reported as the first part
@@ -405,14 +431,18 @@ h2o_status host_streams(h2o_cache* c) {
 }  // namespace
 
 namespace h2o {
-bool smem_attr_done(const void* fn, int* slot_bits) {
-  (void)fn;
+cudaError_t ensure_smem_attr(const void* fn, int bytes, int* slot_bits) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  const int w = dev / 32, bit = 1 << (dev % 32);
-  // atomic: handles may be used from different host threads at once (setting
-  // a function attribute twice is harmless)
-  return (__atomic_fetch_or(&slot_bits[w], bit, __ATOMIC_ACQ_REL) & bit) != 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool tracked = dev >= 0 && dev < 64;
+  const int w = tracked ? dev / 32 : 0, bit = tracked ? 1 << (dev % 32) : 0;
+  // handles may be used from different host threads at once: the bit is a
+  // fast path published after the attribute is in place (acquire / release)
+  if (tracked && (__atomic_load_n(&slot_bits[w], __ATOMIC_ACQUIRE) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && tracked) __atomic_fetch_or(&slot_bits[w], bit, __ATOMIC_RELEASE);
+  return e;
 }
 }  // namespace h2o
 
@@ -547,9 +577,12 @@ h2o_status h2o_attention_backward(h2o_cache* c, const void* q, const void* k_new
       !encode_cache(&m.kc, c->buf.k, BH, c->n, g.capacity, g.head_dim) ||
       !encode_cache(&m.vc, c->buf.v, BH, c->n, g.capacity, g.head_dim))
     return H2O_ERR_CUDA;
-  if (launch_attn_bwd_bf16(g.head_dim, m, p, out, d_out, static_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
-    return H2O_ERR_CUDA;
+  {
+    NvtxRange r("h2o attention backward (row dots, dQ, dK/dV)");
+    if (launch_attn_bwd_bf16(g.head_dim, m, p, out, d_out, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+      return H2O_ERR_CUDA;
+  }
   c->launches += 3;
   return H2O_OK;
 }

@@ -17,8 +17,14 @@
 // exits.  Every call on a device uses the same array and it keeps the last
 // call's contents.  Nothing in it has to start at zero: the first kernel of
 // a call writes every row the second kernel of that call reads.  Calls whose
-// work overlaps on the GPU (two streams, or two host threads) race on it.
+// work overlaps on the GPU (two streams, or two host threads) race on it.  A
+// second static word records an expired bounded wait: each call clears it
+// first (cudaMemsetAsync on its device address, which allocates nothing) and
+// h2o_static_scratch_check reports it.
 #include <math.h>
+
+#include <atomic>
+#include <mutex>
 
 #include "../../include/h2o.h"
 #include "attn.h"
@@ -33,31 +39,44 @@ constexpr long long kStaticScratchRows = 4ll << 20;
 
 static __device__ __align__(256) float g_row_lse2[kStaticScratchRows];
 // Where the kernels latch an expired bounded wait (they never leave one
-// pending); this entry point has no cache state word to put it in.
+// pending); this entry point has no cache state word to put it in.  Each
+// call clears it first; h2o_static_scratch_check reads it.
 static __device__ int g_wait_error;
 
 constexpr int kMaxDevices = 64;
-float* g_scratch_addr[kMaxDevices];  // device address of g_row_lse2, per device
-int* g_error_addr[kMaxDevices];      // device address of g_wait_error, per device
-bool g_scratch_ready[kMaxDevices];
+// device addresses of g_row_lse2 and g_wait_error, per device; published
+// (release) only once both are known, so a reader that sees them non-null
+// (acquire) may use them
+std::atomic<float*> g_scratch_addr[kMaxDevices];
+std::atomic<int*> g_error_addr[kMaxDevices];
+std::mutex g_setup_mutex;
 
-// Resolves the array's device address on the current device, once per
+// Resolves the arrays' device addresses on the current device, once per
 // device.  Host code must not pass `g_row_lse2` itself to a kernel: on the
 // host that name is only a stand-in for the symbol, not a device address.
 h2o_status scratch_address(float** out, int** err) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return H2O_ERR_CUDA;
-  if (!g_scratch_ready[dev]) {
-    void* p = nullptr;
-    void* e = nullptr;
-    if (cudaGetSymbolAddress(&p, g_row_lse2) != cudaSuccess || p == nullptr) return H2O_ERR_CUDA;
-    if (cudaGetSymbolAddress(&e, g_wait_error) != cudaSuccess || e == nullptr) return H2O_ERR_CUDA;
-    g_scratch_addr[dev] = static_cast<float*>(p);
-    g_error_addr[dev] = static_cast<int*>(e);
-    g_scratch_ready[dev] = true;
+  float* a = g_scratch_addr[dev].load(std::memory_order_acquire);
+  int* w = g_error_addr[dev].load(std::memory_order_acquire);
+  if (a == nullptr || w == nullptr) {
+    // first use on this device: one thread looks the addresses up
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    a = g_scratch_addr[dev].load(std::memory_order_relaxed);
+    w = g_error_addr[dev].load(std::memory_order_relaxed);
+    if (a == nullptr || w == nullptr) {
+      void* p = nullptr;
+      void* e = nullptr;
+      if (cudaGetSymbolAddress(&p, g_row_lse2) != cudaSuccess || p == nullptr) return H2O_ERR_CUDA;
+      if (cudaGetSymbolAddress(&e, g_wait_error) != cudaSuccess || e == nullptr) return H2O_ERR_CUDA;
+      a = static_cast<float*>(p);
+      w = static_cast<int*>(e);
+      g_error_addr[dev].store(w, std::memory_order_release);
+      g_scratch_addr[dev].store(a, std::memory_order_release);
+    }
   }
-  *out = g_scratch_addr[dev];
-  *err = g_error_addr[dev];
+  *out = a;
+  *err = w;
   return H2O_OK;
 }
 
@@ -123,6 +142,9 @@ extern "C" H2O_API h2o_status h2o_attention_static_scratch(
   int* err = nullptr;
   h2o_status s = scratch_address(&lse2, &err);
   if (s != H2O_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // this call's kernels latch a timeout into a clean word
+  if (cudaMemsetAsync(err, 0, sizeof(int), st) != cudaSuccess) return H2O_ERR_CUDA;
 
   AttnParams p;
   p.B = g.batch;
@@ -140,7 +162,6 @@ extern "C" H2O_API h2o_status h2o_attention_static_scratch(
   p.colsum = colsum_out;  // written in place: [batch, H_kv, capacity + n_q]
   p.colsum_ld = g.capacity + n_q;
   p.err = err;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   if (g.dtype == H2O_F32) {
     cudaError_t e = launch_attn_f32(g.head_dim, static_cast<const float*>(q),
@@ -169,5 +190,29 @@ extern "C" H2O_API h2o_status h2o_attention_static_scratch(
     return H2O_ERR_CUDA;
   if (launch_attn_fwd_bf16(d, m, p, st) != cudaSuccess) return H2O_ERR_CUDA;
   if (launch_attn_colsum_bf16(d, m, p, st) != cudaSuccess) return H2O_ERR_CUDA;
+  return H2O_OK;
+}
+
+namespace h2o {
+// The static entry point's error word on the current device (null when its
+// address cannot be resolved); the failure-path self-test latches into it.
+int* static_scratch_error_word() {
+  float* a = nullptr;
+  int* w = nullptr;
+  return scratch_address(&a, &w) == H2O_OK ? w : nullptr;
+}
+}  // namespace h2o
+
+extern "C" H2O_API h2o_status h2o_static_scratch_check(void* stream) {
+  float* a = nullptr;
+  int* w = nullptr;
+  h2o_status s = scratch_address(&a, &w);
+  if (s != H2O_OK) return s;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return H2O_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, w, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return H2O_ERR_CUDA;
+  if (word & h2o::kDevErrTimeout) return H2O_ERR_TIMEOUT;
+  if (word & ~h2o::kDevErrTimeout) return H2O_ERR_STATE;
   return H2O_OK;
 }

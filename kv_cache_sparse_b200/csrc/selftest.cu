@@ -1,8 +1,10 @@
 // selftest.cu -- diagnostic entry point h2o_selftest_wait_timeout: one warp
 // waits, with the kernels' bounded wait, on an mbarrier nothing arrives at;
 // the wait gives up after the given limit, latches the timeout bit and the
-// kernel returns (no trap, no hang).
+// kernel returns (no trap, no hang).  Without a word of the caller's, the bit
+// goes to the word h2o_static_scratch_check reports.
 #include "../../include/h2o.h"
+#include "attn.h"
 #include "sm100.cuh"
 
 namespace {
@@ -25,7 +27,10 @@ __global__ void wait_timeout_probe(int* err, uint64_t limit_ns) {
 
 extern "C" H2O_API h2o_status h2o_selftest_wait_timeout(int32_t* err_word, uint32_t limit_us,
                                                         void* stream) {
-  if (!err_word || limit_us == 0 || limit_us > 2000000) return H2O_ERR_INVALID_ARG;
+  if (limit_us == 0 || limit_us > 2000000) return H2O_ERR_INVALID_ARG;
+  // no word given: the static-scratch entry point's word on this device
+  if (!err_word) err_word = h2o::static_scratch_error_word();
+  if (!err_word) return H2O_ERR_CUDA;
   wait_timeout_probe<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       err_word, static_cast<uint64_t>(limit_us) * 1000ull);
   return cudaGetLastError() == cudaSuccess ? H2O_OK : H2O_ERR_CUDA;

@@ -78,3 +78,61 @@ def test_evict_many_steps_bit_exact():
         ref.evict(cs, gh.np64(kn), gh.np64(vn))
         gh.assert_state_equal(gpu.read(), ref, torch.bfloat16, f"step {step}")
     assert gpu.check() == 0
+
+
+SIGNED_CASES = [
+    # B, Hkv, d, C, n, nq, W      launch shape
+    (1, 2, 128, 256, 256, 64, 8),     # cluster of CTAs per unit
+    (4, 8, 64, 256, 256, 64, 0),      # one 1024-thread CTA per unit
+    (40, 8, 64, 96, 96, 32, 4),       # many units: 256-thread CTAs
+]
+
+
+@pytest.mark.parametrize("case", SIGNED_CASES, ids=lambda c: "B{}_Hkv{}_C{}_nq{}".format(
+    c[0], c[1], c[3], c[5]))
+def test_evict_negative_scores_bit_exact(case):
+    """Scores restored by h2o_cache_write and summed weights given to
+    h2o_evict may be negative (and -0): the selection orders them by value
+    like the oracle, which sorts the fp32 values themselves."""
+    B, Hkv, d, C, n, nq, W = case
+    rng = np.random.default_rng(C * 7 + B)
+    shape = gh.shape_of(B, Hkv, Hkv, d, C, nq, W)
+    gpu = binding.H2OCache(shape)
+    ref = gh.oracle_for(shape)
+    t0 = n + 5
+    K, V, sc, pos = gh.random_state(shape, n, t0, rng)
+    sc = (sc - 2.0).astype(np.float32)           # about half of the scores below zero
+    sc[:, :, : n // 8] = np.float32(-0.0)
+    sc[:, :, n:] = 0
+    gh.install_state(gpu, ref, K, V, sc, pos, n, t0)
+    cs = (rng.random((B, Hkv, C + nq)) * 2 - 1).astype(np.float32)
+    cs[:, :, n:C] = 0
+    cs[:, :, C:C + nq // 4] = np.float32(-0.0)
+    kn = torch.randn(B, nq, Hkv, d).to(torch.bfloat16)
+    vn = torch.randn(B, nq, Hkv, d).to(torch.bfloat16)
+    gpu.evict(torch.from_numpy(cs).cuda(), kn.cuda(), vn.cuda())
+    assert gpu.check() == 0
+    ref.evict(cs, gh.np64(kn), gh.np64(vn))
+    gh.assert_state_equal(gpu.read(), ref, torch.bfloat16, str(case))
+
+
+def test_decode_eviction_with_negative_scores():
+    """The decode step's single-token eviction ranks negative scores by
+    value too (the lowest score leaves, the highest index on ties)."""
+    B, Hq, Hkv, d, C, n, W = 2, 8, 2, 128, 600, 600, 0
+    rng = np.random.default_rng(77)
+    shape = gh.shape_of(B, Hq, Hkv, d, C, 4, W)
+    gpu = binding.H2OCache(shape)
+    ref = gh.oracle_for(shape)
+    t0 = n + 9
+    K, V, sc, pos = gh.random_state(shape, n, t0, rng)
+    sc = (sc - 5.0).astype(np.float32)
+    gh.install_state(gpu, ref, K, V, sc, pos, n, t0)
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn(B, 1, Hq, d, generator=g).to(torch.bfloat16)
+    kn = torch.randn(B, 1, Hkv, d, generator=g).to(torch.bfloat16)
+    vn = torch.randn(B, 1, Hkv, d, generator=g).to(torch.bfloat16)
+    O, cs = gpu.step(q.cuda(), kn.cuda(), vn.cuda(), return_colsum=True)
+    assert gpu.check() == 0
+    ref.evict(gh.np64(cs).astype(np.float32), gh.np64(kn), gh.np64(vn))
+    gh.assert_state_equal(gpu.read(), ref, torch.bfloat16, "decode, negative scores")
