@@ -2,12 +2,16 @@
 
 A step is one pass of the whole hot path -- attention forward, summed
 weights, score update + top-C selection, K/V scatter -- over one chunk of
-synthetic input, on a full cache (steady state).  The workload is the
-Qwen3-4B-shaped single cache (H_q 32, H_kv 8, d 128, bf16, C 8192,
-n_q 1024, W 256).  Inputs are drawn on the device before the timed region;
-L2 is flushed (256 MiB write) before every timed step, outside its events.
+synthetic input, on full caches (steady state).  The default workload is the
+largest one that fits a GPU: the 36-layer x 4-sequence stack of
+Qwen3-4B-shaped caches (144 caches; H_q 32, H_kv 8, d 128, bf16, C 8192,
+n_q 1024, W 0).  ``--workload`` selects another (every workload, the fp32
+tiny case included).  Inputs are drawn on the device before the timed
+region; L2 is flushed (256 MiB write) before every timed step, outside its
+events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
 
 Prints one JSON line on rank 0.  With N > 1 (launched by torchrun) every
 rank runs its own independent cache (weak scaling, no collective on the
@@ -16,6 +20,7 @@ data path); the step time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -32,13 +37,20 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from kv_cache_sparse_b200.workloads import QWEN_C8K, WORKLOADS, device_chunk  # noqa: E402
+from kv_cache_sparse_b200.workloads import STACK36, WORKLOADS, DeviceChunkSource  # noqa: E402
 
-WL = QWEN_C8K  # the default workload (the headline line)
+WL = STACK36  # the default workload (the headline line)
 METRIC = "chunk-tokens/s per H2O attention+evict step (1 B200); % bf16 TC peak; evict GB/s"
 UNIT = "chunk-tokens/s"
 KERNELS = ["attn_fwd_kernel", "attn_colsum_kernel", "h2o_select", "reserved"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# fp32 FMA peak from the unit counts: 148 SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz
+F32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# spec targets: attention + summed weights against the bf16 dense peak,
+# the eviction (score update, selection, scatter) against HBM bandwidth
+TARGET_ATTENTION_TC = 0.50
+TARGET_EVICT_HBM = 0.60
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 # ---------------------------------------------------------------- helpers
@@ -53,13 +65,24 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes per launch from the last ncu capture of `kernel`
-    (profiles/traffic.json), or None when its source changed since."""
-    from kv_cache_sparse_b200.ncu_summary import TRAFFIC_FILE, source_digest
+def source_digest(path: str) -> str:
+    """Digest of a kernel source together with the device headers it includes
+    (the key under which profiles/traffic.json records a kernel's counters)."""
+    h = hashlib.sha256()
+    csrc = os.path.dirname(os.path.abspath(path))
+    for p in (path, os.path.join(csrc, "sm100.cuh"), os.path.join(csrc, "common.h")):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the last ncu
+    capture (profiles/traffic.json, keyed "kernel@workload"), or None when
+    the kernel's source changed since."""
     try:
         with open(TRAFFIC_FILE) as f:
-            rec = json.load(f)[kernel]
+            rec = json.load(f)[f"{kernel}@{workload}"]
         src = os.path.join(ROOT, "kv_cache_sparse_b200", "csrc", rec["source"])
         if source_digest(src) != rec["source_sha256_16"]:
             return None
@@ -159,6 +182,19 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
                 "sm_max_mhz": max(r["max"] for r in rows), "reasons": sorted(reasons),
                 "samples": len(rows)}
+
+
+def data_note(wl) -> str:
+    """What the synthetic inputs are (drawn on the device)."""
+    if wl.heavy_p_range is not None:
+        heavy = (f"heavy-hitter density drawn per chunk and cache from "
+                 f"U[{wl.heavy_p_range[0]:.3f}, {wl.heavy_p_range[1]:.3f}]")
+    else:
+        heavy = f"{100 * wl.heavy_p:g}% heavy-hitter keys"
+    drift = (f"; K mean a per-token random walk, step norm {wl.drift_step}"
+             if wl.drift_step > 0 else "")
+    return (f"synthetic (seeded N(0,1) Q/K/V, {heavy} shifted by 3.0 along one fixed unit "
+            f"vector per cache{drift}; drawn on device)")
 
 
 def cpu_cores():
@@ -291,11 +327,18 @@ def run_ours(args, world, rank, local):
     # fill phase (untimed): C / n_q steps (prefill chunks for the decode
     # workloads) bring the cache to steady state
     fill = wl.capacity // wl.fill_chunk
+    src = DeviceChunkSource(wl, seed, dev)
     for c in range(fill):
-        cache.step(*device_chunk(wl, seed, c, dev, n_q=wl.fill_chunk))
+        cache.step(*src.chunk(c, n_q=wl.fill_chunk))
     K, W = args.steps, args.warmup
     KB = min(K, 8)  # extra steps with per-kernel events, for the breakdown
-    chunks = [device_chunk(wl, seed, fill + c, dev) for c in range(W + K + KB)]
+    # the chunks are drawn before the timed region; big workloads (the
+    # 144-cache stack: 1.8 GB per chunk) cycle through a pool of at most 8 GB
+    per_chunk = wl.batch * wl.chunk * (wl.n_q_heads + 2 * wl.n_kv_heads) * wl.head_dim * (
+        2 if wl.dtype == "bf16" else 4)
+    n_pool = max(2, min(W + K + KB, int(8e9 // per_chunk)))
+    pool = [src.chunk(fill + c) for c in range(n_pool)]
+    chunks = [pool[c % n_pool] for c in range(W + K + KB)]
     out = torch.empty(wl.batch, wl.chunk, wl.n_q_heads, wl.head_dim, dtype=wl.torch_dtype(),
                       device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -396,13 +439,16 @@ def run_ours(args, world, rank, local):
     # ---- roofline of the dominant kernel
     peaks, peaks_kind = load_peaks()
     avg = kern.mean(axis=0)
+    f32 = wl.dtype == "f32"
+    names = (["attn_f32 (attention + summed weights, FMA)", "-", "h2o_select", "reserved"]
+             if f32 else KERNELS)
     n = wl.capacity
     flops = attention_flops(wl, n, wl.chunk)
     ebytes = evict_bytes(wl, n, wl.chunk, float(np.mean(kept)))
     tc_peak = peaks["bf16_tflops"]
     hbm_peak = peaks["hbm_gbs"]
     kernels = {}
-    for i, name in enumerate(KERNELS):
+    for i, name in enumerate(names):
         if avg[i] <= 0 or (i == 1 and wl.policy != "h2o"):  # no summed weights launched
             continue
         kernels[name] = {"ms": round(float(avg[i]), 5),
@@ -420,9 +466,19 @@ def run_ours(args, world, rank, local):
                 "peak_kind": f"{peaks_kind} HBM copy",
                 "per_launch": f"{db:.4e} B (K and V rows of the valid slots, scores, positions, "
                               f"q, out, the new K/V rows)"}
+    elif f32:
+        # fp32 caches: attention and summed weights in FMA kernels (no tensor
+        # cores); the kernel pair against the FP32 FMA peak of the unit counts
+        fl = 1.5 * flops   # QK^T, PV and the QK^T recompute of the summed weights
+        achieved = fl / (avg[0] * 1e-3) / 1e12
+        roof = {"kernel": names[0], "bound": "alu", "achieved": round(achieved, 3),
+                "peak": round(F32_FMA_TFLOPS, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / F32_FMA_TFLOPS, 5), "traffic": None,
+                "peak_kind": "nominal FP32 FMA (148 SMs x 128 lanes x 2 x 1965 MHz)",
+                "per_launch": f"{fl:.4e} FLOP (QK^T, PV, QK^T recompute)"}
     elif dom == 0:
         achieved = flops / (avg[0] * 1e-3) / 1e12
-        tr = recorded_traffic("attn_fwd_kernel") if wl is WL else None
+        tr = recorded_traffic("attn_fwd_kernel", wl.name)
         roof = {"kernel": KERNELS[0], "bound": "tensor", "achieved": round(achieved, 2),
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
                 "traffic": tr, "peak_kind": f"{peaks_kind} bf16 dense (burst)",
@@ -431,13 +487,37 @@ def run_ours(args, world, rank, local):
         # the summed-weights kernel: its FLOPs are the QK^T recompute
         rf = flops / 2
         achieved = rf / (avg[dom] * 1e-3) / 1e12
-        tr = recorded_traffic(KERNELS[dom]) if wl is WL else None
+        tr = recorded_traffic(KERNELS[dom], wl.name)
         roof = {"kernel": KERNELS[dom], "bound": "tensor", "achieved": round(achieved, 2),
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
                 "traffic": tr, "peak_kind": f"{peaks_kind} bf16 dense (burst)",
                 "per_launch": f"{rf:.4e} FLOP (QK^T recompute)"}
     attn_ms = avg[0] + avg[1]
     evict_ms = max(avg[2] + avg[3], 1e-9)
+    attn_frac = flops / (attn_ms * 1e-3) / 1e12 / tc_peak
+    evict_frac = ebytes / (evict_ms * 1e-3) / 1e9 / hbm_peak
+    if not decode and not f32:
+        # the two quantities the targets are set on, each against its roofline
+        single = wl.batch * wl.n_kv_heads <= 16
+        roof["targets"] = {
+            "attention_k1_k2": {
+                "kernels": "attn_fwd_kernel + attn_colsum_kernel",
+                "frac": round(attn_frac, 4), "target": TARGET_ATTENTION_TC,
+                "pass": bool(attn_frac >= TARGET_ATTENTION_TC),
+                "of": f"{peaks_kind} bf16 dense (burst) {tc_peak} TFLOP/s",
+                "per_step": f"{flops:.4e} algorithmic FLOP (QK^T + PV; the summed weights' "
+                            f"QK^T recompute not counted)"}
+            if wl.policy == "h2o" else None,
+            "evict_k3": {
+                "kernels": "h2o_select (score update, selection, K/V scatter)",
+                "frac": round(evict_frac, 4), "target": TARGET_EVICT_HBM,
+                "pass": bool(evict_frac >= TARGET_EVICT_HBM),
+                "of": f"{peaks_kind} HBM copy {hbm_peak} GB/s",
+                "per_step": f"{int(ebytes)} algorithmic bytes",
+                "note": ("a single cache moves a few MB per step, less than one launch's "
+                         "latency at full bandwidth: the target is not reachable there"
+                         if single else "many caches: bandwidth-sized work")},
+        }
     extra = {
         "attention_tc_frac": round(flops / (attn_ms * 1e-3) / 1e12 / tc_peak, 4),
         "attention_tflops": round(flops / (attn_ms * 1e-3) / 1e12, 2),
@@ -448,7 +528,10 @@ def run_ours(args, world, rank, local):
         "kernels": kernels,
         "step_ms_p50": round(float(np.median(step_ms)), 5),
         "breakdown": f"per-kernel times from {KB} extra steps with the library's events "
-                     f"between kernels (the timed steps run without them)",
+                     f"between kernels (the timed steps run without them); the events "
+                     f"serialise the kernels, so the programmatic-dependent-launch overlap "
+                     f"of the timed steps is absent and the per-kernel fractions are "
+                     f"slightly pessimistic",
     }
     if decode:  # one token per cache: no tensor-core work, the eviction is fused
         extra = {"kernels": kernels, "kept_new_tokens_per_step": float(np.mean(kept)),
@@ -459,8 +542,8 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": round(total_ms / K, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) Q/K/V with 2% heavy-hitter keys, drawn on device)",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": data_note(wl),
         "config": {"workload": wl.name, "caches_per_gpu": wl.batch, "n_q_heads": wl.n_q_heads,
                    "n_kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "chunk": wl.chunk,
                    "capacity": wl.capacity, "recent_window": wl.window, "policy": wl.policy,
@@ -534,8 +617,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default=WL.name,
-                    choices=[w for w in WORKLOADS if WORKLOADS[w].dtype == "bf16"])
+    ap.add_argument("--workload", default=WL.name, choices=list(WORKLOADS))
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")

@@ -197,26 +197,65 @@ class ChunkSource:
         return Q.to(dt), K.to(dt), V.to(dt)
 
 
-def device_chunk(wl: Workload, seed: int, c: int, device, n_q: Optional[int] = None):
-    """Same distribution as ``ChunkSource.chunk`` drawn on ``device``.
+class DeviceChunkSource:
+    """The distribution of ``ChunkSource`` drawn on ``device`` (for
+    throughput runs, where the values only need the right distribution; it
+    does not reproduce the CPU draws).
 
-    Used for throughput runs, where the values only need the right
-    distribution; it does not reproduce the CPU draws.  The drift of the
-    streaming workload is approximated by a per-chunk offset.
+    * Each cache keeps one heavy-hitter direction for the whole run: the same
+      unit vector ``ChunkSource`` uses (``heavy_direction``).
+    * The heavy density is ``heavy_p``, or drawn per chunk and cache from
+      U[lo, hi] when the workload gives a range.
+    * A drifting workload's K mean is a per-token random walk per (cache, KV
+      head) with steps of norm ``drift_step`` in uniformly random directions,
+      carried from one chunk to the next on the device.  Chunks are meant to
+      be drawn in order; a call that skips ahead starts the walk from a
+      Gaussian draw with the walk's covariance at that token
+      (drift_step^2 * tokens / d per coordinate).
+
+    The last chunk's heavy mask, densities and walk are kept in
+    ``last_heavy`` ([B, n_q] bool), ``last_p`` ([B]) and ``last_walk``
+    ([B, n_q, H_kv, d], or None) for inspection.
     """
-    n_q = wl.chunk if n_q is None else n_q
-    g = _gen(seed, 0xC0DA, c, device=str(device))
-    B, d = wl.batch, wl.head_dim
-    Q = torch.randn(B, n_q, wl.n_q_heads, d, generator=g, device=device)
-    K = torch.randn(B, n_q, wl.n_kv_heads, d, generator=g, device=device)
-    V = torch.randn(B, n_q, wl.n_kv_heads, d, generator=g, device=device)
-    u = torch.randn(B, 1, 1, d, generator=g, device=device)
-    u = u / u.norm(dim=-1, keepdim=True)
-    p = wl.heavy_p if wl.heavy_p_range is None else sum(wl.heavy_p_range) / 2
-    heavy = (torch.rand(B, n_q, 1, 1, generator=g, device=device) < p).float()
-    K += HEAVY_SHIFT * heavy * u
-    if wl.drift_step > 0:
-        K += wl.drift_step * (c * n_q) ** 0.5 * torch.randn(
-            B, 1, wl.n_kv_heads, d, generator=g, device=device) / d ** 0.5
-    dt = wl.torch_dtype()
-    return Q.to(dt), K.to(dt), V.to(dt)
+
+    def __init__(self, wl: Workload, seed: int, device, batch: Optional[int] = None):
+        self.wl = wl
+        self.seed = seed
+        self.device = torch.device(device)
+        self.batch = wl.batch if batch is None else batch
+        self.u = torch.stack([heavy_direction(wl, seed, b) for b in range(self.batch)]).to(
+            self.device)
+        self.mu = torch.zeros(self.batch, wl.n_kv_heads, wl.head_dim, device=self.device)
+        self.next_c = 0
+        self.last_heavy = self.last_p = self.last_walk = None
+
+    def chunk(self, c: int, n_q: Optional[int] = None):
+        wl = self.wl
+        n_q = wl.chunk if n_q is None else n_q
+        dev = self.device
+        g = _gen(self.seed, 0xC0DA, c, device=str(dev))
+        B, d, Hkv = self.batch, wl.head_dim, wl.n_kv_heads
+        Q = torch.randn(B, n_q, wl.n_q_heads, d, generator=g, device=dev)
+        K = torch.randn(B, n_q, Hkv, d, generator=g, device=dev)
+        V = torch.randn(B, n_q, Hkv, d, generator=g, device=dev)
+        if wl.heavy_p_range is not None:
+            lo, hi = wl.heavy_p_range
+            p = lo + (hi - lo) * torch.rand(B, generator=g, device=dev)
+        else:
+            p = torch.full((B,), wl.heavy_p, device=dev)
+        heavy = torch.rand(B, n_q, generator=g, device=dev) < p[:, None]
+        K += HEAVY_SHIFT * heavy[:, :, None, None].float() * self.u[:, None, None, :]
+        self.last_heavy, self.last_p, self.last_walk = heavy, p, None
+        if wl.drift_step > 0:
+            if c != self.next_c:   # skipped ahead: the walk's distribution at token c * n_q
+                std = wl.drift_step * (c * n_q / d) ** 0.5
+                self.mu = std * torch.randn(B, Hkv, d, generator=g, device=dev)
+            xi = torch.randn(B, n_q, Hkv, d, generator=g, device=dev)
+            inc = wl.drift_step * xi / xi.norm(dim=-1, keepdim=True)
+            walk = self.mu[:, None] + torch.cumsum(inc, dim=1)
+            K += walk
+            self.mu = walk[:, -1].clone()
+            self.last_walk = walk
+        self.next_c = c + 1
+        dt = wl.torch_dtype()
+        return Q.to(dt), K.to(dt), V.to(dt)

@@ -7,7 +7,7 @@ import torch
 
 import gpu_helpers as gh
 from kv_cache_sparse_b200 import binding
-from kv_cache_sparse_b200.workloads import QWEN_C8K, TINY, ChunkSource, device_chunk
+from kv_cache_sparse_b200.workloads import QWEN_C8K, TINY, ChunkSource, DeviceChunkSource
 from oracle import h2o_oracle as orc
 
 pytestmark = pytest.mark.gpu
@@ -177,12 +177,13 @@ def test_full_size_qwen_sampled():
     shape = shape_for(wl)
     gpu = binding.H2OCache(shape)
     dev = torch.device("cuda")
+    src = DeviceChunkSource(wl, 0, dev)
     for c in range(wl.capacity // wl.chunk + 1):
-        gpu.step(*device_chunk(wl, 0, c, dev))
+        gpu.step(*src.chunk(c))
     assert gpu.check() == 0
     st = gpu.read()
     assert st["n"] == wl.capacity
-    q, kn, vn = device_chunk(wl, 0, 99, dev)
+    q, kn, vn = src.chunk(wl.capacity // wl.chunk + 1)
     O, cs = gpu.attention(q, kn, vn)
     G = wl.group
     tot = gh.np64(cs).sum(-1)

@@ -9,7 +9,7 @@ import torch
 
 import gpu_helpers as gh
 from kv_cache_sparse_b200 import binding
-from kv_cache_sparse_b200.workloads import QWEN_C16K, STACK36, STREAM1M, device_chunk
+from kv_cache_sparse_b200.workloads import QWEN_C16K, STACK36, STREAM1M, DeviceChunkSource
 from oracle import h2o_oracle as orc
 
 pytestmark = pytest.mark.gpu
@@ -25,12 +25,13 @@ def steady_state_check(wl, fill_steps, samples, evict_caches):
     shape = gh.shape_of(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.capacity,
                         wl.chunk, wl.window, wl.torch_dtype())
     gpu = binding.H2OCache(shape)
+    src = DeviceChunkSource(wl, 0, dev)
     for c in range(fill_steps):
-        gpu.step(*device_chunk(wl, 0, c, dev))
+        gpu.step(*src.chunk(c))
     assert gpu.check() == 0
     st = gpu.read()
     assert st["n"] == wl.capacity
-    q, kn, vn = device_chunk(wl, 0, 10_000, dev)
+    q, kn, vn = src.chunk(fill_steps)
     O, cs = gpu.attention(q, kn, vn)
     G = wl.group
     assert np.allclose(gh.np64(cs).sum(-1), wl.chunk * G, rtol=1e-4)
