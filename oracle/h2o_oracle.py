@@ -40,8 +40,20 @@ The readings taken here, where the sources are silent:
   H2O with the candidate's position in place of its score (positions are
   distinct, so there are no ties), the recent window still protecting, and
   no score kept: old slots keep theirs, placed tokens get 0.
+* The quantised cache of Q-Hitter (page 1 §2 Related Work: Q-Hitter combines
+  H2O with quantisation; summary page Table 5, ``qh2o`` rows), whose format
+  the sources do not give.  Reading: each cache row (one slot of one KV head,
+  K and V separately) is stored as int8 codes with one fp32 scale,
+  symmetric: s = fl32(max|x| / 127), q = clamp(rint(fl32(x / s)), -127, 127)
+  (half to even; q = 0 when the row is all zero); the attention reads the
+  dequantised value bf16(fl32(q * s)) (round to nearest even).  A token is
+  quantised when it is placed into the cache; the chunk's own keys and
+  values enter the step that brings them at their input precision.  The
+  H2O scores are the same summed attention weights as without quantisation.
 
-Parity status: attention output, summed weights and the selection are pinned
+Parity status: the quantiser is pinned by hand-worked rows, its defining
+properties (the largest element maps to +-127, the round-trip bound) and a
+library bf16 rounding.  The attention output, summed weights and the selection are pinned
 by brute force, a library routine (torch SDPA in fp64), closed forms and
 invariants in ``tests/test_oracle_*.py``.  The multi-step trajectory is pinned
 by an independent token-centric re-implementation.  The backward is pinned by
@@ -58,6 +70,41 @@ from typing import List, Optional, Tuple
 import numpy as np
 
 F32 = np.float32
+
+
+# --------------------------------------------------------------------------
+# the quantised cache format (Q-Hitter reading, see the module docstring)
+# --------------------------------------------------------------------------
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """float32 values rounded to the nearest bfloat16 (ties to even), as
+    float32: the upper 16 bits of the float32 pattern after adding half an
+    ulp of the kept part (0x7FFF plus the lowest kept bit)."""
+    b = np.ascontiguousarray(x, dtype=F32).view(np.uint32).astype(np.uint64)
+    r = (b + 0x7FFF + ((b >> 16) & 1)) >> 16 << 16
+    return (r & 0xFFFFFFFF).astype(np.uint32).view(F32)
+
+
+def quantize_row_q8(x: np.ndarray) -> Tuple[np.ndarray, np.float32]:
+    """One cache row (d values) -> (int8 codes, fp32 scale)."""
+    x = np.asarray(x, dtype=F32)
+    amax = F32(np.max(np.abs(x))) if x.size else F32(0)
+    s = F32(amax / F32(127))
+    if s == 0:
+        return np.zeros(x.shape, dtype=np.int8), F32(0)
+    q = np.rint(np.asarray(x / s, dtype=F32)).clip(-127, 127)
+    return q.astype(np.int8), s
+
+
+def dequantize_q8(q: np.ndarray, s) -> np.ndarray:
+    """int8 codes and their scale(s) -> the value the attention reads,
+    bf16(fl32(q * s)), as float64.  One scale per row: s has the shape of q
+    without its last axis."""
+    q = np.asarray(q, dtype=F32)
+    s = np.asarray(s, dtype=F32)
+    if s.ndim:
+        s = s[..., None]
+    return bf16_round((q * s).astype(F32)).astype(np.float64)
 
 
 # --------------------------------------------------------------------------
@@ -242,12 +289,17 @@ class OracleCache:
     K, V: [B, H_kv, C, d] float64 holding the input values exactly;
     scores [B, H_kv, C] float32; pos [B, H_kv, C] int32 (-1 empty);
     n (valid slots, shared) and t0 (position of the next chunk's first token).
+    With kv_format "q8" the cache rows are stored quantised: Kq, Vq
+    [B, H_kv, C, d] int8 and Ks, Vs [B, H_kv, C] float32, and K, V hold their
+    dequantised values (what the attention reads).
     """
 
     def __init__(self, batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
                  capacity: int, window: int, scale: Optional[float] = None,
-                 policy: str = "h2o", sinks: int = 0):
+                 policy: str = "h2o", sinks: int = 0, kv_format: str = "bf16"):
         assert n_q_heads % n_kv_heads == 0
+        assert kv_format in ("bf16", "q8")
+        self.kv_format = kv_format
         assert 0 <= window <= capacity
         assert policy in POLICIES and 0 <= sinks and (policy != "slr" or sinks + window <= capacity)
         self.policy, self.sinks = policy, sinks
@@ -260,6 +312,11 @@ class OracleCache:
         self.pos = np.full((batch, n_kv_heads, capacity), -1, dtype=np.int32)
         self.n = 0
         self.t0 = 0
+        if kv_format == "q8":
+            self.Kq = np.zeros((batch, n_kv_heads, capacity, head_dim), dtype=np.int8)
+            self.Vq = np.zeros_like(self.Kq)
+            self.Ks = np.zeros((batch, n_kv_heads, capacity), dtype=F32)
+            self.Vs = np.zeros_like(self.Ks)
 
     # snapshot / restore --------------------------------------------------
     def state(self):
@@ -272,6 +329,14 @@ class OracleCache:
         self.scores = np.array(scores, dtype=F32)
         self.pos = np.array(pos, dtype=np.int32)
         self.n, self.t0 = int(n), int(t0)
+
+    def load_q8(self, Kq, Ks, Vq, Vs, scores, pos, n, t0):
+        """Restores a quantised cache from its codes and scales."""
+        assert self.kv_format == "q8"
+        self.Kq, self.Vq = np.array(Kq, dtype=np.int8), np.array(Vq, dtype=np.int8)
+        self.Ks, self.Vs = np.array(Ks, dtype=F32), np.array(Vs, dtype=F32)
+        self.load(dequantize_q8(self.Kq, self.Ks), dequantize_q8(self.Vq, self.Vs), scores, pos,
+                  n, t0)
 
     # the two halves of the step -------------------------------------------
     def attention(self, Q, Kn, Vn):
@@ -320,7 +385,13 @@ class OracleCache:
                                             self.t0, colsum32[b, g], n_q, self.W,
                                             self.policy, self.sinks)
                 self.scores[b, g], self.pos[b, g] = sc, ps
-                if pl.slots:
+                if pl.slots and self.kv_format == "q8":
+                    for s_, i_ in zip(pl.slots, pl.tokens):   # quantised on placement
+                        self.Kq[b, g, s_], self.Ks[b, g, s_] = quantize_row_q8(Kn[b, i_, g])
+                        self.Vq[b, g, s_], self.Vs[b, g, s_] = quantize_row_q8(Vn[b, i_, g])
+                        self.K[b, g, s_] = dequantize_q8(self.Kq[b, g, s_], self.Ks[b, g, s_])
+                        self.V[b, g, s_] = dequantize_q8(self.Vq[b, g, s_], self.Vs[b, g, s_])
+                elif pl.slots:
                     self.K[b, g, pl.slots] = Kn[b, pl.tokens, g]
                     self.V[b, g, pl.slots] = Vn[b, pl.tokens, g]
                 row.append(pl)
