@@ -103,9 +103,10 @@ def decode_bytes(wl, n):
     and V rows read once, its score read and written and its position read;
     the queries read and the outputs written; the new K/V rows read and
     written once."""
-    e = 2 if wl.dtype == "bf16" else 4
+    e = 4 if wl.dtype == "f32" else 2          # q, out, new rows
+    ec, es = (1, 4) if wl.dtype == "q8" else (e, 0)  # cache element, row scale bytes
     d = wl.head_dim
-    per_unit = n * (2 * d * e + 12) + 2 * 2 * d * e
+    per_unit = n * (2 * (d * ec + es) + 12) + 2 * (d * e + d * ec + es)
     return wl.batch * (wl.n_kv_heads * per_unit + 2 * wl.n_q_heads * d * e)
 
 
@@ -114,9 +115,10 @@ def evict_bytes(wl, n, nq, kept_total):
     scores and summed weights, write the scores; per kept new token write its
     position and score and read + write its K and V rows."""
     units = wl.batch * wl.n_kv_heads
-    e = 2 if wl.dtype == "bf16" else 4
+    e = 4 if wl.dtype == "f32" else 2          # the new rows
+    ec, es = (1, 4) if wl.dtype == "q8" else (e, 0)  # cache element, row scale bytes
     per_unit = 4 * n + 4 * (n + nq) + 4 * n
-    return units * per_unit + kept_total * (8 + 4 * wl.head_dim * e)
+    return units * per_unit + kept_total * (8 + 2 * (wl.head_dim * e + wl.head_dim * ec + es))
 
 
 class ClockSampler:
@@ -227,7 +229,8 @@ def oracle_sample(wl, steps: int, seed: int = 0, groups=None):
     wl = wl.scaled(n_kv_heads=groups, n_q_heads=groups * wl.group, batch=1)
     rng = np.random.default_rng(seed)
     ref = orc.OracleCache(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.capacity,
-                          wl.window, policy=wl.policy, sinks=wl.sinks)
+                          wl.window, policy=wl.policy, sinks=wl.sinks,
+                          kv_format="q8" if wl.dtype == "q8" else "bf16")
     C = wl.capacity
     g = torch.Generator().manual_seed(seed)
     K = torch.randn(wl.batch, wl.n_kv_heads, C, wl.head_dim, generator=g).to(torch.bfloat16)
@@ -318,7 +321,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     wl = WORKLOADS[args.workload]
     shape = binding.CacheShape(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
-                               wl.capacity, wl.max_chunk, wl.window, wl.torch_dtype(), 0.0,
+                               wl.capacity, wl.max_chunk, wl.window, wl.cache_dtype(), 0.0,
                                wl.policy, wl.sinks)
     cache = binding.H2OCache(shape, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -335,7 +338,7 @@ def run_ours(args, world, rank, local):
     # the chunks are drawn before the timed region; big workloads (the
     # 144-cache stack: 1.8 GB per chunk) cycle through a pool of at most 8 GB
     per_chunk = wl.batch * wl.chunk * (wl.n_q_heads + 2 * wl.n_kv_heads) * wl.head_dim * (
-        2 if wl.dtype == "bf16" else 4)
+        4 if wl.dtype == "f32" else 2)
     n_pool = max(2, min(W + K + KB, int(8e9 // per_chunk)))
     pool = [src.chunk(fill + c) for c in range(n_pool)]
     chunks = [pool[c % n_pool] for c in range(W + K + KB)]
@@ -542,12 +545,14 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": round(total_ms / K, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if wl.dtype == "f32" else "bf16",
         "data": data_note(wl),
         "config": {"workload": wl.name, "caches_per_gpu": wl.batch, "n_q_heads": wl.n_q_heads,
                    "n_kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "chunk": wl.chunk,
                    "capacity": wl.capacity, "recent_window": wl.window, "policy": wl.policy,
                    "sink_tokens": wl.sinks,
+                   "kv_format": ("int8 codes + fp32 row scales" if wl.dtype == "q8" else wl.dtype),
                    "state": "steady (cache full)", "parallelism": f"independent caches x{world}",
                    "l2": "flushed before every timed step (256 MiB write, outside the events)"},
         "roofline": roof,

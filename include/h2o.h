@@ -34,6 +34,8 @@
  *   q, out            [batch, n_q, H_q, head_dim]      element type = dtype
  *   k_new, v_new      [batch, n_q, H_kv, head_dim]     element type = dtype
  *   cache k, v        [batch, H_kv, capacity, head_dim] element type = dtype
+ *                     (Q8: int8 codes, then [batch, H_kv, capacity] float32
+ *                     scales, see h2o_dtype)
  *   scores            [batch, H_kv, capacity]          float32
  *   pos               [batch, H_kv, capacity]          int32, -1 = empty slot
  *   state             [4] int32: n, t0, device error bits, reserved
@@ -52,8 +54,8 @@
  *     streams and events that h2o_chunk_step_host creates on first use.
  *   - All caches of a handle advance together (one n_q per call).  A handle
  *     must not be used from two host threads at once.
- *   - Supported: head_dim 64 or 128; dtype BF16 (tensor-core path) or F32
- *     (fp32 FMA path); H_q a multiple of H_kv; 0 <= recent_window <=
+ *   - Supported: head_dim 64 or 128; dtype BF16 or Q8 (tensor-core path) or
+ *     F32 (fp32 FMA path); H_q a multiple of H_kv; 0 <= recent_window <=
  *     capacity; capacity + max_chunk <= 50176 (the selection keeps one fp32
  *     key per candidate in shared memory).
  */
@@ -81,11 +83,26 @@ typedef enum {
   H2O_ERR_ALIGN = 4,       /* pointer not 16-byte (workspace: 256-byte) aligned */
   H2O_ERR_CUDA = 5,        /* a CUDA runtime call failed                     */
   H2O_ERR_TIMEOUT = 6,     /* a kernel's bounded wait expired (device bit 1) */
-  H2O_ERR_STATE = 7        /* inconsistent eviction plan (device bit 2) or a
-                              kernel's shared-memory layout check (bit 4)    */
+  H2O_ERR_STATE = 7        /* inconsistent eviction plan (device bit 2), a
+                              kernel's shared-memory layout check (bit 4), or,
+                              in the H2O_DEBUG build libh2o_debug.so, a failed
+                              bounds check (bit 8; the access is skipped)    */
 } h2o_status;
 
-typedef enum { H2O_BF16 = 0, H2O_F32 = 1 } h2o_dtype;
+/* Element types.  BF16 and F32: q, k_new, v_new, out and the cache's K and V
+ * all of that type.  Q8 (the quantised cache of Q-Hitter, page 1 §2 Related
+ * Work: "Q-Hitter combines H2O with quantisation"; summary page Table 5,
+ * qh2o rows -- the pages give no format, this is the one read here): q,
+ * k_new, v_new and out are bf16; every cache row (one slot of one KV head, K
+ * and V separately) is stored as head_dim int8 codes and one fp32 scale,
+ *   s = fl32(max|x| / 127),  code = clamp(rint(fl32(x / s)), -127, 127)
+ * (ties to even; an all-zero row has s = 0), and the attention reads
+ * bf16(fl32(code * s)).  A new token is quantised when it is placed into the
+ * cache; within the step that brings it, it is attended at its bf16 input
+ * value.  The cache K (and V) buffer holds the codes
+ * [batch, H_kv, capacity, head_dim] int8 followed by the scales
+ * [batch, H_kv, capacity] float32. */
+typedef enum { H2O_BF16 = 0, H2O_F32 = 1, H2O_Q8 = 2 } h2o_dtype;
 
 /* Eviction policy.  H2O ranks the unprotected candidates by their
  * accumulated attention (the summed weights added to the score each step);
@@ -196,7 +213,7 @@ H2O_API h2o_status h2o_attention(h2o_cache* c, const void* q, const void* k_new,
  * out, d_out: device [batch, n_q, H_q, d] bf16 (O of that call and dL/dO).
  * Outputs, device float32, 16-byte aligned: dq [batch, n_q, H_q, d];
  * dk_cache, dv_cache [batch, H_kv, C, d] (rows of slots >= n are zero);
- * dk_new, dv_new [batch, n_q, H_kv, d].  BF16 caches only (else
+ * dk_new, dv_new [batch, n_q, H_kv, d].  BF16 caches only (F32 and Q8:
  * H2O_ERR_DTYPE); n_q >= 2 (a one-token h2o_attention runs the decode
  * kernels, which keep no row statistics).  Deterministic (fixed reduction
  * order). */
@@ -253,7 +270,8 @@ H2O_API h2o_status h2o_cache_kernel_ms(h2o_cache* c, float* ms4);
  * until the process exits), so
  *   batch * n_q_heads * (n_q rounded up to a multiple of 128) <= 4194304
  * or the call returns H2O_ERR_SHAPE before launching anything.
- * Inputs: cfg (capacity, heads, head_dim, dtype, scale; max_chunk bounds
+ * Inputs: cfg (capacity, heads, head_dim, dtype BF16 or F32 (Q8:
+ * H2O_ERR_DTYPE), scale; max_chunk bounds
  * n_q; recent_window unused), k_cache / v_cache (device, cache layout) with
  * n valid slots, q, k_new, v_new (device, chunk layouts).  Outputs (device):
  * out, and colsum_out in the colsum layout for this n_q (required).
@@ -287,6 +305,14 @@ H2O_API h2o_status h2o_static_scratch_check(void* stream);
  * stays usable.  No trap, no hang. */
 H2O_API h2o_status h2o_selftest_wait_timeout(int32_t* err_word, uint32_t limit_us,
                                              void* stream);
+
+/* Diagnostic of the kernels' FMA-pipe exponential: y[i] = 2^x[i] computed
+ * the way the attention kernels compute part of their exponentials without
+ * the special function unit (Cody-Waite range reduction and a degree-3
+ * minimax polynomial: relative error below 7.5e-5 for -125 <= x <= 0; x
+ * below -125, -inf included, gives about 2^-125).  x, y: device float32 arrays
+ * of n elements.  No counterpart in the paper. */
+H2O_API h2o_status h2o_selftest_exp2(const float* x, float* y, int32_t n, void* stream);
 
 /* Waits for the copies h2o_chunk_step_host still has in flight, then frees
  * the host handle and its copy streams and events.  Device buffers stay the

@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libh2o.so")
 
 H2O_OK = 0
-H2O_BF16, H2O_F32 = 0, 1
+H2O_BF16, H2O_F32, H2O_Q8 = 0, 1, 2
 POLICIES = {"h2o": 0, "lr": 1, "slr": 2}  # h2o_policy
 STATUS_NAMES = {0: "H2O_OK", 1: "H2O_ERR_INVALID_ARG", 2: "H2O_ERR_SHAPE", 3: "H2O_ERR_DTYPE",
                 4: "H2O_ERR_ALIGN", 5: "H2O_ERR_CUDA", 6: "H2O_ERR_TIMEOUT", 7: "H2O_ERR_STATE"}
@@ -26,7 +26,8 @@ EXPORTED = ["h2o_required_bytes", "h2o_cache_create", "h2o_chunk_step", "h2o_chu
             "h2o_cache_host_join", "h2o_attention", "h2o_attention_backward", "h2o_evict",
             "h2o_cache_read", "h2o_cache_write", "h2o_cache_check", "h2o_cache_info",
             "h2o_cache_set_timing", "h2o_cache_kernel_ms", "h2o_attention_static_scratch",
-            "h2o_static_scratch_check", "h2o_selftest_wait_timeout", "h2o_cache_destroy",
+            "h2o_static_scratch_check", "h2o_selftest_wait_timeout", "h2o_selftest_exp2",
+            "h2o_cache_destroy",
             "h2o_status_string"]
 
 
@@ -73,6 +74,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                                  P, P]
     lib.h2o_static_scratch_check.argtypes = [P]
     lib.h2o_selftest_wait_timeout.argtypes = [P, ctypes.c_uint32, P]
+    lib.h2o_selftest_exp2.argtypes = [P, P, I, P]
     lib.h2o_evict.argtypes = [P, P, P, P, I, P]
     lib.h2o_cache_read.argtypes = [P, P, P, P, P, P, P]
     lib.h2o_cache_write.argtypes = [P, P, P, P, P, P, P]
@@ -124,13 +126,22 @@ class CacheShape:
     capacity: int
     max_chunk: int
     recent_window: int
-    dtype: torch.dtype = torch.bfloat16
+    dtype: torch.dtype = torch.bfloat16   # torch.int8: the int8 cache (Q8), bf16 activations
     softmax_scale: float = 0.0
     policy: str = "h2o"     # "h2o", "lr" or "slr"
     sink_tokens: int = 0    # "slr": the first positions that always stay
 
+    @property
+    def q8(self) -> bool:
+        return self.dtype == torch.int8
+
+    @property
+    def act_dtype(self) -> torch.dtype:
+        """Element type of q, k_new, v_new and out."""
+        return torch.bfloat16 if self.q8 else self.dtype
+
     def config(self) -> Config:
-        dt = {torch.bfloat16: H2O_BF16, torch.float32: H2O_F32}[self.dtype]
+        dt = {torch.bfloat16: H2O_BF16, torch.float32: H2O_F32, torch.int8: H2O_Q8}[self.dtype]
         return Config(self.batch, self.n_q_heads, self.n_kv_heads, self.head_dim, self.capacity,
                       self.max_chunk, self.recent_window, dt, self.softmax_scale,
                       POLICIES[self.policy], self.sink_tokens)
@@ -158,8 +169,13 @@ class H2OCache:
         sz = required_bytes(shape)
         s = shape
         kw = dict(device=self.device)
-        self.k = torch.empty(s.batch, s.n_kv_heads, s.capacity, s.head_dim, dtype=s.dtype, **kw)
-        self.v = torch.empty_like(self.k)
+        if s.q8:
+            # int8 codes [B, H_kv, C, d] followed by fp32 scales [B, H_kv, C]
+            self.k = torch.empty(sz.k_bytes, dtype=torch.uint8, **kw)
+            self.v = torch.empty_like(self.k)
+        else:
+            self.k = torch.empty(s.batch, s.n_kv_heads, s.capacity, s.head_dim, dtype=s.dtype, **kw)
+            self.v = torch.empty_like(self.k)
         self.scores = torch.empty(s.batch, s.n_kv_heads, s.capacity, dtype=torch.float32, **kw)
         self.pos = torch.empty(s.batch, s.n_kv_heads, s.capacity, dtype=torch.int32, **kw)
         self.state = torch.zeros(4, dtype=torch.int32, **kw)
@@ -189,7 +205,7 @@ class H2OCache:
     # ----------------------------------------------------------------- shapes
     def _alloc_out(self, n_q):
         s = self.shape
-        return torch.empty(s.batch, n_q, s.n_q_heads, s.head_dim, dtype=s.dtype,
+        return torch.empty(s.batch, n_q, s.n_q_heads, s.head_dim, dtype=s.act_dtype,
                            device=self.device)
 
     def _alloc_colsum(self, n_q):
@@ -200,7 +216,7 @@ class H2OCache:
     def _check_inputs(self, q, k_new, v_new):
         s = self.shape
         for t in (q, k_new, v_new):
-            if t.device != self.device or t.dtype != s.dtype or not t.is_contiguous():
+            if t.device != self.device or t.dtype != s.act_dtype or not t.is_contiguous():
                 raise ValueError("inputs must be contiguous tensors of the cache's dtype on its device")
         n_q = q.shape[1]
         if q.shape != (s.batch, n_q, s.n_q_heads, s.head_dim) or \
@@ -259,7 +275,7 @@ class H2OCache:
         dkn = torch.empty(s.batch, n_q, s.n_kv_heads, s.head_dim, **f)
         dvn = torch.empty_like(dkn)
         out = out.contiguous()
-        d_out = d_out.to(device=self.device, dtype=s.dtype).contiguous()
+        d_out = d_out.to(device=self.device, dtype=s.act_dtype).contiguous()
         _check("h2o_attention_backward", lib().h2o_attention_backward(
             self._h, _ptr(q), _ptr(k_new), _ptr(v_new), n_q, _ptr(out), _ptr(d_out), _ptr(dq),
             _ptr(dkc), _ptr(dvc), _ptr(dkn), _ptr(dvn), _stream(stream)))
@@ -272,6 +288,8 @@ class H2OCache:
                                             n_q, _stream(stream)))
 
     def read(self, stream=None):
+        """The cache state.  For the int8 cache (Q8) k and v are the codes
+        [B, H_kv, C, d] int8 and k_scale, v_scale the row scales [B, H_kv, C]."""
         s = self.shape
         k = torch.empty_like(self.k)
         v = torch.empty_like(self.v)
@@ -281,11 +299,33 @@ class H2OCache:
         _check("h2o_cache_read", lib().h2o_cache_read(self._h, _ptr(k), _ptr(v), _ptr(scores),
                                                       _ptr(pos), nt, _stream(stream)))
         torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
-        del s
-        return dict(k=k, v=v, scores=scores, pos=pos, n=nt[0], t0=nt[1])
+        out = dict(k=k, v=v, scores=scores, pos=pos, n=nt[0], t0=nt[1])
+        if s.q8:
+            for name, raw in (("k", k), ("v", v)):
+                codes, scale = self.split_q8(raw)
+                out[name], out[name + "_scale"] = codes, scale
+        return out
 
-    def write(self, k, v, scores, pos, n, t0, stream=None):
+    def split_q8(self, raw: torch.Tensor):
+        """(codes, scales) views of a raw int8-cache K or V buffer."""
+        s = self.shape
+        nc = s.batch * s.n_kv_heads * s.capacity * s.head_dim
+        codes = raw[:nc].view(torch.int8).view(s.batch, s.n_kv_heads, s.capacity, s.head_dim)
+        scale = raw[nc:].view(torch.float32).view(s.batch, s.n_kv_heads, s.capacity)
+        return codes, scale
+
+    @staticmethod
+    def join_q8(codes: torch.Tensor, scale: torch.Tensor) -> torch.Tensor:
+        """The raw int8-cache buffer from codes and scales."""
+        return torch.cat([codes.contiguous().view(torch.uint8).reshape(-1),
+                          scale.to(torch.float32).contiguous().view(torch.uint8).reshape(-1)])
+
+    def write(self, k, v, scores, pos, n, t0, stream=None, k_scale=None, v_scale=None):
+        """Replaces the state.  For the int8 cache pass the codes as k, v and
+        the row scales as k_scale, v_scale."""
         nt = (ctypes.c_int32 * 2)(n, t0)
+        if self.shape.q8:
+            k, v = self.join_q8(k, k_scale), self.join_q8(v, v_scale)
         k, v = k.to(self.device).contiguous(), v.to(self.device).contiguous()
         scores = scores.to(self.device, torch.float32).contiguous()
         pos = pos.to(self.device, torch.int32).contiguous()

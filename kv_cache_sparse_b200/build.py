@@ -1,7 +1,10 @@
-"""Builds the CUDA library ``libh2o.so`` in-tree for sm_100a with nvcc.
+"""Builds the CUDA library ``libh2o.so`` in-tree for sm_100a with nvcc, and
+its bounds-checked variant ``libh2o_debug.so`` (compiled with -DH2O_DEBUG:
+device-side checks of computed indices latch an error bit instead of
+accessing memory out of bounds; used by the tests, never by default).
 
-Usage: ``python -m kv_cache_sparse_b200.build [--verbose]``.  The library
-lands next to this file, so it travels with the source tree.
+Usage: ``python -m kv_cache_sparse_b200.build [--verbose] [--force] [--debug]``.
+The libraries land next to this file, so they travel with the source tree.
 """
 from __future__ import annotations
 
@@ -14,6 +17,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libh2o.so")
+DEBUG_LIB = os.path.join(HERE, "libh2o_debug.so")
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 
@@ -42,17 +46,20 @@ def deps():
                               glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    objdir = os.path.join(ROOT, "_build")
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Builds libh2o.so (or, with debug=True, libh2o_debug.so) when a source
+    is newer than it; returns its path."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    objdir = os.path.join(ROOT, "_build", "debug" if debug else "")
     os.makedirs(objdir, exist_ok=True)
     nvcc = nvcc_path()
     extra = ["-Xptxas", "-v"] if verbose else []
@@ -60,7 +67,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     procs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src).replace(".cu", ".o"))
-        cmd = [nvcc, *NVCC_FLAGS, *extra, "-I", INCLUDE, "-c", src, "-o", obj]
+        cmd = [nvcc, *NVCC_FLAGS, *(["-DH2O_DEBUG"] if debug else []), *extra, "-I", INCLUDE,
+               "-c", src, "-o", obj]
         procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE,
                                             stderr=subprocess.STDOUT, text=True)))
         objs.append(obj)
@@ -73,13 +81,14 @@ def build(force: bool = False, verbose: bool = False) -> str:
             failed.append(src)
     if failed:
         raise RuntimeError("nvcc failed for: " + ", ".join(failed))
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp, *objs,
            "-lcudart_static", "-ldl", "-lpthread", "-lrt"]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
+                debug="--debug" in sys.argv))

@@ -41,8 +41,9 @@ cudaError_t launch_attn_f32(int head_dim, const float* q, const float* kc, const
                             cudaStream_t st);
 
 // Decode step (n_q = 1, G in {1, 2, 4, 8}): split-KV partials, then the merge,
-// summed weights and (if p.evict) the single-token eviction.  esize 2 (bf16)
-// or 4 (float), head_dim 64 or 128.
+// summed weights and (if p.evict) the single-token eviction.  esize: bytes per
+// cache element -- 2 (bf16), 4 (float), or 1 (int8 codes with per-row scales;
+// q, out and the new rows bf16); head_dim 64 or 128.
 cudaError_t launch_decode(const DecodeParams& p, int esize, int head_dim, cudaStream_t st);
 // Group sizes the decode kernels take (a warp batch holds 32 / G keys).
 bool decode_supported(int G);

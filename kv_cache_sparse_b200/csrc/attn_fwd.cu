@@ -28,14 +28,20 @@
 // Ordering: the MMA thread issues PV_X(t) and then S_X(t+1) into the same
 // TMEM columns; the commit that signals S_X(t+1) also covers PV_X(t), so the
 // softmax that sees S_X(t+1) may rescale O_X and overwrite P_X.
+//
+// The int8 cache (Q8, q8.cuh): warp 0 brings a cache tile's codes of K and of
+// V into one staging buffer each (TMA, no swizzle), and warps 10 and 11
+// dequantise them into the same bf16 rings the MMA reads (128-byte swizzle),
+// with the row scales; the chunk's own tiles still arrive in bf16 by TMA.
 #include <cuda_bf16.h>
 
 #include "attn.h"
+#include "q8.cuh"
 #include "sm100.cuh"
 
 namespace h2o {
 
-template <int D>
+template <int D, bool Q8 = false>
 struct FwdLayout {
   static constexpr int kRegions = D / 64;         // 128-byte column blocks of a row
   static constexpr int kTileBytes = 128 * D * 2;  // 128 rows of Q, K or V
@@ -44,26 +50,39 @@ struct FwdLayout {
   static constexpr int kQOff = 0;  // Q_A, Q_B
   static constexpr int kKOff = kQOff + 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
-  static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
+  // Q8: int8 codes of one K and one V cache tile (128 rows x D bytes each)
+  static constexpr int kCodeBytes = Q8 ? 128 * D : 0;
+  static constexpr int kK8Off = kVOff + kVStages * kTileBytes;
+  static constexpr int kV8Off = kK8Off + kCodeBytes;
+  static constexpr int kBarOff = kV8Off + kCodeBytes;
   // q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2], p_full[2],
-  // o_done[2], drain
-  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1;
+  // o_done[2], drain; Q8: k8_full, k8_empty, v8_full, v8_empty
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1 + (Q8 ? 4 : 0);
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = (kBytes + 1024 < kMaxDynSmem) ? kBytes + 1024 : kMaxDynSmem;
   static_assert(kBytes <= kMaxDynSmem, "shared-memory layout too large");
   static constexpr int kTmemCols = 512;  // S/P_A | S/P_B | O_A | O_B
-  static constexpr int kThreads = 320;
+  // warpgroup 0: warp 0 TMA, warp 1 MMA, warps 2-3 dequantise (Q8) or idle;
+  // warpgroups 1 and 2: the softmax of tiles A and B.  Launched with 168
+  // registers per thread (384 x 168 <= 64 K); warpgroup 0 gives registers
+  // back so that the softmax warpgroups hold kSoftmaxRegs each:
+  // 128 x kLoadRegs + 256 x kSoftmaxRegs <= 384 x 168, and per SM
+  // sub-partition (one warp of each group) kLoadRegs + 2 kSoftmaxRegs <= 512.
+  static constexpr int kThreads = 384;
+  static constexpr uint32_t kLoadRegs = 80;
+  static constexpr uint32_t kSoftmaxRegs = 200;
+  static_assert(128 * kLoadRegs + 256 * kSoftmaxRegs <= 384 * 168, "register budget");
 };
 
-template <int D>
-__global__ void __launch_bounds__(320, 1)
+template <int D, bool Q8>
+__global__ void __launch_bounds__(FwdLayout<D, Q8>::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_kc,
                     const __grid_constant__ CUtensorMap tm_vc,
                     const __grid_constant__ CUtensorMap tm_kn,
                     const __grid_constant__ CUtensorMap tm_vn, const AttnParams p) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, Q8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   if ((smem - smem_raw) + L::kBytes > L::kAlloc) {  // cannot happen with an aligned base
@@ -104,6 +123,8 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t bar_p_full0 = bar_s_full0 + 16;                // [2]: P_X(t) in TMEM
   const uint32_t bar_o_done0 = bar_p_full0 + 16;                // [2]: last PV_X done
   const uint32_t bar_drain = bar_o_done0 + 16;
+  const uint32_t bar_k8_full = bar_drain + 8, bar_k8_empty = bar_drain + 16;  // Q8 only
+  const uint32_t bar_v8_full = bar_drain + 24, bar_v8_empty = bar_drain + 32;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -123,6 +144,12 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(bar_o_done0 + 8 * x, 1);
     }
     mbar_init(bar_drain, 1);
+    if (Q8) {
+      mbar_init(bar_k8_full, 1);
+      mbar_init(bar_k8_empty, 1);
+      mbar_init(bar_v8_full, 1);
+      mbar_init(bar_v8_empty, 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -134,7 +161,9 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp < 4) {
+  // warpgroup 0 (TMA, MMA, dequantising) hands registers to the softmax groups
+  warpgroup_reg_dec<L::kLoadRegs>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -145,11 +174,26 @@ __global__ void __launch_bounds__(320, 1)
         for (int r = 0; r < L::kRegions; ++r)
           tma_load_4d(sbase + L::kQOff + L::kTileBytes + r * 16384, &tm_q, bar_q, r * 64, hB,
                       qtB * 128, b);
-      int issued_k = 0, issued_v = 0;
+      int issued_k = 0, issued_v = 0, issued8 = 0;
       bool ok = true;
       for (int t = 0; t < Tmax && ok; ++t) {
         const bool chunk = t >= NCT;
         const int j0 = (chunk ? t - NCT : t) * 128;
+        if (Q8 && !chunk) {  // the codes of K(t) and V(t) into the staging buffers
+          for (int w = 0; w < 2; ++w) {
+            const uint32_t full = w ? bar_v8_full : bar_k8_full;
+            const uint32_t empty = w ? bar_v8_empty : bar_k8_empty;
+            if (t >= 1 && !mbar_wait(empty, (t + 1) & 1, p.err, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(full, L::kCodeBytes);
+            tma_load_3d(sbase + (w ? L::kV8Off : L::kK8Off), w ? &tm_vc : &tm_kc, full, 0, j0,
+                        b * p.Hkv + g);
+          }
+          issued8 = t + 1;
+          continue;
+        }
         for (int w = 0; w < 2; ++w) {  // K(t), then V(t)
           const int NS = w ? L::kVStages : L::kKStages;
           const uint32_t full0 = w ? bar_v_full0 : bar_k_full0;
@@ -173,9 +217,14 @@ __global__ void __launch_bounds__(320, 1)
       }
       // drain: every issued copy has landed before the CTA can exit
       mbar_wait_drain(bar_q, 0, p.err);
-      for (int t = (issued_k > L::kKStages ? issued_k - L::kKStages : 0); t < issued_k; ++t)
+      if (Q8 && issued8 > 0) {
+        mbar_wait_drain(bar_k8_full, (issued8 - 1) & 1, p.err);
+        mbar_wait_drain(bar_v8_full, (issued8 - 1) & 1, p.err);
+      }
+      const int t_tma = Q8 ? NCT : 0;  // Q8: the cache tiles were not copied by TMA
+      for (int t = max(t_tma, issued_k - L::kKStages); t < issued_k; ++t)
         mbar_wait_drain(bar_k_full0 + 8 * (t % L::kKStages), (t / L::kKStages) & 1, p.err);
-      for (int t = (issued_v > L::kVStages ? issued_v - L::kVStages : 0); t < issued_v; ++t)
+      for (int t = max(t_tma, issued_v - L::kVStages); t < issued_v; ++t)
         mbar_wait_drain(bar_v_full0 + 8 * (t % L::kVStages), (t / L::kVStages) & 1, p.err);
     }
   } else if (warp == 1) {
@@ -240,9 +289,65 @@ __global__ void __launch_bounds__(320, 1)
       mma_commit(bar_drain);
       mbar_wait_drain(bar_drain, 0, p.err);
     }
+  } else if (warp < 4) {
+    // warps 2 and 3: no role without the int8 cache
+    if (Q8) {
+    // ------------------------------------------------------------ dequantise (Q8)
+    // cache tile t: codes (staging) -> bf16 ring slot t % 2 of K, then of V.
+    // 128 x D codes in pieces of 16 (one 16-byte row piece each, consecutive
+    // threads on consecutive pieces); each piece becomes two 16-byte chunks of
+    // its 128-byte region row, at chunk index ^ (row & 7) (the swizzle).
+    constexpr int kPer = D / 16;                    // pieces per row
+    constexpr int kJobs = 128 * kPer / 64;          // pieces per thread and tile
+    const int ct = threadIdx.x - 64;                // 0 .. 63
+    bool ok = true;
+    for (int t = 0; t < NCT && ok; ++t) {
+      const int j0 = t * 128;
+      for (int w = 0; w < 2 && ok; ++w) {
+        const float* scale = (w ? p.v_scale : p.k_scale) + static_cast<size_t>(bg) * p.C;
+        float sc[kJobs];
+#pragma unroll
+        for (int k = 0; k < kJobs; ++k) {
+          const int r = (ct + 64 * k) / kPer;
+          sc[k] = j0 + r < p.n ? scale[j0 + r] : 0.f;
+        }
+        const int NS = w ? L::kVStages : L::kKStages;
+        const int s = t % NS;
+        ok = mbar_wait(w ? bar_v8_full : bar_k8_full, t & 1, p.err, abort_flag);
+        if (ok && t >= NS)
+          ok = mbar_wait((w ? bar_v_empty0 : bar_k_empty0) + 8 * s, ((t / NS) + 1) & 1, p.err,
+                         abort_flag);
+        ok = named_bar_and(1, 64, ok);  // every converter thread takes the same branch
+        if (!ok) break;
+        const uint8_t* codes = smem + (w ? L::kV8Off : L::kK8Off);
+        uint8_t* dst = smem + (w ? L::kVOff : L::kKOff) + s * L::kTileBytes;
+#pragma unroll 4
+        for (int k = 0; k < kJobs; ++k) {
+          const int job = ct + 64 * k;
+          const int r = job / kPer, i = job % kPer;
+          uint32_t wv[8];
+          q8_dequant16(*reinterpret_cast<const uint4*>(codes + r * D + 16 * i), sc[k], wv);
+          const int e = 16 * i;
+          const int reg = e / 64, c16 = (e % 64) / 8;
+          uint8_t* rowp = dst + reg * 16384 + r * 128;
+          *reinterpret_cast<uint4*>(rowp + ((c16 ^ (r & 7)) * 16)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          *reinterpret_cast<uint4*>(rowp + (((c16 + 1) ^ (r & 7)) * 16)) =
+              make_uint4(wv[4], wv[5], wv[6], wv[7]);
+        }
+        fence_proxy_async_smem();  // the MMA reads the operand through the async proxy
+        named_bar_sync(1, 64);     // all 64 converters are done with the codes and the slot
+        if (ct == 0) {
+          mbar_arrive((w ? bar_v_full0 : bar_k_full0) + 8 * s);
+          mbar_arrive(w ? bar_v8_empty : bar_k8_empty);
+        }
+      }
+    }
+    }
+  }
   } else {
     // ------------------------------------------------------------ softmax rows
-    const int x = (warp - 2) >> 2;  // tile A or B
+    warpgroup_reg_inc<L::kSoftmaxRegs>();
+    const int x = (warp - 4) >> 2;  // tile A or B
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const int T = x ? TB : TA;
@@ -369,8 +474,9 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
         }
-        p.nlse2[(static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + i] =
-            (i < p.nq) ? -(m_used + __log2f(l)) : -INFINITY;
+        if (H2O_IN_BOUNDS(i < p.nq_pad && h < p.Hq && b < p.B, p.err))
+          p.nlse2[(static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + i] =
+              (i < p.nq) ? -(m_used + __log2f(l)) : -INFINITY;
       }
     }
   }
@@ -384,22 +490,24 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
-template <int D>
+template <int D, bool Q8>
 static cudaError_t launch_fwd(const AttnMaps& m, const AttnParams& p, cudaStream_t st) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, Q8>;
   static int attr_bits[2] = {0, 0};
-  cudaError_t e =
-      ensure_smem_attr(reinterpret_cast<const void*>(attn_fwd_kernel<D>), L::kAlloc, attr_bits);
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(attn_fwd_kernel<D, Q8>),
+                                   L::kAlloc, attr_bits);
   if (e != cudaSuccess) return e;
   const int pairs = cdiv(p.G * cdiv(p.nq, 128), 2);
   const int grid = p.B * p.Hkv * pairs;
-  attn_fwd_kernel<D><<<grid, L::kThreads, L::kAlloc, st>>>(m.q, m.kc, m.vc, m.kn, m.vn, p);
+  attn_fwd_kernel<D, Q8><<<grid, L::kThreads, L::kAlloc, st>>>(m.q, m.kc, m.vc, m.kn, m.vn, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_fwd_bf16(int head_dim, const AttnMaps& m, const AttnParams& p,
                                  cudaStream_t st) {
-  return head_dim == 128 ? launch_fwd<128>(m, p, st) : launch_fwd<64>(m, p, st);
+  const bool q8 = p.k_scale != nullptr;  // int8 cache
+  if (head_dim == 128) return q8 ? launch_fwd<128, true>(m, p, st) : launch_fwd<128, false>(m, p, st);
+  return q8 ? launch_fwd<64, true>(m, p, st) : launch_fwd<64, false>(m, p, st);
 }
 
 }  // namespace h2o

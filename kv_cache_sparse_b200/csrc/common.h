@@ -11,6 +11,22 @@ namespace h2o {
 constexpr int kDevErrTimeout = 1;  // a bounded mbarrier wait expired
 constexpr int kDevErrPlan = 2;     // freed-slot and kept-token counts disagree
 constexpr int kDevErrSmem = 4;     // dynamic shared memory too small after alignment
+constexpr int kDevErrBounds = 8;   // H2O_DEBUG builds: an index failed its bounds check
+
+// Bounds checks of the H2O_DEBUG build (libh2o_debug.so): a failed check
+// latches kDevErrBounds in the error word and the access is skipped; it never
+// traps.  In the normal build the checks compile to nothing.
+#if defined(__CUDACC__)
+#ifdef H2O_DEBUG
+__device__ __forceinline__ bool debug_in_bounds(bool ok, int* err) {
+  if (!ok) atomicOr(err, kDevErrBounds);
+  return ok;
+}
+#define H2O_IN_BOUNDS(cond, err) ::h2o::debug_in_bounds((cond), (err))
+#else
+#define H2O_IN_BOUNDS(cond, err) true
+#endif
+#endif
 
 // Largest dynamic shared memory a CTA may request on sm_100 (227 KiB).
 constexpr int kMaxDynSmem = 232448;
@@ -55,6 +71,10 @@ struct AttnParams {
   float* colsum;        // [B, Hkv, colsum_ld]
   int colsum_ld;        // row stride of colsum (>= C + nq)
   int* err;             // device error word (state + 2)
+  // int8 cache (Q8): one fp32 scale per (cache, KV head, slot) of K and V,
+  // [B*Hkv, C]; null for the bf16 cache
+  const float* k_scale;
+  const float* v_scale;
 };
 
 // Arguments of the backward kernels (attn_bwd.cu).
@@ -96,6 +116,11 @@ struct EvictParams {
   int* state;               // [4]: n, t0, err, reserved
   int policy;               // kPolicyH2O (rank by score), kPolicyLR / kPolicySLR (by position)
   int sinks;                // kPolicySLR: positions < sinks are protected
+  // int8 cache (Q8): new rows (bf16, esize 2 in k_new / v_new) are quantised
+  // into the cache's int8 codes (esize is then 1) and per-slot scales
+  int q8;
+  float* k_scale;           // [B*Hkv, C]
+  float* v_scale;
 };
 
 // ---------------------------------------------------------------- decode (n_q = 1)
@@ -135,6 +160,9 @@ struct DecodeParams {
   int evict;                // 1: score update and placement after the attention
   int policy;               // as in EvictParams
   int sinks;
+  float* k_scale;           // int8 cache (Q8): per-slot scales [B*Hkv, C]; else null
+  float* v_scale;
 };
+
 
 }  // namespace h2o

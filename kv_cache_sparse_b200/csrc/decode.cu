@@ -39,6 +39,7 @@
 #include <cuda_bf16.h>
 
 #include "attn.h"
+#include "q8.cuh"
 #include "sm100.cuh"
 
 namespace h2o {
@@ -80,6 +81,20 @@ __device__ __forceinline__ void lds_row<float, 2>(const uint8_t* src, float (&f)
   f[0] = v.x; f[1] = v.y;
 }
 
+// E codes of an int8 cache row (Q8) and its scale -> the values the
+// attention reads (q8.cuh).
+template <int E>
+__device__ __forceinline__ void lds_q8(const uint8_t* src, float s, float (&f)[E]) {
+  if (E == 4) {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(src);
+#pragma unroll
+    for (int e = 0; e < E; ++e) f[e] = q8_value(static_cast<int8_t>((u >> (8 * e)) & 0xFF), s);
+  } else {
+#pragma unroll
+    for (int e = 0; e < E; ++e) f[e] = q8_value(static_cast<int8_t>(src[e]), s);
+  }
+}
+
 __device__ __forceinline__ float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
 __device__ __forceinline__ float to_float(float v) { return v; }
 __device__ __forceinline__ void store(__nv_bfloat16* dst, float v) { *dst = __float2bfloat16_rn(v); }
@@ -113,20 +128,25 @@ __device__ __forceinline__ void copy_row(void* dst, const void* src, int bytes, 
         *reinterpret_cast<const uint4*>(static_cast<const char*>(src) + o);
 }
 
-template <typename T, int D, int G>
+// T: element type of q, out and the new rows; Q8: the cache holds int8 codes
+// with one fp32 scale per row instead of T.
+template <typename T, int D, int G, bool Q8>
 struct PartialLayout {
-  static constexpr int KC = decode_chunk_keys(D, sizeof(T));
-  static constexpr int kRow = D * static_cast<int>(sizeof(T));
-  static constexpr int kK = 0;                          // [KC][D] T
-  static constexpr int kV = kK + KC * kRow;             // [KC][D] T
+  static constexpr int kCode = Q8 ? 1 : static_cast<int>(sizeof(T));  // bytes per cache element
+  static constexpr int KC = decode_chunk_keys(D, kCode);
+  static constexpr int kRow = D * kCode;
+  static constexpr int kK = 0;                          // [KC][D] cache rows of K
+  static constexpr int kV = kK + KC * kRow;             // [KC][D] of V
   static constexpr int kX = kV + KC * kRow;             // [G][KC] float: logits, then P
   static constexpr int kO = kX + G * KC * 4;            // [warps][G][D] float
-  static constexpr int kBytes = kO + kWarps * G * D * 4;
+  static constexpr int kS = kO + kWarps * G * D * 4;    // Q8: [2][KC] float scales of K, V
+  static constexpr int kN = kS + (Q8 ? 2 * KC * 4 : 0);  // Q8: the new token's K, V rows (T)
+  static constexpr int kBytes = kN + (Q8 ? 2 * D * static_cast<int>(sizeof(T)) : 0);
 };
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool Q8>
 __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p) {
-  using L = PartialLayout<T, D, G>;
+  using L = PartialLayout<T, D, G, Q8>;
   constexpr int KC = L::KC;
   constexpr int E = D / 32;   // row elements per lane
   constexpr int KB = 32 / G;  // keys per warp batch: 32 (key, head) pairs
@@ -166,10 +186,32 @@ __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p)
     mbar_arrive_expect_tx(bV, bytes);
     bulk_load(smem_u32(sV), static_cast<const uint8_t*>(p.v_cache) + off, bytes, bV);
   }
+  constexpr int kNewRow = D * static_cast<int>(sizeof(T));  // the new rows are T
+  uint8_t* sNK = Q8 ? dsm + L::kN : sK + rows * L::kRow;  // the new token's rows
+  uint8_t* sNV = Q8 ? dsm + L::kN + kNewRow : sV + rows * L::kRow;
   if (warp == 0 && nkc > rows) {  // the new token is key n, in this chunk
-    copy_row(sK + rows * L::kRow, static_cast<const uint8_t*>(p.k_new) + bg * L::kRow, L::kRow, lane);
-    copy_row(sV + rows * L::kRow, static_cast<const uint8_t*>(p.v_new) + bg * L::kRow, L::kRow, lane);
+    copy_row(sNK, static_cast<const uint8_t*>(p.k_new) + bg * kNewRow, kNewRow, lane);
+    copy_row(sNV, static_cast<const uint8_t*>(p.v_new) + bg * kNewRow, kNewRow, lane);
   }
+  float* sScale = reinterpret_cast<float*>(dsm + L::kS);  // Q8 only
+  if (Q8) {
+    for (int i = tid; i < KC; i += kThreads) {
+      const size_t at = static_cast<size_t>(bg) * p.C + j0 + i;
+      sScale[i] = i < rows ? p.k_scale[at] : 0.f;
+      sScale[KC + i] = i < rows ? p.v_scale[at] : 0.f;
+    }
+  }
+  // this lane's slice of key (value) row k of the chunk as floats
+  auto kv_row = [&](int k, bool is_v, float (&f)[E]) {
+    if (Q8) {
+      if (k == rows)
+        lds_row<T, E>((is_v ? sNV : sNK) + lane * E * sizeof(T), f);
+      else
+        lds_q8<E>((is_v ? sV : sK) + k * L::kRow + lane * E, sScale[(is_v ? KC : 0) + k], f);
+    } else {
+      lds_row<T, E>((is_v ? sV : sK) + k * L::kRow + lane * E * sizeof(T), f);
+    }
+  };
   // this lane's slice of the G query rows
   float qf[G][E];
   {
@@ -190,7 +232,7 @@ __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p)
 #pragma unroll
       for (int k = 0; k < KB; ++k) {
         float kf[E];
-        lds_row<T, E>(sK + (k0 + k) * L::kRow + lane * E * sizeof(T), kf);
+        kv_row(min(k0 + k, KC - 1), false, kf);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float a = 0.f;
@@ -248,7 +290,7 @@ __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p)
   if (ok) {
     for (int k = warp; k < nkc; k += kWarps) {
       float vf[E];
-      lds_row<T, E>(sV + k * L::kRow + lane * E * sizeof(T), vf);
+      kv_row(k, true, vf);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float pw = xs[h * KC + k];
@@ -262,7 +304,7 @@ __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p)
 #pragma unroll
     for (int e = 0; e < E; ++e) ored[(warp * G + h) * D + lane * E + e] = o[h][e];
   __syncthreads();
-  if (ok) {
+  if (ok && H2O_IN_BOUNDS(chunk < p.part_ld, err)) {
     float* part = p.part + (static_cast<size_t>(bg) * p.part_ld + chunk) * G * (D + 2);
     for (int i = tid; i < G * D; i += kThreads) {
       float s = 0.f;
@@ -280,7 +322,7 @@ __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p)
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool Q8>
 __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) {
   __shared__ float fac[kDecodeMaxG][kMaxChunks];  // 2^(chunk max - head max)
   __shared__ float lse[kDecodeMaxG], lh[kDecodeMaxG];
@@ -364,11 +406,27 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
   const int sinks = p.policy == kPolicySLR ? p.sinks : 0;
   float* score = p.scores + static_cast<size_t>(bg) * C;
   int* pos = p.pos + static_cast<size_t>(bg) * C;
-  const size_t row_bytes = static_cast<size_t>(D) * sizeof(T);
+  const size_t row_bytes = static_cast<size_t>(D) * (Q8 ? 1 : sizeof(T));  // cache rows
+  const size_t new_bytes = static_cast<size_t>(D) * sizeof(T);
   char* kc = static_cast<char*>(p.k_cache) + static_cast<size_t>(bg) * C * row_bytes;
   char* vc = static_cast<char*>(p.v_cache) + static_cast<size_t>(bg) * C * row_bytes;
-  const char* kn = static_cast<const char*>(p.k_new) + static_cast<size_t>(bg) * row_bytes;
-  const char* vn = static_cast<const char*>(p.v_new) + static_cast<size_t>(bg) * row_bytes;
+  const char* kn = static_cast<const char*>(p.k_new) + static_cast<size_t>(bg) * new_bytes;
+  const char* vn = static_cast<const char*>(p.v_new) + static_cast<size_t>(bg) * new_bytes;
+  // the new token's rows into slot `slot`: copied, or quantised (Q8); one warp
+  auto place_new = [&](int slot) {
+    if (!H2O_IN_BOUNDS(slot >= 0 && slot < C, p.state + 2)) return;
+    if (Q8) {
+      q8_quantize_row_warp<D>(reinterpret_cast<const __nv_bfloat16*>(kn),
+                              reinterpret_cast<int8_t*>(kc + static_cast<size_t>(slot) * row_bytes),
+                              p.k_scale + static_cast<size_t>(bg) * C + slot, lane);
+      q8_quantize_row_warp<D>(reinterpret_cast<const __nv_bfloat16*>(vn),
+                              reinterpret_cast<int8_t*>(vc + static_cast<size_t>(slot) * row_bytes),
+                              p.v_scale + static_cast<size_t>(bg) * C + slot, lane);
+    } else {
+      copy_row(kc + static_cast<size_t>(slot) * row_bytes, kn, static_cast<int>(row_bytes), lane);
+      copy_row(vc + static_cast<size_t>(slot) * row_bytes, vn, static_cast<int>(row_bytes), lane);
+    }
+  };
   if (bg == 0 && slice == 0 && tid == 0) {
     p.state[0] = min(C, n + 1);
     p.state[1] = p.t0 + 1;
@@ -382,10 +440,7 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
         score[n] = by_score ? cs[C] : 0.f;
         pos[n] = p.t0;
       }
-      if (warp == 0) {
-        copy_row(kc + n * row_bytes, kn, static_cast<int>(row_bytes), lane);
-        copy_row(vc + n * row_bytes, vn, static_cast<int>(row_bytes), lane);
-      }
+      if (warp == 0) place_new(n);
     }
     return;
   }
@@ -421,7 +476,8 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
   if (tid == 0) {
     unsigned long long m = wmin[0];
     for (int w = 1; w < kWarps; ++w) m = wmin[w] < m ? wmin[w] : m;
-    p.best[static_cast<size_t>(bg) * p.slices_ld + slice] = m;
+    if (H2O_IN_BOUNDS(slice < p.slices_ld, p.state + 2))
+      p.best[static_cast<size_t>(bg) * p.slices_ld + slice] = m;
     __threadfence();  // candidate, scores and summed weights before the ticket
     is_last = atomicAdd(&p.ticket[bg], 1) == static_cast<int>(gridDim.x) - 1;
   }
@@ -446,30 +502,29 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
       score[e] = by_score ? __ldcg(&cs[C]) : 0.f;
       pos[e] = p.t0;
     }
-    copy_row(kc + static_cast<size_t>(e) * row_bytes, kn, static_cast<int>(row_bytes), lane);
-    copy_row(vc + static_cast<size_t>(e) * row_bytes, vn, static_cast<int>(row_bytes), lane);
+    place_new(e);
   }
 }
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool Q8>
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t st) {
-  using L = PartialLayout<T, D, G>;
+  using L = PartialLayout<T, D, G, Q8>;
   static int attr_bits[2] = {0, 0};
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(decode_partial<T, D, G>),
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(decode_partial<T, D, G, Q8>),
                                    L::kBytes, attr_bits);
   if (e != cudaSuccess) return e;
-  decode_partial<T, D, G><<<dim3(p.n_chunks, p.B * p.Hkv), kThreads, L::kBytes, st>>>(p);
+  decode_partial<T, D, G, Q8><<<dim3(p.n_chunks, p.B * p.Hkv), kThreads, L::kBytes, st>>>(p);
   return cudaGetLastError();
 }
 
-template <typename T, int D>
+template <typename T, int D, bool Q8 = false>
 cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
   cudaError_t e;
   switch (p.G) {
-    case 1: e = launch_partial<T, D, 1>(p, st); break;
-    case 2: e = launch_partial<T, D, 2>(p, st); break;
-    case 4: e = launch_partial<T, D, 4>(p, st); break;
-    case 8: e = launch_partial<T, D, 8>(p, st); break;
+    case 1: e = launch_partial<T, D, 1, Q8>(p, st); break;
+    case 2: e = launch_partial<T, D, 2, Q8>(p, st); break;
+    case 4: e = launch_partial<T, D, 4, Q8>(p, st); break;
+    case 8: e = launch_partial<T, D, 8, Q8>(p, st); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
@@ -483,7 +538,7 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_finish<T, D>, p);
+  return cudaLaunchKernelEx(&cfg, decode_finish<T, D, Q8>, p);
 }
 
 }  // namespace
@@ -493,6 +548,9 @@ bool decode_supported(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
 cudaError_t launch_decode(const DecodeParams& p, int esize, int head_dim, cudaStream_t st) {
   if (p.n_chunks > kMaxChunks || !decode_supported(p.G) || p.n_slices > p.slices_ld)
     return cudaErrorInvalidValue;
+  if (esize == 1)  // int8 cache, bf16 activations
+    return head_dim == 128 ? launch<__nv_bfloat16, 128, true>(p, st)
+                           : launch<__nv_bfloat16, 64, true>(p, st);
   if (esize == 2)
     return head_dim == 128 ? launch<__nv_bfloat16, 128>(p, st) : launch<__nv_bfloat16, 64>(p, st);
   return head_dim == 128 ? launch<float, 128>(p, st) : launch<float, 64>(p, st);

@@ -30,6 +30,7 @@
 //      then copies their K and V rows into the slots (16-byte vector loads
 //      and stores, whole rows per warp, several loads in flight per thread).
 #include "attn.h"
+#include "q8.cuh"
 #include "sm100.cuh"
 
 namespace h2o {
@@ -99,14 +100,49 @@ __device__ __forceinline__ void copy_rows(const EvictParams& e, int b, int g, in
 #pragma unroll
     for (int u = 0; u < kCopyBatch; ++u) {
       const int q = q0 + u * tok_step;
-      if (q < count) buf[u] = __ldg(src0 + static_cast<size_t>(tok_of(q)) * src_tok);
+      if (q < count && H2O_IN_BOUNDS(tok_of(q) >= 0 && tok_of(q) < e.nq, e.state + 2))
+        buf[u] = __ldg(src0 + static_cast<size_t>(tok_of(q)) * src_tok);
     }
 #pragma unroll
     for (int u = 0; u < kCopyBatch; ++u) {
       const int q = q0 + u * tok_step;
-      if (q < count) dst0[static_cast<size_t>(slot_of(q)) * vpr_s] = buf[u];
+      if (q < count && H2O_IN_BOUNDS(slot_of(q) >= 0 && slot_of(q) < e.C, e.state + 2))
+        dst0[static_cast<size_t>(slot_of(q)) * vpr_s] = buf[u];
     }
   }
+}
+
+// The int8 cache (Q8): the placed tokens' rows are quantised on the way in.
+// One warp per (token, K or V) row: the row's scale from a warp maximum, its
+// codes written by every lane (q8.cuh).
+template <int NT, int D, class SlotOf, class TokOf>
+__device__ __forceinline__ void quantize_rows(const EvictParams& e, int b, int g, int count,
+                                              SlotOf slot_of, TokOf tok_of) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t bg = static_cast<size_t>(b) * e.Hkv + g;
+  for (int j = warp; j < 2 * count; j += NT / 32) {
+    const int q = j >> 1;
+    const bool is_v = j & 1;
+    const int tok = tok_of(q), slot = slot_of(q);
+    if (!H2O_IN_BOUNDS(tok >= 0 && tok < e.nq && slot >= 0 && slot < e.C, e.state + 2)) continue;
+    const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(is_v ? e.v_new : e.k_new) +
+                               ((static_cast<size_t>(b) * e.nq + tok) * e.Hkv + g) * D;
+    int8_t* dst = static_cast<int8_t*>(is_v ? e.v_cache : e.k_cache) + (bg * e.C + slot) * D;
+    float* sc = (is_v ? e.v_scale : e.k_scale) + bg * e.C + slot;
+    q8_quantize_row_warp<D>(src, dst, sc, lane);
+  }
+}
+
+// The K/V rows of the placed tokens: copied, or quantised for the int8 cache.
+template <int NT, class SlotOf, class TokOf>
+__device__ __forceinline__ void place_rows(const EvictParams& e, int b, int g, int count,
+                                           SlotOf slot_of, TokOf tok_of) {
+  if (!e.q8)
+    copy_rows<NT>(e, b, g, count, slot_of, tok_of);
+  else if (e.d == 128)
+    quantize_rows<NT, 128>(e, b, g, count, slot_of, tok_of);
+  else
+    quantize_rows<NT, 64>(e, b, g, count, slot_of, tok_of);
 }
 
 constexpr int kLoadBatch = 8;  // global loads in flight per thread in the first pass
@@ -212,19 +248,61 @@ __device__ __forceinline__ void find_bin(const int* h, int k, int lane, int* sel
   }
 }
 
+// The single-CTA selection finds the C-th largest key in three digits of
+// 11, 11 and 10 bits (most significant first).  The first digit's histogram
+// is built while the keys are made; the second pass also copies the keys of
+// the chosen first-digit bin into a short list (when they fit), and the last
+// digit is counted over that list only.
+constexpr int kWideBins = 2048;  // 11-bit digits
+constexpr int kListCap = 1024;   // keys of the chosen first-digit bin kept for the last pass
+
+// Adds one to hist[bin] for every lane of the warp with bin >= 0 (lanes with
+// the same bin add together).
+__device__ __forceinline__ void warp_hist_add(int* hist, int bin, int lane) {
+  const unsigned same = __match_any_sync(0xffffffffu, bin);
+  if (bin >= 0 && (__ffs(same) - 1) == lane) atomicAdd(&hist[bin], __popc(same));
+}
+
+// Block-wide: the bin of hist[0, nbins) (counted from the top) that holds the
+// k-th largest key, and the number of keys in the bins above it.  nbins is a
+// multiple of NT; every thread takes nbins / NT consecutive bins.
+template <int NT>
+__device__ __forceinline__ void find_bin_block(const int* hist, int nbins, int k,
+                                               uint64_t* warp_sums, int* sel_bin,
+                                               int* sel_above) {
+  const int per = nbins / NT;
+  const int top = nbins - 1 - static_cast<int>(threadIdx.x) * per;  // this thread: top .. top-per+1
+  int loc = 0;
+  for (int e8 = 0; e8 < per; ++e8) loc += hist[top - e8];
+  uint64_t tot;
+  int run = static_cast<int>(block_excl_scan64<NT>(static_cast<uint64_t>(loc), warp_sums, &tot));
+  if (run < k && run + loc >= k) {
+    for (int e8 = 0; e8 < per; ++e8) {
+      const int cnt = hist[top - e8];
+      if (run + cnt >= k) {
+        *sel_bin = top - e8;
+        *sel_above = run;
+        break;
+      }
+      run += cnt;
+    }
+  }
+}
+
 template <int NT>
 __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
     h2o_select(const EvictParams e, int plan_smem) {
-  constexpr int kSub = (NT == 1024) ? 8 : 2;  // sub-histograms spread the first passes' atomics
   extern __shared__ uint32_t keys[];          // [n + nq], then (plan_smem) the plan [2][nq]
-  __shared__ int hist[kSub][kBins];           // warp w counts into hist[w % kSub]
+  __shared__ int hist[kWideBins];
+  __shared__ uint32_t list[kListCap];
+  __shared__ int list_n;
   __shared__ uint64_t warp_sums[32];
   __shared__ int sel_bin, sel_above;
 
   const int bg = blockIdx.x;
   const int b = bg / e.Hkv, g = bg % e.Hkv;
   const int tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
+  const int lane = tid & 31;
   const int n = e.n, nq = e.nq, C = e.C;
   const int NC = n + nq;
   float* __restrict__ score = e.scores + static_cast<size_t>(bg) * C;
@@ -240,6 +318,9 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
   // W > nq, by the sinks only under SLR
   const bool old_protectable = evict && (e.W > nq || sinks > 0);
   const bool need_pos = old_protectable || !by_score;
+  for (int i = tid; i < kWideBins; i += NT) hist[i] = 0;
+  if (tid == 0) list_n = 0;
+  __syncthreads();
   griddep_wait();  // the summed weights come from the preceding kernel
   if (bg == 0 && tid == 0) {
     e.state[0] = min(C, n + nq);
@@ -309,48 +390,90 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
       pos[n + i] = e.t0 + i;
     }
     if (tid == 0) e.plan_count[bg] = nq;
-    copy_rows<NT>(e, b, g, nq, [n](int q) { return n + q; }, [](int q) { return q; });
+    place_rows<NT>(e, b, g, nq, [n](int q) { return n + q; }, [](int q) { return q; });
     return;
   }
   __syncthreads();
 
-  // 2. radix select of the C-th largest key: four 8-bit digits, MSB first
-  uint32_t prefix = 0, pmask = 0;
+  // 2. the C-th largest key, three digits: bits 31..21 over every key;
+  //    bits 20..10 over the keys of the chosen first-digit bin, which are also
+  //    listed (when they fit); bits 9..0 over that list (or, when it
+  //    overflowed, over every key with the chosen 22-bit prefix)
+  const int iters = (NC + NT - 1) / NT;
+  for (int it = 0; it < iters; ++it) {
+    const int x = it * NT + tid;
+    warp_hist_add(hist, x < NC ? static_cast<int>(keys[x] >> 21) : -1, lane);
+  }
+  __syncthreads();
   int k = C;  // rank (1-based, descending) still to locate
-#pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    constexpr int nb = kBins;
-    for (int i = tid; i < kSub * kBins; i += NT) (&hist[0][0])[i] = 0;
-    __syncthreads();
-    int* my_hist = hist[warp % kSub];
-    const int iters = (NC + NT - 1) / NT;
-    for (int it = 0; it < iters; ++it) {
-      const int x = it * NT + tid;
-      int bin = -1;
-      if (x < NC) {
-        const uint32_t key = keys[x];
-        if ((key & pmask) == prefix) bin = static_cast<int>((key >> shift) & (nb - 1));
+  find_bin_block<NT>(hist, kWideBins, k, warp_sums, &sel_bin, &sel_above);
+  __syncthreads();
+  const uint32_t d1 = static_cast<uint32_t>(sel_bin);
+  k -= sel_above;
+  for (int i = tid; i < kWideBins; i += NT) hist[i] = 0;
+  __syncthreads();
+  for (int it = 0; it < iters; ++it) {
+    const int x = it * NT + tid;
+    const uint32_t key = x < NC ? keys[x] : 0u;
+    const bool in = x < NC && (key >> 21) == d1;
+    warp_hist_add(hist, in ? static_cast<int>((key >> 10) & (kWideBins - 1)) : -1, lane);
+    const unsigned ball = __ballot_sync(0xffffffffu, in);
+    int base = 0;
+    if (lane == 0 && ball) base = atomicAdd(&list_n, __popc(ball));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    const int at = base + __popc(ball & ((1u << lane) - 1u));
+    if (in && at < kListCap) list[at] = key;
+  }
+  __syncthreads();
+  find_bin_block<NT>(hist, kWideBins, k, warp_sums, &sel_bin, &sel_above);
+  __syncthreads();
+  const uint32_t pre22 = (d1 << 11) | static_cast<uint32_t>(sel_bin);  // key >> 10
+  k -= sel_above;
+  const int listed = list_n;
+  for (int i = tid; i < 1024; i += NT) hist[i] = 0;
+  __syncthreads();
+  const bool use_list = listed <= kListCap;
+  const int m = use_list ? listed : NC;
+  for (int it = 0; it < (m + NT - 1) / NT; ++it) {
+    const int x = it * NT + tid;
+    const uint32_t key = x < m ? (use_list ? list[x] : keys[x]) : 0u;
+    const bool in = x < m && (key >> 10) == pre22;
+    warp_hist_add(hist, in ? static_cast<int>(key & 1023u) : -1, lane);
+  }
+  __syncthreads();
+  find_bin_block<NT>(hist, 1024, k, warp_sums, &sel_bin, &sel_above);
+  __syncthreads();
+  const uint32_t prefix = (pre22 << 10) | static_cast<uint32_t>(sel_bin);
+  k -= sel_above;
+
+  // when no new token is kept (so n == C and nothing moves: the scores are
+  // already updated) the ordered pass below is not needed.  Kept new tokens:
+  // those above T, and of the keys equal to T the first k in candidate order,
+  // where the old slots come first.
+  {
+    const uint32_t T0 = prefix;
+    int gt_new = 0, eq_old = 0, eq_new = 0;
+    for (int x = tid; x < NC; x += NT) {
+      const uint32_t key = keys[x];
+      if (x < n) {
+        eq_old += key == T0;
+      } else {
+        gt_new += key > T0;
+        eq_new += key == T0;
       }
-      const unsigned same = __match_any_sync(0xffffffffu, bin);
-      if (bin >= 0 && (__ffs(same) - 1) == lane) atomicAdd(&my_hist[bin], __popc(same));
     }
-    __syncthreads();
-    if (kSub > 1) {
-      for (int i = tid; i < nb; i += NT) {
-        int t = 0;
-#pragma unroll
-        for (int h = 0; h < kSub; ++h) t += hist[h][i];
-        hist[0][i] = t;
-      }
-      __syncthreads();
+    uint64_t tot;
+    block_excl_scan64<NT>(static_cast<uint64_t>(gt_new) | (static_cast<uint64_t>(eq_old) << 16) |
+                              (static_cast<uint64_t>(eq_new) << 32),
+                          warp_sums, &tot);
+    const int t_gt_new = static_cast<int>(tot & 0xFFFF);
+    const int t_eq_old = static_cast<int>((tot >> 16) & 0xFFFF);
+    const int t_eq_new = static_cast<int>((tot >> 32) & 0xFFFF);
+    const int kept_new = t_gt_new + max(0, min(t_eq_new, k - t_eq_old));
+    if (kept_new == 0 && n == C) {
+      if (tid == 0) e.plan_count[bg] = 0;
+      return;
     }
-    if (warp == 0) find_bin(hist[0], k, lane, &sel_bin, &sel_above);
-    __syncthreads();
-    prefix |= static_cast<uint32_t>(sel_bin) << shift;
-    pmask |= static_cast<uint32_t>(nb - 1) << shift;
-    k -= sel_above;
-    __syncthreads();
   }
   const uint32_t T = prefix;  // C-th largest key; keep the first k keys equal to T
 
@@ -409,18 +532,20 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
     bool kept = key > T;
     if (key == T) kept = eq_rank++ < k;
     if (x < n) {
-      if (!kept) p_slots[fo++] = x;
-    } else if (kept) {
+      if (!kept && H2O_IN_BOUNDS(fo < nq, e.state + 2)) p_slots[fo++] = x;
+    } else if (kept && H2O_IN_BOUNDS(nw < nq, e.state + 2)) {
       p_toks[nw++] = x - n;
     }
   }
   int em = tot_free_old + (e_lo - n);
-  for (int s = e_lo; s < e_hi; ++s) p_slots[em++] = s;
+  for (int s = e_lo; s < e_hi; ++s)
+    if (H2O_IN_BOUNDS(em < nq, e.state + 2)) p_slots[em++] = s;
   __syncthreads();
   // 4. scores and positions of the placed tokens (and the plan, when it was
   //    built in shared memory), then their K/V rows
   for (int q = tid; q < tot_new; q += NT) {
     const int s = p_slots[q], i = p_toks[q];
+    if (!H2O_IN_BOUNDS(s >= 0 && s < C && i >= 0 && i < nq, e.state + 2)) continue;
     score[s] = by_score ? cs[C + i] : 0.f;
     pos[s] = e.t0 + i;
     if (plan_smem) {
@@ -429,7 +554,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
     }
   }
   if (tid == 0) e.plan_count[bg] = tot_new;
-  copy_rows<NT>(e, b, g, tot_new, [p_slots](int q) { return p_slots[q]; },
+  place_rows<NT>(e, b, g, tot_new, [p_slots](int q) { return p_slots[q]; },
                 [p_toks](int q) { return p_toks[q]; });
 }
 
@@ -503,7 +628,7 @@ __global__ void __launch_bounds__(NT, 1) h2o_select_cluster(const EvictParams e)
       pos[n + i] = e.t0 + i;
     }
     if (rank == 0 && tid == 0) e.plan_count[bg] = nq;
-    copy_rows<NT>(e, b, g, i_hi - i_lo, [n, i_lo](int q) { return n + i_lo + q; },
+    place_rows<NT>(e, b, g, i_hi - i_lo, [n, i_lo](int q) { return n + i_lo + q; },
                   [i_lo](int q) { return i_lo + q; });
     return;
   }
@@ -609,13 +734,14 @@ __global__ void __launch_bounds__(NT, 1) h2o_select_cluster(const EvictParams e)
       bool kept = key > T;
       if (key == T) kept = eq_rank++ < k;
       if (x < n) {
-        if (!kept) slots[fo++] = x;
-      } else if (kept) {
+        if (!kept && H2O_IN_BOUNDS(fo < e.plan_ld, e.state + 2)) slots[fo++] = x;
+      } else if (kept && H2O_IN_BOUNDS(nw < e.plan_ld, e.state + 2)) {
         toks[nw++] = x - n;
       }
     }
     int em = tot_free_old + (e_lo - n);
-    for (int s2 = e_lo; s2 < e_hi; ++s2) slots[em++] = s2;
+    for (int s2 = e_lo; s2 < e_hi; ++s2)
+      if (H2O_IN_BOUNDS(em < e.plan_ld, e.state + 2)) slots[em++] = s2;
   }
   cluster_sync_all();  // the plan is complete; no CTA reads another's shared memory after this
   if (bad) {
@@ -630,11 +756,12 @@ __global__ void __launch_bounds__(NT, 1) h2o_select_cluster(const EvictParams e)
   const int q_lo = min(tot_new, rank * qs), q_hi = min(tot_new, q_lo + qs);
   for (int q = q_lo + tid; q < q_hi; q += NT) {
     const int s2 = slots[q], i = toks[q];
+    if (!H2O_IN_BOUNDS(s2 >= 0 && s2 < C && i >= 0 && i < nq, e.state + 2)) continue;
     score[s2] = sx.by_score ? cs[C + i] : 0.f;
     pos[s2] = e.t0 + i;
   }
   if (rank == 0 && tid == 0) e.plan_count[bg] = tot_new;
-  copy_rows<NT>(e, b, g, q_hi - q_lo, [slots, q_lo](int q) { return slots[q_lo + q]; },
+  place_rows<NT>(e, b, g, q_hi - q_lo, [slots, q_lo](int q) { return slots[q_lo + q]; },
                 [toks, q_lo](int q) { return toks[q_lo + q]; });
 }
 

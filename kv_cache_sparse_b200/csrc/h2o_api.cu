@@ -29,6 +29,8 @@ using namespace h2o;
 struct h2o_cache {
   h2o_config cfg;
   h2o_buffers buf;
+  float* k_scale = nullptr;  // int8 cache (Q8): the scales behind the codes of K
+  float* v_scale = nullptr;  // and of V, [batch, H_kv, capacity]
   int n = 0;
   int t0 = 0;
   uint64_t launches = 0;
@@ -83,7 +85,10 @@ struct NvtxRange {
   NvtxRange& operator=(const NvtxRange&) = delete;
 };
 
-size_t esize_of(h2o_dtype t) { return t == H2O_BF16 ? 2 : 4; }
+// bytes per element of q, k_new, v_new and out
+size_t esize_of(h2o_dtype t) { return t == H2O_F32 ? 4 : 2; }
+// bytes per element of the cache's K and V rows (int8 codes for Q8)
+size_t cache_esize(h2o_dtype t) { return t == H2O_F32 ? 4 : (t == H2O_Q8 ? 1 : 2); }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -113,7 +118,7 @@ Layout workspace_layout(const h2o_config& c) {
   L.count = take(BHkv * 4);
   // decode steps (n_q = 1): stored logits and the split-KV partials
   const size_t G = static_cast<size_t>(c.n_q_heads / c.n_kv_heads);
-  L.dpart_ld = cdiv(c.capacity + 1, decode_chunk_keys(c.head_dim, static_cast<int>(esize_of(c.dtype))));
+  L.dpart_ld = cdiv(c.capacity + 1, decode_chunk_keys(c.head_dim, static_cast<int>(cache_esize(c.dtype))));
   L.dslices_ld = cdiv(c.capacity + 1, kDecodeSliceKeys);
   const bool dec = decode_supported(static_cast<int>(G));
   L.dlog = take(dec ? BHkv * G * (static_cast<size_t>(c.capacity) + 1) * 4 : 0);
@@ -133,7 +138,7 @@ Layout workspace_layout(const h2o_config& c) {
 
 h2o_status check_config(const h2o_config* c) {
   if (!c) return H2O_ERR_INVALID_ARG;
-  if (c->dtype != H2O_BF16 && c->dtype != H2O_F32) return H2O_ERR_DTYPE;
+  if (c->dtype != H2O_BF16 && c->dtype != H2O_F32 && c->dtype != H2O_Q8) return H2O_ERR_DTYPE;
   if (c->batch < 1 || c->n_q_heads < 1 || c->n_kv_heads < 1 || c->capacity < 1 ||
       c->max_chunk < 1)
     return H2O_ERR_SHAPE;
@@ -199,6 +204,21 @@ bool encode_cache(CUtensorMap* tm, const void* base, int BH, int n, int C, int d
   return encode_bf16(tm, base, 3, dims, strides, box);
 }
 
+// int8 codes of the Q8 cache [B*Hkv, C, d], the first n rows visible: dims
+// (d, n, B*Hkv), box (d, 128, 1), no swizzle (the kernels dequantise the tile
+// into their 128-byte-swizzled bf16 operand)
+bool encode_cache_q8(CUtensorMap* tm, const void* base, int BH, int n, int C, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)(n > 0 ? n : 1), (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)C * d};
+  const cuuint32_t box[3] = {(cuuint32_t)d, 128, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 h2o_status cuda_status(cudaError_t e) { return e == cudaSuccess ? H2O_OK : H2O_ERR_CUDA; }
 
 // Records timing event i (0: before K1, i: after kernel i) when timing is on.
@@ -220,7 +240,7 @@ h2o_status check_step_args(h2o_cache* c, const void* q, const void* kn, const vo
 
 AttnParams attn_params(h2o_cache* c, int nq, void* out) {
   const h2o_config& g = c->cfg;
-  AttnParams p;
+  AttnParams p{};
   p.B = g.batch;
   p.Hq = g.n_q_heads;
   p.Hkv = g.n_kv_heads;
@@ -236,6 +256,8 @@ AttnParams attn_params(h2o_cache* c, int nq, void* out) {
   p.colsum = c->colsum;
   p.colsum_ld = c->colsum_ld;
   p.err = c->buf.state + 2;
+  p.k_scale = c->k_scale;
+  p.v_scale = c->v_scale;
   return p;
 }
 
@@ -262,11 +284,13 @@ h2o_status run_attention(h2o_cache* c, const void* q, const void* kn, const void
   }
   AttnMaps m;
   const int BH = g.batch * g.n_kv_heads;
+  const bool q8 = g.dtype == H2O_Q8;
+  auto enc = q8 ? encode_cache_q8 : encode_cache;
   if (!encode_chunk(&m.q, q, g.batch, nq, g.n_q_heads, g.head_dim) ||
       !encode_chunk(&m.kn, kn, g.batch, nq, g.n_kv_heads, g.head_dim) ||
       !encode_chunk(&m.vn, vn, g.batch, nq, g.n_kv_heads, g.head_dim) ||
-      !encode_cache(&m.kc, c->buf.k, BH, c->n, g.capacity, g.head_dim) ||
-      !encode_cache(&m.vc, c->buf.v, BH, c->n, g.capacity, g.head_dim))
+      !enc(&m.kc, c->buf.k, BH, c->n, g.capacity, g.head_dim) ||
+      !enc(&m.vc, c->buf.v, BH, c->n, g.capacity, g.head_dim))
     return H2O_ERR_CUDA;
   cudaError_t e;
   {
@@ -293,12 +317,12 @@ h2o_status run_attention(h2o_cache* c, const void* q, const void* kn, const void
 h2o_status run_evict(h2o_cache* c, const float* colsum, int ld, const void* kn, const void* vn,
                      int nq, cudaStream_t st) {
   const h2o_config& g = c->cfg;
-  EvictParams e;
+  EvictParams e{};
   e.B = g.batch;
   e.Hkv = g.n_kv_heads;
   e.C = g.capacity;
   e.d = g.head_dim;
-  e.esize = static_cast<int>(esize_of(g.dtype));
+  e.esize = static_cast<int>(cache_esize(g.dtype));
   e.n = c->n;
   e.t0 = c->t0;
   e.nq = nq;
@@ -318,6 +342,9 @@ h2o_status run_evict(h2o_cache* c, const float* colsum, int ld, const void* kn, 
   e.state = c->buf.state;
   e.policy = g.policy;
   e.sinks = g.sink_tokens;
+  e.q8 = g.dtype == H2O_Q8 ? 1 : 0;
+  e.k_scale = c->k_scale;
+  e.v_scale = c->v_scale;
   if (!c->ev_used[2]) {  // eviction on its own: time it from here
     for (int i = 0; i < 5; ++i) c->ev_used[i] = false;
     mark(c, 2, st);
@@ -346,7 +373,7 @@ bool decode_path(const h2o_cache* c, int nq) {
 h2o_status run_decode(h2o_cache* c, const void* q, const void* kn, const void* vn, void* out,
                       bool evict, cudaStream_t st) {
   const h2o_config& g = c->cfg;
-  DecodeParams d;
+  DecodeParams d{};
   d.B = g.batch;
   d.Hkv = g.n_kv_heads;
   d.G = g.n_q_heads / g.n_kv_heads;
@@ -354,7 +381,7 @@ h2o_status run_decode(h2o_cache* c, const void* q, const void* kn, const void* v
   d.n = c->n;
   d.t0 = c->t0;
   d.W = g.recent_window;
-  d.n_chunks = cdiv(c->n + 1, decode_chunk_keys(g.head_dim, static_cast<int>(esize_of(g.dtype))));
+  d.n_chunks = cdiv(c->n + 1, decode_chunk_keys(g.head_dim, static_cast<int>(cache_esize(g.dtype))));
   d.part_ld = c->dec_part_ld;
   d.n_slices = cdiv(c->n + 1, kDecodeSliceKeys);
   d.slices_ld = c->dec_slices_ld;
@@ -384,11 +411,13 @@ h2o_status run_decode(h2o_cache* c, const void* q, const void* kn, const void* v
   d.evict = evict ? 1 : 0;
   d.policy = g.policy;
   d.sinks = g.sink_tokens;
+  d.k_scale = c->k_scale;
+  d.v_scale = c->v_scale;
   for (int i = 0; i < 5; ++i) c->ev_used[i] = false;
   mark(c, 0, st);
   {
     NvtxRange r("h2o decode step (split-KV attention, merge, eviction)");
-    if (launch_decode(d, static_cast<int>(esize_of(g.dtype)), g.head_dim, st) != cudaSuccess)
+    if (launch_decode(d, static_cast<int>(cache_esize(g.dtype)), g.head_dim, st) != cudaSuccess)
       return H2O_ERR_CUDA;
   }
   c->fwd_nq = 0;  // the decode path keeps no row statistics
@@ -453,7 +482,9 @@ h2o_status h2o_required_bytes(const h2o_config* cfg, h2o_sizes* out) {
   if (s != H2O_OK) return s;
   if (!out) return H2O_ERR_INVALID_ARG;
   const size_t slots = static_cast<size_t>(cfg->batch) * cfg->n_kv_heads * cfg->capacity;
-  out->k_bytes = slots * cfg->head_dim * esize_of(cfg->dtype);
+  // int8 cache: the codes, then one fp32 scale per row
+  out->k_bytes = slots * cfg->head_dim * cache_esize(cfg->dtype) +
+                 (cfg->dtype == H2O_Q8 ? slots * sizeof(float) : 0);
   out->v_bytes = out->k_bytes;
   out->scores_bytes = slots * 4;
   out->pos_bytes = slots * 4;
@@ -474,11 +505,17 @@ h2o_status h2o_cache_create(const h2o_config* cfg, const h2o_buffers* bufs, void
     return H2O_ERR_ALIGN;
   const Layout L = workspace_layout(*cfg);
   if (bufs->workspace_bytes < L.total) return H2O_ERR_SHAPE;
-  if (cfg->dtype == H2O_BF16 && !encode_fn()) return H2O_ERR_CUDA;
+  if (cfg->dtype != H2O_F32 && !encode_fn()) return H2O_ERR_CUDA;
   h2o_cache* c = new (std::nothrow) h2o_cache();
   if (!c) return H2O_ERR_INVALID_ARG;
   c->cfg = *cfg;
   c->buf = *bufs;
+  if (cfg->dtype == H2O_Q8) {
+    const size_t codes = static_cast<size_t>(cfg->batch) * cfg->n_kv_heads * cfg->capacity *
+                         cfg->head_dim;
+    c->k_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(bufs->k) + codes);
+    c->v_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(bufs->v) + codes);
+  }
   uint8_t* ws = static_cast<uint8_t*>(bufs->workspace);
   c->nq_pad = L.nq_pad;
   c->colsum_ld = L.colsum_ld;
@@ -549,7 +586,7 @@ h2o_status h2o_attention_backward(h2o_cache* c, const void* q, const void* k_new
     return H2O_ERR_ALIGN;
   // the row statistics must be those of h2o_attention on this state and n_q
   if (c->fwd_nq != n_q || c->fwd_n != c->n) return H2O_ERR_STATE;
-  BwdParams p;
+  BwdParams p{};
   p.B = g.batch;
   p.Hq = g.n_q_heads;
   p.Hkv = g.n_kv_heads;
@@ -717,7 +754,7 @@ h2o_status h2o_cache_check(h2o_cache* c, void* stream) {
   if (cudaMemcpy(&word, c->buf.state + 2, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
     return H2O_ERR_CUDA;
   if (word & kDevErrTimeout) return H2O_ERR_TIMEOUT;
-  if (word & (kDevErrPlan | kDevErrSmem)) return H2O_ERR_STATE;
+  if (word & (kDevErrPlan | kDevErrSmem | kDevErrBounds)) return H2O_ERR_STATE;
   return H2O_OK;
 }
 

@@ -146,7 +146,7 @@ extern "C" H2O_API h2o_status h2o_attention_static_scratch(
   // this call's kernels latch a timeout into a clean word
   if (cudaMemsetAsync(err, 0, sizeof(int), st) != cudaSuccess) return H2O_ERR_CUDA;
 
-  AttnParams p;
+  AttnParams p{};
   p.B = g.batch;
   p.Hq = g.n_q_heads;
   p.Hkv = g.n_kv_heads;
@@ -162,6 +162,8 @@ extern "C" H2O_API h2o_status h2o_attention_static_scratch(
   p.colsum = colsum_out;  // written in place: [batch, H_kv, capacity + n_q]
   p.colsum_ld = g.capacity + n_q;
   p.err = err;
+  p.k_scale = nullptr;  // bf16 / fp32 cache (this entry point takes no int8 cache)
+  p.v_scale = nullptr;
 
   if (g.dtype == H2O_F32) {
     cudaError_t e = launch_attn_f32(g.head_dim, static_cast<const float*>(q),

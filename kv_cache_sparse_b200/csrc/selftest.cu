@@ -2,7 +2,9 @@
 // waits, with the kernels' bounded wait, on an mbarrier nothing arrives at;
 // the wait gives up after the given limit, latches the timeout bit and the
 // kernel returns (no trap, no hang).  Without a word of the caller's, the bit
-// goes to the word h2o_static_scratch_check reports.
+// goes to the word h2o_static_scratch_check reports.  h2o_selftest_exp2
+// evaluates the kernels' FMA-pipe exp2 (exp2_fma2) on given inputs, so that
+// it can be checked against the library exp2f.
 #include "../../include/h2o.h"
 #include "attn.h"
 #include "sm100.cuh"
@@ -23,7 +25,26 @@ __global__ void wait_timeout_probe(int* err, uint64_t limit_ns) {
   h2o::mbar_wait_until(b, 0, err, &abort_flag, limit_ns);
 }
 
+__global__ void exp2_fma_probe(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float a = x[i], b = i + 1 < n ? x[i + 1] : 0.f;
+  float ya, yb;
+  h2o::exp2_fma2(ya, yb, a, b);
+  y[i] = ya;
+  if (i + 1 < n) y[i + 1] = yb;
+}
+
 }  // namespace
+
+extern "C" H2O_API h2o_status h2o_selftest_exp2(const float* x, float* y, int32_t n,
+                                                void* stream) {
+  if (!x || !y || n < 0) return H2O_ERR_INVALID_ARG;
+  if (n == 0) return H2O_OK;
+  const int pairs = (n + 1) / 2;
+  exp2_fma_probe<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? H2O_OK : H2O_ERR_CUDA;
+}
 
 extern "C" H2O_API h2o_status h2o_selftest_wait_timeout(int32_t* err_word, uint32_t limit_us,
                                                         void* stream) {

@@ -188,10 +188,39 @@ __device__ __forceinline__ void griddep_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- register budgets
+
+// Changes the registers per thread of the calling warpgroup (all four warps
+// execute it): the released registers go to warpgroups that raise theirs.
+template <uint32_t N>
+__device__ __forceinline__ void warpgroup_reg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void warpgroup_reg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- named barriers
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier over nthreads threads that also ANDs a predicate across them:
+// every participant gets the same result.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // ---------------------------------------------------------------- tcgen05
@@ -280,6 +309,36 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+// Each thread of the warp reads 16 consecutive 32-bit columns of its lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// Each thread of the warp writes 16 (8) consecutive 32-bit columns of its lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -341,6 +400,55 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
       "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// (a0, a1) + (b0, b1) rounded toward minus infinity, and (a0, a1) - (b0, b1).
+__device__ __forceinline__ void fadd2_rm(float& d0, float& d1, float a0, float a1, float b0,
+                                         float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rm.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+__device__ __forceinline__ void fsub2(float& d0, float& d1, float a0, float a1, float b0,
+                                      float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// 2^x for two values on the FMA pipe instead of the special function unit,
+// for kernels whose exponentials would otherwise saturate it.  Cody and
+// Waite's range reduction: x = j + f with j = floor(x) and f in [0, 1);
+// 2^f from the degree-3 polynomial that minimises the largest relative error
+// on [0, 1] (Remez exchange; coefficients from exp2_poly.py; relative error
+// below 7.5e-5); j added to the exponent field.  j comes from the low
+// mantissa bits of x + 1.5 * 2^23 rounded down, and (bits << 23) adds it to
+// the exponent modulo 2^9, so x is clamped to >= -125 (about 2^-125, not 0,
+// for smaller x, -inf included: the callers' sums treat such terms as 0; the
+// clamp also keeps the result normal, since p(0) is a little below 1).
+constexpr float kExp2C0 = 0.99992521856271555f;
+constexpr float kExp2C1 = 0.69583354049475288f;
+constexpr float kExp2C2 = 0.22606715542748335f;
+constexpr float kExp2C3 = 0.078024522640479307f;
+
+__device__ __forceinline__ void exp2_fma2(float& y0, float& y1, float x0, float x1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  float t0, t1, j0, j1, f0, f1, p0, p1;
+  fadd2_rm(t0, t1, x0, x1, kMagic, kMagic);  // kMagic + floor(x)
+  fsub2(j0, j1, t0, t1, kMagic, kMagic);     // floor(x), exact
+  fsub2(f0, f1, x0, x1, j0, j1);             // f in [0, 1)
+  ffma2(p0, p1, f0, f1, kExp2C3, kExp2C3, kExp2C2, kExp2C2);
+  ffma2(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
+  ffma2(p0, p1, p0, p1, f0, f1, kExp2C0, kExp2C0);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // Three-input maximum (one instruction on sm_100).

@@ -45,7 +45,7 @@ class Workload:
     capacity: int
     window: int
     seq_len: int
-    dtype: str                      # "bf16" or "f32"
+    dtype: str                      # "bf16", "f32" or "q8" (int8 cache, bf16 activations)
     heavy_p: float = 0.02           # probability that a position is heavy
     heavy_p_range: Optional[Tuple[float, float]] = None  # per-chunk U[lo, hi]
     drift_step: float = 0.0         # norm of the per-token mean step of K
@@ -72,7 +72,13 @@ class Workload:
         return self.n_q_heads // self.n_kv_heads
 
     def torch_dtype(self) -> torch.dtype:
-        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+        """Element type of q, k_new, v_new and out."""
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def cache_dtype(self) -> torch.dtype:
+        """The cache's element type as the binding names it (torch.int8: the
+        int8 cache with per-row scales)."""
+        return torch.int8 if self.dtype == "q8" else self.torch_dtype()
 
     def scaled(self, **changes) -> "Workload":
         """A copy with some fields replaced (used for scaled-down tests)."""
@@ -117,10 +123,16 @@ LR_C8K = dataclasses.replace(QWEN_C8K, name="qwen3_4b_lr_c8192_q1024_w256", poli
 SLR_C8K = dataclasses.replace(QWEN_C8K, name="qwen3_4b_slr4_c8192_q1024_w256", policy="slr",
                               sinks=4)
 
+# The headline cache quantised (Q-Hitter: H2O with an int8 cache, summary
+# page Table 5's qh2o rows), and its decode step.
+QH2O_C8K = dataclasses.replace(QWEN_C8K, name="qwen3_4b_qh2o_c8192_q1024_w256", dtype="q8")
+QH2O_DECODE_C8K = dataclasses.replace(DECODE_C8K, name="qwen3_4b_qh2o_decode_c8192_w256",
+                                      dtype="q8")
+
 WORKLOADS = {w.name: w for w in (TINY, QWEN_C8K, QWEN_C16K, STACK36, STREAM1M, DECODE_C8K,
-                                 DECODE_STACK36, LR_C8K, SLR_C8K)}
+                                 DECODE_STACK36, LR_C8K, SLR_C8K, QH2O_C8K, QH2O_DECODE_C8K)}
 ORDERED = [TINY, QWEN_C8K, QWEN_C16K, STACK36, STREAM1M, DECODE_C8K, DECODE_STACK36, LR_C8K,
-           SLR_C8K]
+           SLR_C8K, QH2O_C8K, QH2O_DECODE_C8K]
 
 
 def _seed64(*words: int) -> int:

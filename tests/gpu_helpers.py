@@ -37,7 +37,8 @@ def shape_of(B, Hq, Hkv, d, C, max_chunk, W, dtype=torch.bfloat16, scale=0.0):
 def oracle_for(shape: binding.CacheShape) -> orc.OracleCache:
     scale = shape.softmax_scale if shape.softmax_scale > 0 else None
     return orc.OracleCache(shape.batch, shape.n_q_heads, shape.n_kv_heads, shape.head_dim,
-                           shape.capacity, shape.recent_window, scale=scale)
+                           shape.capacity, shape.recent_window, scale=scale,
+                           kv_format="q8" if shape.q8 else "bf16")
 
 
 def push_oracle_state(gpu: binding.H2OCache, ref: orc.OracleCache):
@@ -52,8 +53,39 @@ def pull_state(gpu: binding.H2OCache):
 
 
 def load_oracle_from_gpu(ref: orc.OracleCache, st):
+    if ref.kv_format == "q8":
+        ref.load_q8(st["k"].cpu().numpy(), st["k_scale"].cpu().numpy(), st["v"].cpu().numpy(),
+                    st["v_scale"].cpu().numpy(), st["scores"].cpu().numpy(),
+                    st["pos"].cpu().numpy(), st["n"], st["t0"])
+        return
     ref.load(np64(st["k"]), np64(st["v"]), st["scores"].cpu().numpy(),
              st["pos"].cpu().numpy(), st["n"], st["t0"])
+
+
+def random_state_q8(shape, n, t0, rng, score_levels=None):
+    """A plausible int8-cache state: codes and row scales of n valid slots
+    (the quantised form of N(0,1) rows), scores and distinct positions."""
+    K, V, sc, pos = random_state(shape.__class__(**{**shape.__dict__, "dtype": torch.bfloat16}),
+                                 n, t0, rng, score_levels)
+    B, Hkv, C, d = shape.batch, shape.n_kv_heads, shape.capacity, shape.head_dim
+    out = []
+    for X in (K, V):
+        codes = np.zeros((B, Hkv, C, d), np.int8)
+        scales = np.zeros((B, Hkv, C), np.float32)
+        x = X.float().numpy()
+        for b in range(B):
+            for g in range(Hkv):
+                for s_ in range(n):
+                    codes[b, g, s_], scales[b, g, s_] = orc.quantize_row_q8(x[b, g, s_])
+        out += [codes, scales]
+    return out[0], out[1], out[2], out[3], sc, pos
+
+
+def install_state_q8(gpu, ref, Kq, Ks, Vq, Vs, sc, pos, n, t0):
+    gpu.write(torch.from_numpy(Kq), torch.from_numpy(Vq), torch.from_numpy(sc),
+              torch.from_numpy(pos), n, t0, k_scale=torch.from_numpy(Ks),
+              v_scale=torch.from_numpy(Vs))
+    ref.load_q8(Kq, Ks, Vq, Vs, sc, pos, n, t0)
 
 
 def random_state(shape, n, t0, rng, score_levels=None):
@@ -109,6 +141,14 @@ def assert_state_equal(st, ref: orc.OracleCache, dtype, what=""):
     assert np.array_equal(st["pos"].cpu().numpy(), ref.pos), f"{what}: positions differ"
     assert np.array_equal(st["scores"].cpu().numpy().view(np.uint32),
                           ref.scores.astype(np.float32).view(np.uint32)), f"{what}: scores differ"
+    if ref.kv_format == "q8":
+        assert np.array_equal(st["k"].cpu().numpy(), ref.Kq), f"{what}: K codes differ"
+        assert np.array_equal(st["v"].cpu().numpy(), ref.Vq), f"{what}: V codes differ"
+        assert np.array_equal(st["k_scale"].cpu().numpy().view(np.uint32),
+                              ref.Ks.view(np.uint32)), f"{what}: K scales differ"
+        assert np.array_equal(st["v_scale"].cpu().numpy().view(np.uint32),
+                              ref.Vs.view(np.uint32)), f"{what}: V scales differ"
+        return
     kref = torch.from_numpy(ref.K).to(dtype)
     vref = torch.from_numpy(ref.V).to(dtype)
     assert torch.equal(bits(st["k"]), bits(kref)), f"{what}: cache K differs"
