@@ -47,6 +47,8 @@ cudaError_t launch_attn_f32(int head_dim, const float* q, const float* kc, const
 cudaError_t launch_decode(const DecodeParams& p, int esize, int head_dim, cudaStream_t st);
 // Group sizes the decode kernels take (a warp batch holds 32 / G keys).
 bool decode_supported(int G);
+// Kernel launches per decode step (1: the merge runs in each unit's last CTA).
+int decode_launches();
 
 // Backward of the attention (bf16, head_dim 64 or 128): D_i, then dK/dV and
 // dQ; out and dout are [B, nq, Hq, d] bf16.

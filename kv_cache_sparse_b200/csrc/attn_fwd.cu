@@ -19,7 +19,8 @@
 //                 S_X(t) = Q_X K(t)^T  into TMEM columns [128X, 128X+128)
 //                 O_X   += P_X(t) V(t) into TMEM columns 256 + 128X, with
 //                 P_X(t) read from TMEM (bf16, written over S_X(t))
-//   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B: one thread
+//   warps 2..3  int8 cache only: dequantisation (below); otherwise idle
+//   warps 4..7  softmax of tile A, warps 8..11 softmax of tile B: one thread
 //               per query row (TMEM lane) reads its 128 logits once, takes
 //               the row max, then P = 2^(x - m) (packed f32x2 arithmetic for
 //               the scaling and the row sum) as bf16 back into TMEM; lazy
@@ -30,7 +31,7 @@
 // softmax that sees S_X(t+1) may rescale O_X and overwrite P_X.
 //
 // The int8 cache (Q8, q8.cuh): warp 0 brings a cache tile's codes of K and of
-// V into one staging buffer each (TMA, no swizzle), and warps 10 and 11
+// V into one staging buffer each (TMA, no swizzle), and warps 2 and 3
 // dequantise them into the same bf16 rings the MMA reads (128-byte swizzle),
 // with the row scales; the chunk's own tiles still arrive in bf16 by TMA.
 #include <cuda_bf16.h>
@@ -40,6 +41,16 @@
 #include "sm100.cuh"
 
 namespace h2o {
+
+// Pairs of keys (of every 8) whose exponentials run on the FMA pipe
+// (exp2_fma2) rather than the special function unit (16 per clock per SM).
+// Measured on the headline cache: 0 of 8 157.7 us, 2 of 8 172.7 us, 3 of 8
+// 179.2 us -- the tile's softmax chain is bound by latency, not by the
+// unit's throughput, and the extra instructions lengthen it.
+constexpr int kFwdEmuPairsOf8 = 0;
+// Softmax warps spin on the S barrier instead of suspending (a suspended
+// warp wakes up later, on the critical chain of its tile).
+constexpr bool kFwdSpinS = false;
 
 template <int D, bool Q8 = false>
 struct FwdLayout {
@@ -360,7 +371,8 @@ __global__ void __launch_bounds__(FwdLayout<D, Q8>::kThreads, 1)
     float l = 0.f;
     bool ok = true;
     for (int t = 0; t < T; ++t) {
-      ok = mbar_wait(bar_s_full0 + 8 * x, t & 1, p.err, abort_flag);
+      ok = kFwdSpinS ? mbar_wait_spin(bar_s_full0 + 8 * x, t & 1, p.err, abort_flag)
+                     : mbar_wait(bar_s_full0 + 8 * x, t & 1, p.err, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -422,7 +434,17 @@ __global__ void __launch_bounds__(FwdLayout<D, Q8>::kThreads, 1)
           float x0, x1;
           ffma2(x0, x1, __uint_as_float(v[64 * hh + j]), __uint_as_float(v[64 * hh + j + 1]), c, c,
                 nm, nm);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          float p0, p1;
+          if (((j >> 1) & 7) < kFwdEmuPairsOf8) {
+            exp2_fma2(p0, p1, x0, x1);
+            if (masked) {  // the FMA-pipe exp2 floors at 2^-125: masked keys read 0
+              p0 = (64 * hh + j < lim) ? p0 : 0.f;
+              p1 = (64 * hh + j + 1 < lim) ? p1 : 0.f;
+            }
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
           const int a = (j >> 1) & 1;
           fadd2(ls[2 * a], ls[2 * a + 1], ls[2 * a], ls[2 * a + 1], p0, p1);
           pk[j >> 1] = pack_bf16x2(p0, p1);

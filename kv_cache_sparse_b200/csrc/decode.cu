@@ -20,8 +20,16 @@
 //                   product of pair l.  The logits are stored for the summed
 //                   weights; one warp per head takes the chunk's max and sum;
 //                   P V is accumulated per lane over the head-dim slice, the
-//                   eight warps' partial sums added in a fixed order.
-//   decode_finish   grid (cdiv(n + 1, 1024), B*Hkv), 256 threads, programmatic
+//                   eight warps' partial sums (over the K rows, which are no
+//                   longer needed) added in a fixed order.  Then an atomic
+//                   ticket per (cache, KV head) elects the last CTA to
+//                   finish, which merges the unit (merge_unit): per-head
+//                   lse2 over the chunks, O, the summed weights of all n + 1
+//                   keys with the score update and the eviction candidate on
+//                   the way, and the new token's placement.  One launch per
+//                   step.
+//   decode_finish   (the two-launch form, kDecodeFused = false) grid
+//                   (cdiv(n + 1, 1024), B*Hkv), 256 threads, programmatic
 //                   dependent launch.  Every CTA merges the chunk statistics
 //                   of each head (lse2) and a share of the outputs O.  Each CTA
 //                   writes the summed weights colsum[j] = sum_h 2^(x_hj -
@@ -135,16 +143,187 @@ struct PartialLayout {
   static constexpr int kCode = Q8 ? 1 : static_cast<int>(sizeof(T));  // bytes per cache element
   static constexpr int KC = decode_chunk_keys(D, kCode);
   static constexpr int kRow = D * kCode;
-  static constexpr int kK = 0;                          // [KC][D] cache rows of K
+  static constexpr int kK = 0;                          // [KC][D] cache rows of K; after the
+                                                        // logits: [warps][G][D] float sums of P V
   static constexpr int kV = kK + KC * kRow;             // [KC][D] of V
   static constexpr int kX = kV + KC * kRow;             // [G][KC] float: logits, then P
-  static constexpr int kO = kX + G * KC * 4;            // [warps][G][D] float
-  static constexpr int kS = kO + kWarps * G * D * 4;    // Q8: [2][KC] float scales of K, V
+  static constexpr int kS = kX + G * KC * 4;            // Q8: [2][KC] float scales of K, V
   static constexpr int kN = kS + (Q8 ? 2 * KC * 4 : 0);  // Q8: the new token's K, V rows (T)
   static constexpr int kBytes = kN + (Q8 ? 2 * D * static_cast<int>(sizeof(T)) : 0);
+  static_assert(kWarps * G * D * 4 <= KC * kRow, "the P V sums must fit over the K rows");
+  // the merge (last CTA of a unit) reuses the K and V rows for [G][chunks] factors
+  static constexpr int kMaxChunksL = (kMaxCandidates + 1 + KC - 1) / KC;
+  static_assert(G * kMaxChunksL * 4 <= kX, "merge factors must fit over the K and V rows");
 };
 
+// The merge of one (cache, KV head) unit by one CTA, once every split-KV
+// partial and logit of the unit is written: per-head log-sum-exp over the
+// chunks, O, the summed weights of the n + 1 keys and, when evicting, the
+// score update, the eviction candidate (the lowest rank value, the highest
+// index among equals) and the new token's placement.  fac: [G][n_chunks]
+// shared floats.  Data the other CTAs wrote is read through L2 (__ldcg).
 template <typename T, int D, int G, bool Q8>
+__device__ __forceinline__ void merge_unit(const DecodeParams& p, int bg, float* fac) {
+  __shared__ float lse[G], lh[G];
+  __shared__ unsigned long long wmin[kWarps];
+  __shared__ float s_new;  // the new token's summed weight
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int NCk = p.n_chunks, C = p.C, n = p.n;
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  constexpr size_t kChunkStride = static_cast<size_t>(G) * (D + 2);
+  const float* part = p.part + static_cast<size_t>(bg) * p.part_ld * kChunkStride;
+
+  // ---- per-head log-sum-exp over the chunks (one warp per head)
+  if (warp < G) {
+    float m = -INFINITY;
+    for (int c = lane; c < NCk; c += 32) m = fmaxf(m, __ldcg(part + c * kChunkStride + warp * (D + 2) + D));
+    m = warp_max(m);
+    float l = 0.f;
+    for (int c = lane; c < NCk; c += 32) {
+      const float* st = part + c * kChunkStride + warp * (D + 2) + D;
+      const float f = ex2_approx(__ldcg(st) - m);
+      fac[warp * NCk + c] = f;
+      l = fmaf(__ldcg(st + 1), f, l);
+    }
+    l = warp_sum(l);
+    if (lane == 0) {
+      lh[warp] = l;
+      lse[warp] = m + __log2f(l);
+    }
+  }
+  __syncthreads();
+
+  // ---- O: thread t merges outputs t, t + 256, ... over the chunks
+  {
+    T* out = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.Hkv * G + g * G) * D;
+    for (int i = tid; i < G * D; i += kThreads) {
+      const int h = i / D, d = i % D;
+      const float* src = part + h * (D + 2) + d;
+      const float* fh = fac + h * NCk;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int c = 0; c < NCk; ++c) acc = fmaf(__ldcg(src + c * kChunkStride), fh[c], acc);
+      store(out + i, acc / lh[h]);
+    }
+  }
+
+  // ---- summed weights of the n + 1 keys, with the score update and this
+  //      thread's eviction candidate on the way
+  const float* lg = p.logits + static_cast<size_t>(bg) * G * (C + 1);
+  float* cs = p.colsum + static_cast<size_t>(bg) * p.colsum_ld;
+  float* score = p.scores + static_cast<size_t>(bg) * C;
+  int* pos = p.pos + static_cast<size_t>(bg) * C;
+  const bool by_score = p.policy == kPolicyH2O;
+  const int sinks = p.policy == kPolicySLR ? p.sinks : 0;
+  const bool full = p.evict && n >= C;
+  // unprotected: position < t0 + 1 - W (and, under SLR, >= the sink count).
+  // Candidate key: rank value (the score as an order-preserving key, or the
+  // position) then the inverted index, so that the minimum is the lowest
+  // value with the highest index.
+  const long long limit = static_cast<long long>(p.t0) + 1 - p.W;
+  float lse_r[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) lse_r[h] = lse[h];
+  unsigned long long best = ~0ull;
+#pragma unroll 4
+  for (int j = tid; j <= n; j += kThreads) {
+    float x[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) x[h] = __ldcg(lg + static_cast<size_t>(h) * (C + 1) + j);
+    float sw = 0.f;
+#pragma unroll
+    for (int h = 0; h < G; ++h) sw += ex2_approx(x[h] - lse_r[h]);
+    if (j == n) {
+      cs[C] = sw;
+      s_new = sw;
+      continue;
+    }
+    cs[j] = sw;
+    if (!p.evict) continue;
+    if (!full) {
+      if (by_score) score[j] = __fadd_rn(score[j], sw);
+      continue;
+    }
+    const int ps = pos[j];
+    uint32_t rank;
+    if (by_score) {
+      const float sc = __fadd_rn(score[j], sw);
+      score[j] = sc;
+      rank = ordered_key(sc);
+    } else {
+      rank = static_cast<uint32_t>(ps);
+    }
+    if (ps < limit && ps >= sinks) {
+      const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - j);
+      best = key < best ? key : best;
+    }
+  }
+  for (int j = n + tid; j < C; j += kThreads) cs[j] = 0.f;  // empty slots received nothing
+  __syncthreads();  // s_new
+  if (!p.evict) return;
+
+  // ---- eviction
+  const size_t row_bytes = static_cast<size_t>(D) * (Q8 ? 1 : sizeof(T));  // cache rows
+  const size_t new_bytes = static_cast<size_t>(D) * sizeof(T);
+  char* kc = static_cast<char*>(p.k_cache) + static_cast<size_t>(bg) * C * row_bytes;
+  char* vc = static_cast<char*>(p.v_cache) + static_cast<size_t>(bg) * C * row_bytes;
+  const char* kn = static_cast<const char*>(p.k_new) + static_cast<size_t>(bg) * new_bytes;
+  const char* vn = static_cast<const char*>(p.v_new) + static_cast<size_t>(bg) * new_bytes;
+  // the new token's rows into slot `slot`: copied, or quantised (Q8); one warp
+  auto place_new = [&](int slot) {
+    if (!H2O_IN_BOUNDS(slot >= 0 && slot < C, p.state + 2)) return;
+    if (Q8) {
+      q8_quantize_row_warp<D>(reinterpret_cast<const __nv_bfloat16*>(kn),
+                              reinterpret_cast<int8_t*>(kc + static_cast<size_t>(slot) * row_bytes),
+                              p.k_scale + static_cast<size_t>(bg) * C + slot, lane);
+      q8_quantize_row_warp<D>(reinterpret_cast<const __nv_bfloat16*>(vn),
+                              reinterpret_cast<int8_t*>(vc + static_cast<size_t>(slot) * row_bytes),
+                              p.v_scale + static_cast<size_t>(bg) * C + slot, lane);
+    } else {
+      copy_row(kc + static_cast<size_t>(slot) * row_bytes, kn, static_cast<int>(row_bytes), lane);
+      copy_row(vc + static_cast<size_t>(slot) * row_bytes, vn, static_cast<int>(row_bytes), lane);
+    }
+  };
+  if (bg == 0 && tid == 0) {
+    p.state[0] = min(C, n + 1);
+    p.state[1] = p.t0 + 1;
+  }
+  if (!full) {  // room left: the new token takes slot n
+    if (tid == 0) {
+      score[n] = by_score ? s_new : 0.f;
+      pos[n] = p.t0;
+    }
+    if (warp == 0) place_new(n);
+    return;
+  }
+  if (tid == 0 && p.t0 < limit && p.t0 >= sinks) {  // W = 0: the new token competes
+    const uint32_t rank = by_score ? ordered_key(s_new) : static_cast<uint32_t>(p.t0);
+    const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - C);
+    best = key < best ? key : best;
+  }
+  best = warp_min64(best);
+  if (lane == 0) wmin[warp] = best;
+  __syncthreads();  // also: every slot's score is updated before one is replaced
+  if (warp != 0) return;
+  unsigned long long m = lane < kWarps ? wmin[lane] : ~0ull;
+  m = warp_min64(m);
+  if (m == ~0ull) {  // cannot happen: W + sinks <= C leaves an unprotected candidate
+    if (lane == 0) atomicOr(&p.state[2], kDevErrPlan);
+    return;
+  }
+  const int e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(m & 0xffffffffu));
+  if (e < C) {  // an old slot leaves; the new token takes it
+    if (lane == 0) {
+      score[e] = by_score ? s_new : 0.f;
+      pos[e] = p.t0;
+    }
+    place_new(e);
+  }
+}
+
+// kFused: the last CTA of each (cache, KV head) also merges it (merge_unit),
+// so that the step is one launch; otherwise decode_finish follows.
+template <typename T, int D, int G, bool Q8, bool kFused>
 __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p) {
   using L = PartialLayout<T, D, G, Q8>;
   constexpr int KC = L::KC;
@@ -154,7 +333,7 @@ __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p)
   uint8_t* sK = dsm + L::kK;
   uint8_t* sV = dsm + L::kV;
   float* xs = reinterpret_cast<float*>(dsm + L::kX);
-  float* ored = reinterpret_cast<float*>(dsm + L::kO);
+  float* ored = reinterpret_cast<float*>(dsm + L::kK);  // written once the K rows are used
   __shared__ __align__(8) uint64_t bars[2];
   __shared__ int abort_flag;
   __shared__ float hstat[G][2];  // chunk max, chunk sum
@@ -299,6 +478,11 @@ __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p)
       }
     }
   }
+  if (!ok && tid == 0 && rows > 0) {  // a wait gave up: the copies land before their
+    mbar_wait_drain(bK, 0, err);      // buffers are written or the CTA exits
+    mbar_wait_drain(bV, 0, err);
+  }
+  __syncthreads();  // every warp is done with the K rows
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
@@ -316,10 +500,18 @@ __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p)
       part[tid * (D + 2) + D] = hstat[tid][0];
       part[tid * (D + 2) + D + 1] = hstat[tid][1];
     }
-  } else if (tid == 0 && rows > 0) {  // a wait gave up: let the copies land before exit
-    mbar_wait_drain(bK, 0, err);
-    mbar_wait_drain(bV, 0, err);
   }
+  if (!kFused) return;
+  // ---- the last CTA of this (cache, KV head) to get here merges the unit
+  __shared__ int is_last;
+  __threadfence();  // this CTA's logits and partials, before the ticket
+  __syncthreads();
+  if (tid == 0) is_last = atomicAdd(&p.ticket[bg], 1) == static_cast<int>(gridDim.x) - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();  // every CTA of the unit took its ticket after its writes
+  if (tid == 0) p.ticket[bg] = 0;  // ready for the next step
+  merge_unit<T, D, G, Q8>(p, bg, reinterpret_cast<float*>(dsm));
 }
 
 template <typename T, int D, bool Q8>
@@ -506,14 +698,19 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
   }
 }
 
+// One launch per step (the merge in each unit's last CTA) or two (a merge
+// kernel over slices of the keys).
+constexpr bool kDecodeFused = true;
+
 template <typename T, int D, int G, bool Q8>
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t st) {
   using L = PartialLayout<T, D, G, Q8>;
   static int attr_bits[2] = {0, 0};
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(decode_partial<T, D, G, Q8>),
-                                   L::kBytes, attr_bits);
+  const void* fn = reinterpret_cast<const void*>(decode_partial<T, D, G, Q8, kDecodeFused>);
+  cudaError_t e = ensure_smem_attr(fn, L::kBytes, attr_bits);
   if (e != cudaSuccess) return e;
-  decode_partial<T, D, G, Q8><<<dim3(p.n_chunks, p.B * p.Hkv), kThreads, L::kBytes, st>>>(p);
+  decode_partial<T, D, G, Q8, kDecodeFused>
+      <<<dim3(p.n_chunks, p.B * p.Hkv), kThreads, L::kBytes, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -527,7 +724,7 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
     case 8: e = launch_partial<T, D, 8, Q8>(p, st); break;
     default: return cudaErrorInvalidValue;
   }
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || kDecodeFused) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.n_slices, p.B * p.Hkv);
   cfg.blockDim = dim3(kThreads);
@@ -544,6 +741,8 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
 }  // namespace
 
 bool decode_supported(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
+
+int decode_launches() { return kDecodeFused ? 1 : 2; }
 
 cudaError_t launch_decode(const DecodeParams& p, int esize, int head_dim, cudaStream_t st) {
   if (p.n_chunks > kMaxChunks || !decode_supported(p.G) || p.n_slices > p.slices_ld)

@@ -328,7 +328,11 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
   }
 
   // 1. accumulate scores and build the keys; loads are batched so that
-  //    kLoadBatch of them are in flight per thread
+  //    kLoadBatch of them are in flight per thread.  On the way: the lowest
+  //    unprotected old key, the highest unprotected new key, the protected
+  //    count (for the shortcut below).
+  uint32_t old_min = 0xFFFFFFFFu, new_max = 0u;
+  int n_prot = 0;
   for (int x0 = tid; x0 < n; x0 += kLoadBatch * NT) {
     float sc[kLoadBatch], cv[kLoadBatch];
     int ps[kLoadBatch];
@@ -360,6 +364,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
           key = static_cast<uint32_t>(ps[k]);  // the most recent rank highest
         }
         keys[x] = prot ? kProtectedKey : key;
+        if (prot) ++n_prot; else old_min = min(old_min, key);
       }
     }
   }
@@ -376,8 +381,9 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
       if (i < nq) {
         const long long p = static_cast<long long>(e.t0) + i;
         const bool prot = evict && (p >= limit || p < sinks);
-        keys[n + i] = prot ? kProtectedKey
-                           : (by_score ? score_key(cv[k]) : static_cast<uint32_t>(p));
+        const uint32_t key = by_score ? score_key(cv[k]) : static_cast<uint32_t>(p);
+        keys[n + i] = prot ? kProtectedKey : key;
+        if (prot) ++n_prot; else new_max = max(new_max, key);
       }
     }
   }
@@ -393,7 +399,46 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
     place_rows<NT>(e, b, g, nq, [n](int q) { return n + q; }, [](int q) { return q; });
     return;
   }
-  __syncthreads();
+  // A full cache, nothing protected, and no new key above the lowest old key:
+  // the C old entries are the top C (an old slot also wins a tie: its index
+  // is lower), so nothing moves and the scores are already updated.  This is
+  // the steady state of caches without a recent window, where one chunk's
+  // summed weights stay below the weights the cache's entries have gathered.
+  {
+    uint32_t a = old_min, z = new_max;
+    int pr = n_prot;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
+      z = max(z, __shfl_xor_sync(0xffffffffu, z, o));
+      pr += __shfl_xor_sync(0xffffffffu, pr, o);
+    }
+    __shared__ uint32_t red_min[NT / 32], red_max[NT / 32];
+    __shared__ int red_prot[NT / 32];
+    if (lane == 0) {
+      red_min[tid >> 5] = a;
+      red_max[tid >> 5] = z;
+      red_prot[tid >> 5] = pr;
+    }
+    __syncthreads();
+    if (tid < 32) {
+      a = tid < NT / 32 ? red_min[tid] : 0xFFFFFFFFu;
+      z = tid < NT / 32 ? red_max[tid] : 0u;
+      pr = tid < NT / 32 ? red_prot[tid] : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
+        z = max(z, __shfl_xor_sync(0xffffffffu, z, o));
+        pr += __shfl_xor_sync(0xffffffffu, pr, o);
+      }
+      if (tid == 0) sel_bin = (n == C && pr == 0 && z <= a) ? 1 : 0;
+    }
+    __syncthreads();
+    if (sel_bin) {
+      if (tid == 0) e.plan_count[bg] = 0;
+      return;
+    }
+  }
 
   // 2. the C-th largest key, three digits: bits 31..21 over every key;
   //    bits 20..10 over the keys of the chosen first-digit bin, which are also

@@ -421,8 +421,8 @@ h2o_status run_decode(h2o_cache* c, const void* q, const void* kn, const void* v
       return H2O_ERR_CUDA;
   }
   c->fwd_nq = 0;  // the decode path keeps no row statistics
-  c->launches += 2;
-  mark(c, 1, st);  // both kernels are reported as the first part
+  c->launches += decode_launches();
+  mark(c, 1, st);  // the whole step is reported as the first part
   mark(c, 2, st);
   mark(c, 3, st);
   if (evict) {

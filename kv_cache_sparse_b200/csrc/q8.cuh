@@ -51,9 +51,28 @@ __device__ __forceinline__ void q8_quantize_row_warp(const __nv_bfloat16* src, i
   if (lane == 0) *scale = s;
 }
 
+// (a0, a1) - (b0, b1) and (a0, a1) * (b0, b1), packed f32x2, round to nearest.
+__device__ __forceinline__ void q8_sub2(float& d0, float& d1, float a0, float a1, float b) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b));
+}
+
+__device__ __forceinline__ void q8_mul2(float& d0, float& d1, float a0, float a1, float b) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b));
+}
+
 // 16 codes (one 16-byte chunk) times the row scale -> 16 bf16 values packed in
-// 8 words, ready for a 128-byte-swizzled MMA operand.  The codes go through
-// fp32 exactly: 2^23 + (code + 128) built by byte permutes, minus 2^23 + 128.
+// 8 words (element 2k in the low half of word k), ready for an MMA operand.
+// A code c goes through fp32 exactly: the bytes c + 128 are placed under the
+// exponent of 2^23 by byte permutes (2^23 + c + 128) and 2^23 + 128 is
+// subtracted; then one rounding for c * s (fp32) and one for bf16.
 __device__ __forceinline__ void q8_dequant16(uint4 codes, float s, uint32_t (&out)[8]) {
   const uint32_t w[4] = {codes.x ^ 0x80808080u, codes.y ^ 0x80808080u, codes.z ^ 0x80808080u,
                          codes.w ^ 0x80808080u};  // offset binary: code + 128
@@ -61,15 +80,16 @@ __device__ __forceinline__ void q8_dequant16(uint4 codes, float s, uint32_t (&ou
   for (int i = 0; i < 4; ++i) {
     float f[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      // 0x4B0000uu: 2^23 + u
-      const uint32_t bits = __byte_perm(w[i], 0x4B000000u, 0x7650 + j);
-      f[j] = __fmul_rn(__uint_as_float(bits) - 8388736.0f, s);
-    }
-    out[2 * i] = (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f[1]))) << 16) |
-                 __bfloat16_as_ushort(__float2bfloat16_rn(f[0]));
-    out[2 * i + 1] = (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f[3]))) << 16) |
-                     __bfloat16_as_ushort(__float2bfloat16_rn(f[2]));
+    for (int j = 0; j < 4; ++j) f[j] = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7650 + j));
+    q8_sub2(f[0], f[1], f[0], f[1], 8388736.0f);  // 2^23 + 128
+    q8_sub2(f[2], f[3], f[2], f[3], 8388736.0f);
+    q8_mul2(f[0], f[1], f[0], f[1], s);
+    q8_mul2(f[2], f[3], f[2], f[3], s);
+    uint32_t lo, hi;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(f[1]), "f"(f[0]));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(f[3]), "f"(f[2]));
+    out[2 * i] = lo;
+    out[2 * i + 1] = hi;
   }
 }
 

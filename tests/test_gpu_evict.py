@@ -136,3 +136,31 @@ def test_decode_eviction_with_negative_scores():
     assert gpu.check() == 0
     ref.evict(gh.np64(cs).astype(np.float32), gh.np64(kn), gh.np64(vn))
     gh.assert_state_equal(gpu.read(), ref, torch.bfloat16, "decode, negative scores")
+
+
+@pytest.mark.parametrize("B,Hkv,C,nq,W,tie", [(40, 8, 96, 32, 0, False), (40, 8, 96, 32, 0, True),
+                                              (4, 8, 256, 64, 0, False), (40, 8, 96, 32, 4, False)])
+def test_evict_no_new_key_above_the_cache(B, Hkv, C, nq, W, tie):
+    """Every new token's weight at or below every old slot's score: with no
+    recent window nothing enters the cache (an old slot also wins a tie); with
+    a window the protected tokens still enter.  Bit-exact against the oracle."""
+    rng = np.random.default_rng(C + nq + W + int(tie))
+    shape = gh.shape_of(B, Hkv, Hkv, 64, C, nq, W)
+    gpu = binding.H2OCache(shape)
+    ref = gh.oracle_for(shape)
+    t0 = C + 7
+    K, V, _, pos = gh.random_state(shape, C, t0, rng)
+    sc = (1.0 + rng.random((B, Hkv, C)) * 3).astype(np.float32)   # old scores in [1, 4)
+    gh.install_state(gpu, ref, K, V, sc, pos, C, t0)
+    cs = np.zeros((B, Hkv, C + nq), np.float32)
+    cs[:, :, :C] = (rng.random((B, Hkv, C)) * 0.5).astype(np.float32)
+    cs[:, :, C:] = (rng.random((B, Hkv, nq)) * 0.5).astype(np.float32)   # new: below 1
+    if tie:   # a new token exactly at the lowest updated old score
+        low = (sc + cs[:, :, :C]).astype(np.float32).min(axis=-1)
+        cs[:, :, C + 3] = low
+    kn = torch.randn(B, nq, Hkv, 64).to(torch.bfloat16)
+    vn = torch.randn(B, nq, Hkv, 64).to(torch.bfloat16)
+    gpu.evict(torch.from_numpy(cs).cuda(), kn.cuda(), vn.cuda())
+    assert gpu.check() == 0
+    ref.evict(cs, gh.np64(kn), gh.np64(vn))
+    gh.assert_state_equal(gpu.read(), ref, torch.bfloat16, f"W={W} tie={tie}")
