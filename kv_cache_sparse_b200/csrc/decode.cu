@@ -151,19 +151,16 @@ struct PartialLayout {
   static constexpr int kN = kS + (Q8 ? 2 * KC * 4 : 0);  // Q8: the new token's K, V rows (T)
   static constexpr int kBytes = kN + (Q8 ? 2 * D * static_cast<int>(sizeof(T)) : 0);
   static_assert(kWarps * G * D * 4 <= KC * kRow, "the P V sums must fit over the K rows");
-  // the merge (last CTA of a unit) reuses the K and V rows for [G][chunks] factors
-  static constexpr int kMaxChunksL = (kMaxCandidates + 1 + KC - 1) / KC;
-  static_assert(G * kMaxChunksL * 4 <= kX, "merge factors must fit over the K and V rows");
 };
 
 // The merge of one (cache, KV head) unit by one CTA, once every split-KV
 // partial and logit of the unit is written: per-head log-sum-exp over the
 // chunks, O, the summed weights of the n + 1 keys and, when evicting, the
 // score update, the eviction candidate (the lowest rank value, the highest
-// index among equals) and the new token's placement.  fac: [G][n_chunks]
-// shared floats.  Data the other CTAs wrote is read through L2 (__ldcg).
+// index among equals) and the new token's placement.  Data the other CTAs
+// wrote is read through L2 (__ldcg).
 template <typename T, int D, int G, bool Q8>
-__device__ __forceinline__ void merge_unit(const DecodeParams& p, int bg, float* fac) {
+__device__ __forceinline__ void merge_unit(const DecodeParams& p, int bg) {
   __shared__ float lse[G], lh[G];
   __shared__ unsigned long long wmin[kWarps];
   __shared__ float s_new;  // the new token's summed weight
@@ -174,6 +171,7 @@ __device__ __forceinline__ void merge_unit(const DecodeParams& p, int bg, float*
   const float* part = p.part + static_cast<size_t>(bg) * p.part_ld * kChunkStride;
 
   // ---- per-head log-sum-exp over the chunks (one warp per head)
+  __shared__ float mh[G];  // the head's largest chunk max
   if (warp < G) {
     float m = -INFINITY;
     for (int c = lane; c < NCk; c += 32) m = fmaxf(m, __ldcg(part + c * kChunkStride + warp * (D + 2) + D));
@@ -181,28 +179,30 @@ __device__ __forceinline__ void merge_unit(const DecodeParams& p, int bg, float*
     float l = 0.f;
     for (int c = lane; c < NCk; c += 32) {
       const float* st = part + c * kChunkStride + warp * (D + 2) + D;
-      const float f = ex2_approx(__ldcg(st) - m);
-      fac[warp * NCk + c] = f;
-      l = fmaf(__ldcg(st + 1), f, l);
+      l = fmaf(__ldcg(st + 1), ex2_approx(__ldcg(st) - m), l);
     }
     l = warp_sum(l);
     if (lane == 0) {
+      mh[warp] = m;
       lh[warp] = l;
       lse[warp] = m + __log2f(l);
     }
   }
   __syncthreads();
 
-  // ---- O: thread t merges outputs t, t + 256, ... over the chunks
+  // ---- O: thread t merges outputs t, t + 256, ... over the chunks, each
+  //      chunk's sum scaled by 2^(chunk max - head max)
   {
     T* out = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.Hkv * G + g * G) * D;
     for (int i = tid; i < G * D; i += kThreads) {
       const int h = i / D, d = i % D;
       const float* src = part + h * (D + 2) + d;
-      const float* fh = fac + h * NCk;
+      const float* mx = part + h * (D + 2) + D;
+      const float m = mh[h];
       float acc = 0.f;
 #pragma unroll 8
-      for (int c = 0; c < NCk; ++c) acc = fmaf(__ldcg(src + c * kChunkStride), fh[c], acc);
+      for (int c = 0; c < NCk; ++c)
+        acc = fmaf(__ldcg(src + c * kChunkStride), ex2_approx(__ldcg(mx + c * kChunkStride) - m), acc);
       store(out + i, acc / lh[h]);
     }
   }
@@ -321,58 +321,40 @@ __device__ __forceinline__ void merge_unit(const DecodeParams& p, int bg, float*
   }
 }
 
-// kFused: the last CTA of each (cache, KV head) also merges it (merge_unit),
-// so that the step is one launch; otherwise decode_finish follows.
-template <typename T, int D, int G, bool Q8, bool kFused>
-__global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p) {
+// The split-KV partial of one chunk (keys [chunk*KC, +KC) of the n + 1 of a
+// (cache, KV head) unit bg): logits (stored for the summed weights), the
+// chunk's max and sum per head, and the unnormalised P V, written to the
+// unit's partials.  The caller has issued the bulk copies of the chunk's
+// cache rows into sK / sV (completing bK / bV with the given parity) when
+// the chunk holds cache slots; this copies the new token's rows (when key n
+// is in the chunk) and, int8 cache, the rows' scales.  sK is reused for the
+// warps' P V sums once the logits are done.  Returns false when a wait gave
+// up (after letting the copies land).
+template <typename T, int D, int G, bool Q8>
+__device__ __forceinline__ bool chunk_partial(const DecodeParams& p, int bg, int chunk,
+                                              uint8_t* sK, uint8_t* sV, uint8_t* sN,
+                                              float* sScale, float* xs, uint32_t bK, uint32_t bV,
+                                              uint32_t parity, int* abort_flag,
+                                              const float (&qf)[G][D / 32]) {
   using L = PartialLayout<T, D, G, Q8>;
   constexpr int KC = L::KC;
   constexpr int E = D / 32;   // row elements per lane
   constexpr int KB = 32 / G;  // keys per warp batch: 32 (key, head) pairs
-  extern __shared__ __align__(128) uint8_t dsm[];
-  uint8_t* sK = dsm + L::kK;
-  uint8_t* sV = dsm + L::kV;
-  float* xs = reinterpret_cast<float*>(dsm + L::kX);
-  float* ored = reinterpret_cast<float*>(dsm + L::kK);  // written once the K rows are used
-  __shared__ __align__(8) uint64_t bars[2];
-  __shared__ int abort_flag;
   __shared__ float hstat[G][2];  // chunk max, chunk sum
-  // the merge kernel may start; it waits for this grid before reading
-  griddep_launch_dependents();
-
-  const int bg = blockIdx.y;
-  const int b = bg / p.Hkv, g = bg % p.Hkv;
-  const int chunk = blockIdx.x;
+  float* ored = reinterpret_cast<float*>(sK);  // written once the K rows are used
   const int j0 = chunk * KC;
   const int nk = p.n + 1;
   const int nkc = min(KC, nk - j0);           // keys of this chunk (>= 1)
   const int rows = max(0, min(KC, p.n - j0));  // of them cache slots
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int* err = p.state + 2;
-  const uint32_t bK = smem_u32(&bars[0]), bV = smem_u32(&bars[1]);
-  if (tid == 0) {
-    mbar_init(bK, 1);
-    mbar_init(bV, 1);
-    abort_flag = 0;
-    fence_barrier_init();
-  }
-  __syncthreads();
-  if (tid == 0 && rows > 0) {
-    const size_t off = (static_cast<size_t>(bg) * p.C + j0) * L::kRow;
-    const uint32_t bytes = static_cast<uint32_t>(rows) * L::kRow;
-    mbar_arrive_expect_tx(bK, bytes);
-    bulk_load(smem_u32(sK), static_cast<const uint8_t*>(p.k_cache) + off, bytes, bK);
-    mbar_arrive_expect_tx(bV, bytes);
-    bulk_load(smem_u32(sV), static_cast<const uint8_t*>(p.v_cache) + off, bytes, bV);
-  }
   constexpr int kNewRow = D * static_cast<int>(sizeof(T));  // the new rows are T
-  uint8_t* sNK = Q8 ? dsm + L::kN : sK + rows * L::kRow;  // the new token's rows
-  uint8_t* sNV = Q8 ? dsm + L::kN + kNewRow : sV + rows * L::kRow;
+  uint8_t* sNK = Q8 ? sN : sK + rows * L::kRow;  // the new token's rows
+  uint8_t* sNV = Q8 ? sN + kNewRow : sV + rows * L::kRow;
   if (warp == 0 && nkc > rows) {  // the new token is key n, in this chunk
     copy_row(sNK, static_cast<const uint8_t*>(p.k_new) + bg * kNewRow, kNewRow, lane);
     copy_row(sNV, static_cast<const uint8_t*>(p.v_new) + bg * kNewRow, kNewRow, lane);
   }
-  float* sScale = reinterpret_cast<float*>(dsm + L::kS);  // Q8 only
   if (Q8) {
     for (int i = tid; i < KC; i += kThreads) {
       const size_t at = static_cast<size_t>(bg) * p.C + j0 + i;
@@ -391,17 +373,9 @@ __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p)
       lds_row<T, E>((is_v ? sV : sK) + k * L::kRow + lane * E * sizeof(T), f);
     }
   };
-  // this lane's slice of the G query rows
-  float qf[G][E];
-  {
-    const T* q = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hkv * G + g * G) * D;
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-      for (int e = 0; e < E; ++e) qf[h][e] = to_float(q[h * D + lane * E + e]);
-  }
-  __syncthreads();  // the new token's rows are in place
-  bool ok = rows == 0 || mbar_wait(bK, 0, err, &abort_flag);
+  __syncthreads();  // the new token's rows and the scales are in place
+  bool ok = rows == 0 || mbar_wait(bK, parity, err, abort_flag);
+  ok = __all_sync(0xffffffffu, ok);
 
   // ---- logits: a warp batch is KB keys x G heads = 32 dot products
   if (ok) {
@@ -458,7 +432,8 @@ __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p)
       hstat[warp][1] = l;
     }
   }
-  if (ok && rows > 0) ok = mbar_wait(bV, 0, err, &abort_flag);
+  if (ok && rows > 0) ok = mbar_wait(bV, parity, err, abort_flag);
+  ok = __all_sync(0xffffffffu, ok);
   __syncthreads();
   // ---- P V: each lane its head-dim slice, warps over the keys
   float o[G][E];
@@ -479,8 +454,8 @@ __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p)
     }
   }
   if (!ok && tid == 0 && rows > 0) {  // a wait gave up: the copies land before their
-    mbar_wait_drain(bK, 0, err);      // buffers are written or the CTA exits
-    mbar_wait_drain(bV, 0, err);
+    mbar_wait_drain(bK, parity, err);  // buffers are written or reused
+    mbar_wait_drain(bV, parity, err);
   }
   __syncthreads();  // every warp is done with the K rows
 #pragma unroll
@@ -501,17 +476,157 @@ __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p)
       part[tid * (D + 2) + D + 1] = hstat[tid][1];
     }
   }
-  if (!kFused) return;
-  // ---- the last CTA of this (cache, KV head) to get here merges the unit
+  return ok;
+}
+
+// Ticket of unit bg after one of its chunks: true in the CTA that finished
+// the unit's last chunk, after which every chunk's logits and partials are
+// visible to it (and the ticket is reset for the next step).
+__device__ __forceinline__ bool last_of_unit(const DecodeParams& p, int bg) {
   __shared__ int is_last;
   __threadfence();  // this CTA's logits and partials, before the ticket
   __syncthreads();
-  if (tid == 0) is_last = atomicAdd(&p.ticket[bg], 1) == static_cast<int>(gridDim.x) - 1;
+  if (threadIdx.x == 0) is_last = atomicAdd(&p.ticket[bg], 1) == p.n_chunks - 1;
   __syncthreads();
-  if (!is_last) return;
-  __threadfence();  // every CTA of the unit took its ticket after its writes
-  if (tid == 0) p.ticket[bg] = 0;  // ready for the next step
-  merge_unit<T, D, G, Q8>(p, bg, reinterpret_cast<float*>(dsm));
+  const bool last = is_last != 0;
+  if (last) {
+    __threadfence();  // every CTA of the unit took its ticket after its writes
+    if (threadIdx.x == 0) p.ticket[bg] = 0;  // ready for the next step
+  }
+  return last;
+}
+
+// This lane's slice of the G query rows of unit bg.
+template <typename T, int D, int G>
+__device__ __forceinline__ void load_q(const DecodeParams& p, int bg, float (&qf)[G][D / 32]) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  const T* q = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hkv * G + g * G) * D;
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < E; ++e) qf[h][e] = to_float(q[h * D + lane * E + e]);
+}
+
+// Bulk copies of the cache rows of chunk `chunk` of unit bg (cache slots
+// only; nothing when the chunk holds just the new token).
+template <typename T, int D, int G, bool Q8>
+__device__ __forceinline__ void load_chunk(const DecodeParams& p, int bg, int chunk, uint8_t* sK,
+                                           uint8_t* sV, uint32_t bK, uint32_t bV) {
+  using L = PartialLayout<T, D, G, Q8>;
+  const int j0 = chunk * L::KC;
+  const int rows = max(0, min(L::KC, p.n - j0));
+  if (rows == 0) {  // nothing to copy: the phases still complete, so that a
+    mbar_arrive(bK);  // reused stage keeps its parity
+    mbar_arrive(bV);
+    return;
+  }
+  const size_t off = (static_cast<size_t>(bg) * p.C + j0) * L::kRow;
+  const uint32_t bytes = static_cast<uint32_t>(rows) * L::kRow;
+  mbar_arrive_expect_tx(bK, bytes);
+  bulk_load(smem_u32(sK), static_cast<const uint8_t*>(p.k_cache) + off, bytes, bK);
+  mbar_arrive_expect_tx(bV, bytes);
+  bulk_load(smem_u32(sV), static_cast<const uint8_t*>(p.v_cache) + off, bytes, bV);
+}
+
+// One CTA per chunk; kFused: the last CTA of each (cache, KV head) also
+// merges it (merge_unit), so that the step is one launch; otherwise
+// decode_finish follows.
+template <typename T, int D, int G, bool Q8, bool kFused>
+__global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p) {
+  using L = PartialLayout<T, D, G, Q8>;
+  extern __shared__ __align__(128) uint8_t dsm[];
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ int abort_flag;
+  // the merge kernel may start; it waits for this grid before reading
+  griddep_launch_dependents();
+  const int bg = blockIdx.y;
+  const int chunk = blockIdx.x;
+  const uint32_t bK = smem_u32(&bars[0]), bV = smem_u32(&bars[1]);
+  if (threadIdx.x == 0) {
+    mbar_init(bK, 1);
+    mbar_init(bV, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) load_chunk<T, D, G, Q8>(p, bg, chunk, dsm + L::kK, dsm + L::kV, bK, bV);
+  float qf[G][D / 32];
+  load_q<T, D, G>(p, bg, qf);
+  chunk_partial<T, D, G, Q8>(p, bg, chunk, dsm + L::kK, dsm + L::kV, dsm + L::kN,
+                             reinterpret_cast<float*>(dsm + L::kS),
+                             reinterpret_cast<float*>(dsm + L::kX), bK, bV, 0u, &abort_flag, qf);
+  if (!kFused) return;
+  if (last_of_unit(p, bg)) merge_unit<T, D, G, Q8>(p, bg);
+}
+
+// decode_stream: the same work with one CTA per SM streaming the chunks
+// (chunk-major within each unit: item i is chunk i mod n_chunks of unit
+// i / n_chunks; CTA c takes items c, c + grid, ...).  The cache rows of the
+// CTA's next kStages - 1 chunks are in flight (bulk copies into a ring of
+// stages) while it works on one, so the copies keep HBM busy through the
+// compute and the merges; the CTA that finishes a unit's last chunk merges
+// the unit.
+template <typename T, int D, int G, bool Q8>
+struct StreamLayout {
+  using PL = PartialLayout<T, D, G, Q8>;
+  static constexpr int kStages = 3;
+  // one stage: K rows, V rows, (Q8) the scales of both and the new token's rows
+  static constexpr int kStageBytes = (PL::kX + (PL::kN - PL::kS) +
+                                      (Q8 ? 2 * D * static_cast<int>(sizeof(T)) : 0) + 127) /
+                                     128 * 128;
+  static constexpr int kSOff = PL::kX;                   // within a stage: the scales
+  static constexpr int kNOff = kSOff + (PL::kN - PL::kS);  // the new token's rows
+  static constexpr int kX = kStages * kStageBytes;        // [G][KC] float
+  static constexpr int kBytes = kX + G * PL::KC * 4;
+  static_assert(kBytes <= kMaxDynSmem, "decode stream layout too large");
+};
+
+template <typename T, int D, int G, bool Q8>
+__global__ void __launch_bounds__(kThreads, 1) decode_stream(const DecodeParams p) {
+  using L = StreamLayout<T, D, G, Q8>;
+  using PL = PartialLayout<T, D, G, Q8>;
+  extern __shared__ __align__(128) uint8_t dsm[];
+  __shared__ __align__(8) uint64_t bars[2 * L::kStages];
+  __shared__ int abort_flag;
+  const int NCk = p.n_chunks;
+  const int total = p.B * p.Hkv * NCk;
+  const int first = static_cast<int>(blockIdx.x), stride = static_cast<int>(gridDim.x);
+  auto stage = [&](int k) { return dsm + (k % L::kStages) * L::kStageBytes; };
+  auto barK = [&](int k) { return smem_u32(&bars[2 * (k % L::kStages)]); };
+  auto barV = [&](int k) { return smem_u32(&bars[2 * (k % L::kStages) + 1]); };
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2 * L::kStages; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // the first kStages chunks of this CTA
+  if (threadIdx.x == 0)
+    for (int k = 0; k < L::kStages; ++k) {
+      const int i = first + k * stride;
+      if (i >= total) break;
+      load_chunk<T, D, G, Q8>(p, i / NCk, i % NCk, stage(k), stage(k) + PL::kV, barK(k), barV(k));
+    }
+  float qf[G][D / 32];
+  for (int k = 0, i = first; i < total; ++k, i += stride) {
+    const int bg = i / NCk, chunk = i % NCk;
+    load_q<T, D, G>(p, bg, qf);
+    uint8_t* st = stage(k);
+    chunk_partial<T, D, G, Q8>(p, bg, chunk, st, st + PL::kV, st + L::kNOff,
+                               reinterpret_cast<float*>(st + L::kSOff),
+                               reinterpret_cast<float*>(dsm + L::kX), barK(k), barV(k),
+                               static_cast<uint32_t>((k / L::kStages) & 1), &abort_flag, qf);
+    const bool last = last_of_unit(p, bg);  // its barriers also end every use of the stage
+    const int inext = i + L::kStages * stride;
+    if (threadIdx.x == 0 && inext < total) {
+      fence_proxy_async_smem();  // the stage's generic reads and writes before the copies
+      load_chunk<T, D, G, Q8>(p, inext / NCk, inext % NCk, st, st + PL::kV, barK(k), barV(k));
+    }
+    if (last) merge_unit<T, D, G, Q8>(p, bg);
+    __syncthreads();  // the merge's shared scratch before the next chunk
+  }
 }
 
 template <typename T, int D, bool Q8>
@@ -699,11 +814,35 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
 }
 
 // One launch per step (the merge in each unit's last CTA) or two (a merge
-// kernel over slices of the keys).
+// kernel over slices of the keys); with one launch, one CTA per chunk or one
+// streaming CTA per SM.
 constexpr bool kDecodeFused = true;
+constexpr bool kDecodeStream = true;
+
+template <typename T, int D, int G, bool Q8>
+cudaError_t launch_stream(const DecodeParams& p, cudaStream_t st) {
+  using L = StreamLayout<T, D, G, Q8>;
+  static int attr_bits[2] = {0, 0};
+  const void* fn = reinterpret_cast<const void*>(decode_stream<T, D, G, Q8>);
+  cudaError_t e = ensure_smem_attr(fn, L::kBytes, attr_bits);
+  if (e != cudaSuccess) return e;
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0, v = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    sms = v;
+  }
+  const long long total = static_cast<long long>(p.B) * p.Hkv * p.n_chunks;
+  const int grid = static_cast<int>(total < sms ? total : sms);
+  decode_stream<T, D, G, Q8><<<grid, kThreads, L::kBytes, st>>>(p);
+  return cudaGetLastError();
+}
 
 template <typename T, int D, int G, bool Q8>
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t st) {
+  if (kDecodeFused && kDecodeStream) return launch_stream<T, D, G, Q8>(p, st);
   using L = PartialLayout<T, D, G, Q8>;
   static int attr_bits[2] = {0, 0};
   const void* fn = reinterpret_cast<const void*>(decode_partial<T, D, G, Q8, kDecodeFused>);
