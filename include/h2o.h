@@ -167,9 +167,8 @@ H2O_API h2o_status h2o_cache_create(const h2o_config* cfg, const h2o_buffers* bu
  * layouts above with 1 <= n_q <= max_chunk (n_q = 0 is a no-op).
  * colsum_out (device, may be NULL) receives the summed weights in the colsum
  * layout.  Advances n and t0.  A decode step (n_q = 1, at most 8 query heads
- * per KV head) runs as one launch (split-KV attention; the last CTA of each
- * (cache, KV head) merges it, writes the summed weights and does the
- * single-token eviction), other steps as three. */
+ * per KV head) runs as two launches (split-KV attention; merge, summed
+ * weights and the single-token eviction), other steps as three. */
 H2O_API h2o_status h2o_chunk_step(h2o_cache* c, const void* q, const void* k_new,
                           const void* v_new, int32_t n_q, void* out,
                           float* colsum_out, void* stream);

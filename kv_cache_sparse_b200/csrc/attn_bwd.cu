@@ -9,7 +9,8 @@
 //   dV = P^T dO,  dP = dO V^T,  dS = P (dP - D) with D_i = <dO_i, O_i>,
 //   dQ = scale dS K,  dK = scale dS^T Q,
 // dK and dV summed over the G query heads of a KV head.  Three kernels:
-//   bwd_rowdot   D_i for every (cache, head, query): one warp per row.
+//   bwd_rowdot   -scale * D_i for every (cache, head, query): one warp per
+//                row (0 for the padding rows up to the next multiple of 128).
 //   bwd_dkdv     key-stationary, like the column-sum kernel: one CTA per
 //                (cache, KV head, 128 keys), looping over the (head, query
 //                tile) units that see its keys.  The MMAs compute
@@ -41,22 +42,23 @@ namespace h2o {
 
 __global__ void bwd_rowdot(const __nv_bfloat16* __restrict__ out,
                            const __nv_bfloat16* __restrict__ dout, const BwdParams p, int d) {
-  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);  // (b, i, h)
+  // one warp per row (b, h, i) of the padded statistic; i >= nq gets 0
+  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  const int rows = p.B * p.nq * p.Hq;
+  const int rows = p.B * p.Hq * p.nq_pad;
   if (row >= rows) return;
-  const __nv_bfloat16* o = out + static_cast<size_t>(row) * d;
-  const __nv_bfloat16* g = dout + static_cast<size_t>(row) * d;
+  const int i = row % p.nq_pad;
+  const int h = (row / p.nq_pad) % p.Hq;
+  const int b = row / (p.nq_pad * p.Hq);
   float s = 0.f;
-  for (int e = lane; e < d; e += 32) s = fmaf(__bfloat162float(o[e]), __bfloat162float(g[e]), s);
+  if (i < p.nq) {
+    const size_t at = ((static_cast<size_t>(b) * p.nq + i) * p.Hq + h) * d;
+    for (int e = lane; e < d; e += 32) s = fmaf(__bfloat162float(out[at + e]), __bfloat162float(dout[at + e]), s);
 #pragma unroll
-  for (int o2 = 16; o2 > 0; o2 >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o2);
-  if (lane == 0) {
-    const int h = row % p.Hq;
-    const int i = (row / p.Hq) % p.nq;
-    const int b = row / (p.Hq * p.nq);
-    p.dsum[(static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + i] = s;
+    for (int o2 = 16; o2 > 0; o2 >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o2);
   }
+  // stored as -scale * D_i, the term the row arithmetic adds to scale * dP
+  if (lane == 0) p.dsum[row] = -p.scale * s;
 }
 
 // ---------------------------------------------------------------- dK, dV
@@ -84,26 +86,47 @@ struct DkdvLayout {
 constexpr int kBwdThreads = 64 + 2 * 128;
 
 // Row arithmetic shared by the two kernels: from 32 logits s and 32 dP
-// values of one row (or one key), the bf16 pairs of P and of scale * dS.
-// nls[c] = -lse2 of the query of column c (or of the row), dv[c] = its D.
-template <bool kMask>
+// values of one row (or one key), the bf16 pairs of P and of scale * dS =
+// P (scale dP - scale D).  Column c's statistics: -lse2 in nls and -scale*D
+// in nds, either per column (kCol: 32 floats each in shared memory, read 16
+// bytes at a time) or one value for the whole row (nls[0], nds[0]).  Pairs
+// of columns go through packed f32x2 arithmetic.
+template <bool kMask, bool kCol>
 __device__ __forceinline__ void p_ds_32(const uint32_t (&s)[32], const uint32_t (&dp)[32],
-                                        const float* nls, const float* dv, float c, float scale,
+                                        const float* nls, const float* nds, float c, float scale,
                                         int first_valid, int last_valid, uint32_t (&pp)[16],
                                         uint32_t (&dd)[16]) {
 #pragma unroll
-  for (int k = 0; k < 32; k += 2) {
-    float p0 = ex2_approx(fmaf(__uint_as_float(s[k]), c, nls[k]));
-    float p1 = ex2_approx(fmaf(__uint_as_float(s[k + 1]), c, nls[k + 1]));
+  for (int k = 0; k < 32; k += 4) {
+    float4 nl, nd;
+    if (kCol) {
+      nl = *reinterpret_cast<const float4*>(nls + k);
+      nd = *reinterpret_cast<const float4*>(nds + k);
+    } else {
+      nl = make_float4(nls[0], nls[0], nls[0], nls[0]);
+      nd = make_float4(nds[0], nds[0], nds[0], nds[0]);
+    }
+    float x0, x1, x2, x3;
+    ffma2(x0, x1, __uint_as_float(s[k]), __uint_as_float(s[k + 1]), c, c, nl.x, nl.y);
+    ffma2(x2, x3, __uint_as_float(s[k + 2]), __uint_as_float(s[k + 3]), c, c, nl.z, nl.w);
+    float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
     if (kMask) {
       p0 = (k >= first_valid && k <= last_valid) ? p0 : 0.f;
       p1 = (k + 1 >= first_valid && k + 1 <= last_valid) ? p1 : 0.f;
+      p2 = (k + 2 >= first_valid && k + 2 <= last_valid) ? p2 : 0.f;
+      p3 = (k + 3 >= first_valid && k + 3 <= last_valid) ? p3 : 0.f;
     }
-    // P = 0 (masked, padding or underflow) gives dS = 0 whatever D holds
-    const float d0 = p0 != 0.f ? p0 * (__uint_as_float(dp[k]) - dv[k]) * scale : 0.f;
-    const float d1 = p1 != 0.f ? p1 * (__uint_as_float(dp[k + 1]) - dv[k + 1]) * scale : 0.f;
+    // every term is finite (padding rows have P = 0 and -scale*D = 0), so a
+    // zero P gives a zero dS
+    float t0, t1, t2, t3, d0, d1, d2, d3;
+    ffma2(t0, t1, __uint_as_float(dp[k]), __uint_as_float(dp[k + 1]), scale, scale, nd.x, nd.y);
+    ffma2(t2, t3, __uint_as_float(dp[k + 2]), __uint_as_float(dp[k + 3]), scale, scale, nd.z, nd.w);
+    fmul2(d0, d1, p0, p1, t0, t1);
+    fmul2(d2, d3, p2, p3, t2, t3);
     pp[k >> 1] = pack_bf16x2(p0, p1);
+    pp[(k >> 1) + 1] = pack_bf16x2(p2, p3);
     dd[k >> 1] = pack_bf16x2(d0, d1);
+    dd[(k >> 1) + 1] = pack_bf16x2(d2, d3);
   }
 }
 
@@ -304,7 +327,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const float* nls = reinterpret_cast<const float*>(smem + L::kRowOff + s * 1024);
-      const float* dvv = nls + 128;
+      const float* nds = nls + 128;
       const int qt = qt_min + u % span;
       const bool diag = is_chunk && qt == kt;  // query col sees key row iff row <= col
 #pragma unroll
@@ -315,10 +338,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(lane_base + 128 + 32 * q32, dp);
         tmem_wait_ld();
         if (diag)
-          p_ds_32<true>(sv, dp, nls + 32 * q32, dvv + 32 * q32, c, scale, row - 32 * q32, 1 << 30,
-                        pp, dd);
+          p_ds_32<true, true>(sv, dp, nls + 32 * q32, nds + 32 * q32, c, scale, row - 32 * q32,
+                              1 << 30, pp, dd);
         else
-          p_ds_32<false>(sv, dp, nls + 32 * q32, dvv + 32 * q32, c, scale, 0, 0, pp, dd);
+          p_ds_32<false, true>(sv, dp, nls + 32 * q32, nds + 32 * q32, c, scale, 0, 0, pp, dd);
         // bf16 pairs over the half's first columns: queries [32 q32, +32) ->
         // columns [64 hf + 16 q2, +16)
         tmem_st16(lane_base + 64 * hf + 16 * q2, pp);
@@ -559,14 +582,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float c = p.scale_log2, scale = p.scale;
     const size_t ridx = (static_cast<size_t>(b) * p.Hq + h) * p.nq_pad + i;
-    const float nl = p.nlse2[ridx];  // -inf for padding rows: P = 0
-    const float dsum = i < p.nq ? p.dsum[ridx] : 0.f;
-    float nls[32], dvv[32];
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      nls[k] = nl;
-      dvv[k] = dsum;
-    }
+    const float nls[1] = {p.nlse2[ridx]};  // -inf for padding rows: P = 0
+    const float nds[1] = {p.dsum[ridx]};   // -scale * D_i (0 for padding rows)
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       ok = mbar_wait(bar_s0 + 8 * hf, t & 1, p.err, abort_flag);
@@ -593,9 +610,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(lane_base + 128 + 32 * q32, dp);
         tmem_wait_ld();
         if (masked)
-          p_ds_32<true>(sv, dp, nls, dvv, c, scale, 0, last - 32 * q32, pp, dd);
+          p_ds_32<true, false>(sv, dp, nls, nds, c, scale, 0, last - 32 * q32, pp, dd);
         else
-          p_ds_32<false>(sv, dp, nls, dvv, c, scale, 0, 0, pp, dd);
+          p_ds_32<false, false>(sv, dp, nls, nds, c, scale, 0, 0, pp, dd);
         // scale*dS over S: keys [32 q32, +32) -> columns [64 hf + 16 q2, +16)
         tmem_st16(lane_base + 64 * hf + 16 * q2, dd);
       }
@@ -639,7 +656,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 template <int D>
 static cudaError_t launch_bwd_d(const BwdMaps& m, const BwdParams& p, const void* out,
                                 const void* dout, cudaStream_t st) {
-  const int rows = p.B * p.nq * p.Hq;
+  const int rows = p.B * p.Hq * p.nq_pad;
   bwd_rowdot<<<cdiv(rows, 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(out),
                                             static_cast<const __nv_bfloat16*>(dout), p, D);
   cudaError_t e = cudaGetLastError();

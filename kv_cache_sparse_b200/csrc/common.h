@@ -83,7 +83,7 @@ struct BwdParams {
   float scale;            // softmax scale (natural)
   float scale_log2;       // scale * log2(e)
   const float* nlse2;     // [B, Hq, nq_pad]: the forward's -lse2 (-inf for padding rows)
-  float* dsum;            // [B, Hq, nq_pad]: D_i = <dO_i, O_i>
+  float* dsum;            // [B, Hq, nq_pad]: -scale * D_i, D_i = <dO_i, O_i> (0 past nq)
   float* dq;              // [B, nq, Hq, d]
   float* dk_cache;        // [B, Hkv, C, d]
   float* dv_cache;

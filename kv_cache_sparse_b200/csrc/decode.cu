@@ -151,6 +151,9 @@ struct PartialLayout {
   static constexpr int kN = kS + (Q8 ? 2 * KC * 4 : 0);  // Q8: the new token's K, V rows (T)
   static constexpr int kBytes = kN + (Q8 ? 2 * D * static_cast<int>(sizeof(T)) : 0);
   static_assert(kWarps * G * D * 4 <= KC * kRow, "the P V sums must fit over the K rows");
+  // the merge (last CTA of a unit) reuses the K and V rows for 2 x [G][chunks] floats
+  static constexpr int kMaxChunksL = (kMaxCandidates + 1 + KC - 1) / KC;
+  static_assert(2 * G * kMaxChunksL * 4 <= kX, "merge scratch must fit over the K and V rows");
 };
 
 // The merge of one (cache, KV head) unit by one CTA, once every split-KV
@@ -158,9 +161,16 @@ struct PartialLayout {
 // chunks, O, the summed weights of the n + 1 keys and, when evicting, the
 // score update, the eviction candidate (the lowest rank value, the highest
 // index among equals) and the new token's placement.  Data the other CTAs
-// wrote is read through L2 (__ldcg).
+// wrote is read through L2 (__ldcg); each pass issues its loads in batches
+// before using them, so that one CTA keeps many in flight.  scratch: shared
+// memory for 2 * G * n_chunks floats.
+// Loads per thread per batch: G * kMergeBatch<G> logits (keys) or kR *
+// kMergeBatch<G> partial outputs (chunks).
+template <int G>
+constexpr int kMergeBatch = G >= 8 ? 2 : 16 / G;
+
 template <typename T, int D, int G, bool Q8>
-__device__ __forceinline__ void merge_unit(const DecodeParams& p, int bg) {
+__device__ __forceinline__ void merge_unit(const DecodeParams& p, int bg, float* scratch) {
   __shared__ float lse[G], lh[G];
   __shared__ unsigned long long wmin[kWarps];
   __shared__ float s_new;  // the new token's summed weight
@@ -169,46 +179,73 @@ __device__ __forceinline__ void merge_unit(const DecodeParams& p, int bg) {
   const int b = bg / p.Hkv, g = bg % p.Hkv;
   constexpr size_t kChunkStride = static_cast<size_t>(G) * (D + 2);
   const float* part = p.part + static_cast<size_t>(bg) * p.part_ld * kChunkStride;
+  float* fac = scratch;                // [G][NCk]: chunk max, then 2^(chunk max - head max)
+  float* csum = scratch + G * NCk;     // [G][NCk]: chunk sums
 
-  // ---- per-head log-sum-exp over the chunks (one warp per head)
-  __shared__ float mh[G];  // the head's largest chunk max
+  // ---- per-head log-sum-exp over the chunks: the chunk statistics into
+  //      shared memory (all loads in flight), then one warp per head
+  for (int i = tid; i < G * NCk; i += kThreads) {
+    const int h = i / NCk, c = i % NCk;
+    const float* st = part + c * kChunkStride + h * (D + 2) + D;
+    fac[i] = __ldcg(st);
+    csum[i] = __ldcg(st + 1);
+  }
+  __syncthreads();
   if (warp < G) {
     float m = -INFINITY;
-    for (int c = lane; c < NCk; c += 32) m = fmaxf(m, __ldcg(part + c * kChunkStride + warp * (D + 2) + D));
+    for (int c = lane; c < NCk; c += 32) m = fmaxf(m, fac[warp * NCk + c]);
     m = warp_max(m);
     float l = 0.f;
     for (int c = lane; c < NCk; c += 32) {
-      const float* st = part + c * kChunkStride + warp * (D + 2) + D;
-      l = fmaf(__ldcg(st + 1), ex2_approx(__ldcg(st) - m), l);
+      const float f = ex2_approx(fac[warp * NCk + c] - m);
+      fac[warp * NCk + c] = f;
+      l = fmaf(csum[warp * NCk + c], f, l);
     }
     l = warp_sum(l);
     if (lane == 0) {
-      mh[warp] = m;
       lh[warp] = l;
       lse[warp] = m + __log2f(l);
     }
   }
   __syncthreads();
 
-  // ---- O: thread t merges outputs t, t + 256, ... over the chunks, each
-  //      chunk's sum scaled by 2^(chunk max - head max)
+  // ---- O: thread t merges outputs t, t + 256, ... (kR of them) over the
+  //      chunks, kMergeBatch<G> chunks of loads at a time
   {
+    constexpr int kR = (G * D + kThreads - 1) / kThreads;
     T* out = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.Hkv * G + g * G) * D;
-    for (int i = tid; i < G * D; i += kThreads) {
-      const int h = i / D, d = i % D;
-      const float* src = part + h * (D + 2) + d;
-      const float* mx = part + h * (D + 2) + D;
-      const float m = mh[h];
-      float acc = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < NCk; ++c)
-        acc = fmaf(__ldcg(src + c * kChunkStride), ex2_approx(__ldcg(mx + c * kChunkStride) - m), acc);
-      store(out + i, acc / lh[h]);
+    float acc[kR];
+#pragma unroll
+    for (int r = 0; r < kR; ++r) acc[r] = 0.f;
+    for (int c0 = 0; c0 < NCk; c0 += kMergeBatch<G>) {
+      float v[kMergeBatch<G>][kR];
+#pragma unroll
+      for (int u = 0; u < kMergeBatch<G>; ++u)
+#pragma unroll
+        for (int r = 0; r < kR; ++r) {
+          const int i = tid + r * kThreads;
+          v[u][r] = (c0 + u < NCk && i < G * D)
+                        ? __ldcg(part + (c0 + u) * kChunkStride + (i / D) * (D + 2) + (i % D))
+                        : 0.f;
+        }
+#pragma unroll
+      for (int u = 0; u < kMergeBatch<G>; ++u)
+#pragma unroll
+        for (int r = 0; r < kR; ++r) {
+          const int i = tid + r * kThreads;
+          if (c0 + u < NCk && i < G * D) acc[r] = fmaf(v[u][r], fac[(i / D) * NCk + c0 + u], acc[r]);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+      const int i = tid + r * kThreads;
+      if (i < G * D) store(out + i, acc[r] / lh[i / D]);
     }
   }
 
   // ---- summed weights of the n + 1 keys, with the score update and this
-  //      thread's eviction candidate on the way
+  //      thread's eviction candidate on the way; kMergeBatch<G> keys per thread
+  //      per batch, their loads issued before any of them is used
   const float* lg = p.logits + static_cast<size_t>(bg) * G * (C + 1);
   float* cs = p.colsum + static_cast<size_t>(bg) * p.colsum_ld;
   float* score = p.scores + static_cast<size_t>(bg) * C;
@@ -225,37 +262,48 @@ __device__ __forceinline__ void merge_unit(const DecodeParams& p, int bg) {
 #pragma unroll
   for (int h = 0; h < G; ++h) lse_r[h] = lse[h];
   unsigned long long best = ~0ull;
-#pragma unroll 4
-  for (int j = tid; j <= n; j += kThreads) {
-    float x[G];
+  for (int j0 = tid; j0 <= n; j0 += kMergeBatch<G> * kThreads) {
+    float x[kMergeBatch<G>][G], sc[kMergeBatch<G>];
+    int ps[kMergeBatch<G>];
 #pragma unroll
-    for (int h = 0; h < G; ++h) x[h] = __ldcg(lg + static_cast<size_t>(h) * (C + 1) + j);
-    float sw = 0.f;
+    for (int u = 0; u < kMergeBatch<G>; ++u) {
+      const int j = j0 + u * kThreads;
+      const bool key = j <= n, slot = j < n;
 #pragma unroll
-    for (int h = 0; h < G; ++h) sw += ex2_approx(x[h] - lse_r[h]);
-    if (j == n) {
-      cs[C] = sw;
-      s_new = sw;
-      continue;
+      for (int h = 0; h < G; ++h) x[u][h] = key ? __ldcg(lg + static_cast<size_t>(h) * (C + 1) + j) : 0.f;
+      sc[u] = (slot && p.evict && by_score) ? score[j] : 0.f;
+      ps[u] = (slot && full) ? pos[j] : 0;
     }
-    cs[j] = sw;
-    if (!p.evict) continue;
-    if (!full) {
-      if (by_score) score[j] = __fadd_rn(score[j], sw);
-      continue;
-    }
-    const int ps = pos[j];
-    uint32_t rank;
-    if (by_score) {
-      const float sc = __fadd_rn(score[j], sw);
-      score[j] = sc;
-      rank = ordered_key(sc);
-    } else {
-      rank = static_cast<uint32_t>(ps);
-    }
-    if (ps < limit && ps >= sinks) {
-      const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - j);
-      best = key < best ? key : best;
+#pragma unroll
+    for (int u = 0; u < kMergeBatch<G>; ++u) {
+      const int j = j0 + u * kThreads;
+      if (j > n) continue;
+      float sw = 0.f;
+#pragma unroll
+      for (int h = 0; h < G; ++h) sw += ex2_approx(x[u][h] - lse_r[h]);
+      if (j == n) {
+        cs[C] = sw;
+        s_new = sw;
+        continue;
+      }
+      cs[j] = sw;
+      if (!p.evict) continue;
+      if (!full) {
+        if (by_score) score[j] = __fadd_rn(sc[u], sw);
+        continue;
+      }
+      uint32_t rank;
+      if (by_score) {
+        const float v = __fadd_rn(sc[u], sw);
+        score[j] = v;
+        rank = ordered_key(v);
+      } else {
+        rank = static_cast<uint32_t>(ps[u]);
+      }
+      if (ps[u] < limit && ps[u] >= sinks) {
+        const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - j);
+        best = key < best ? key : best;
+      }
     }
   }
   for (int j = n + tid; j < C; j += kThreads) cs[j] = 0.f;  // empty slots received nothing
@@ -534,7 +582,7 @@ __device__ __forceinline__ void load_chunk(const DecodeParams& p, int bg, int ch
 // merges it (merge_unit), so that the step is one launch; otherwise
 // decode_finish follows.
 template <typename T, int D, int G, bool Q8, bool kFused>
-__global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 3) decode_partial(const DecodeParams p) {
   using L = PartialLayout<T, D, G, Q8>;
   extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ __align__(8) uint64_t bars[2];
@@ -558,80 +606,14 @@ __global__ void __launch_bounds__(kThreads) decode_partial(const DecodeParams p)
                              reinterpret_cast<float*>(dsm + L::kS),
                              reinterpret_cast<float*>(dsm + L::kX), bK, bV, 0u, &abort_flag, qf);
   if (!kFused) return;
-  if (last_of_unit(p, bg)) merge_unit<T, D, G, Q8>(p, bg);
-}
-
-// decode_stream: the same work with one CTA per SM streaming the chunks
-// (chunk-major within each unit: item i is chunk i mod n_chunks of unit
-// i / n_chunks; CTA c takes items c, c + grid, ...).  The cache rows of the
-// CTA's next kStages - 1 chunks are in flight (bulk copies into a ring of
-// stages) while it works on one, so the copies keep HBM busy through the
-// compute and the merges; the CTA that finishes a unit's last chunk merges
-// the unit.
-template <typename T, int D, int G, bool Q8>
-struct StreamLayout {
-  using PL = PartialLayout<T, D, G, Q8>;
-  static constexpr int kStages = 3;
-  // one stage: K rows, V rows, (Q8) the scales of both and the new token's rows
-  static constexpr int kStageBytes = (PL::kX + (PL::kN - PL::kS) +
-                                      (Q8 ? 2 * D * static_cast<int>(sizeof(T)) : 0) + 127) /
-                                     128 * 128;
-  static constexpr int kSOff = PL::kX;                   // within a stage: the scales
-  static constexpr int kNOff = kSOff + (PL::kN - PL::kS);  // the new token's rows
-  static constexpr int kX = kStages * kStageBytes;        // [G][KC] float
-  static constexpr int kBytes = kX + G * PL::KC * 4;
-  static_assert(kBytes <= kMaxDynSmem, "decode stream layout too large");
-};
-
-template <typename T, int D, int G, bool Q8>
-__global__ void __launch_bounds__(kThreads, 1) decode_stream(const DecodeParams p) {
-  using L = StreamLayout<T, D, G, Q8>;
-  using PL = PartialLayout<T, D, G, Q8>;
-  extern __shared__ __align__(128) uint8_t dsm[];
-  __shared__ __align__(8) uint64_t bars[2 * L::kStages];
-  __shared__ int abort_flag;
-  const int NCk = p.n_chunks;
-  const int total = p.B * p.Hkv * NCk;
-  const int first = static_cast<int>(blockIdx.x), stride = static_cast<int>(gridDim.x);
-  auto stage = [&](int k) { return dsm + (k % L::kStages) * L::kStageBytes; };
-  auto barK = [&](int k) { return smem_u32(&bars[2 * (k % L::kStages)]); };
-  auto barV = [&](int k) { return smem_u32(&bars[2 * (k % L::kStages) + 1]); };
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < 2 * L::kStages; ++i) mbar_init(smem_u32(&bars[i]), 1);
-    abort_flag = 0;
-    fence_barrier_init();
-  }
-  __syncthreads();
-  // the first kStages chunks of this CTA
-  if (threadIdx.x == 0)
-    for (int k = 0; k < L::kStages; ++k) {
-      const int i = first + k * stride;
-      if (i >= total) break;
-      load_chunk<T, D, G, Q8>(p, i / NCk, i % NCk, stage(k), stage(k) + PL::kV, barK(k), barV(k));
-    }
-  float qf[G][D / 32];
-  for (int k = 0, i = first; i < total; ++k, i += stride) {
-    const int bg = i / NCk, chunk = i % NCk;
-    load_q<T, D, G>(p, bg, qf);
-    uint8_t* st = stage(k);
-    chunk_partial<T, D, G, Q8>(p, bg, chunk, st, st + PL::kV, st + L::kNOff,
-                               reinterpret_cast<float*>(st + L::kSOff),
-                               reinterpret_cast<float*>(dsm + L::kX), barK(k), barV(k),
-                               static_cast<uint32_t>((k / L::kStages) & 1), &abort_flag, qf);
-    const bool last = last_of_unit(p, bg);  // its barriers also end every use of the stage
-    const int inext = i + L::kStages * stride;
-    if (threadIdx.x == 0 && inext < total) {
-      fence_proxy_async_smem();  // the stage's generic reads and writes before the copies
-      load_chunk<T, D, G, Q8>(p, inext / NCk, inext % NCk, st, st + PL::kV, barK(k), barV(k));
-    }
-    if (last) merge_unit<T, D, G, Q8>(p, bg);
-    __syncthreads();  // the merge's shared scratch before the next chunk
-  }
+  // the merge's scratch reuses the K and V rows (every copy has landed)
+  if (last_of_unit(p, bg)) merge_unit<T, D, G, Q8>(p, bg, reinterpret_cast<float*>(dsm));
 }
 
 template <typename T, int D, bool Q8>
 __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) {
-  __shared__ float fac[kDecodeMaxG][kMaxChunks];  // 2^(chunk max - head max)
+  // [G][n_chunks] each: chunk max, then 2^(chunk max - head max); chunk sums
+  extern __shared__ float fin_smem[];
   __shared__ float lse[kDecodeMaxG], lh[kDecodeMaxG];
   __shared__ unsigned long long wmin[kWarps];
   __shared__ int is_last;
@@ -649,16 +631,28 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
   const float* part = p.part + static_cast<size_t>(bg) * p.part_ld * G * (D + 2);
   auto pidx = [&](int c, int h) { return (static_cast<size_t>(c) * G + h) * (D + 2); };
 
-  // ---- per-head log-sum-exp over the chunks (one warp per head)
+  // ---- per-head log-sum-exp over the chunks: the chunk statistics into
+  //      shared memory (every load in flight at once), then one warp per head
+  __shared__ float s_new;  // the new token's summed weight (its slice)
+  float* fac_ = fin_smem;
+  float* csum_ = fin_smem + G * NCk;
+  auto fac = [&](int h, int c) -> float& { return fac_[h * NCk + c]; };
+  auto csum = [&](int h, int c) -> float& { return csum_[h * NCk + c]; };
+  for (int i = tid; i < G * NCk; i += kThreads) {
+    const int h = i / NCk, c = i % NCk;
+    fac(h, c) = part[pidx(c, h) + D];
+    csum(h, c) = part[pidx(c, h) + D + 1];
+  }
+  __syncthreads();
   if (warp < G) {
     float m = -INFINITY;
-    for (int c = lane; c < NCk; c += 32) m = fmaxf(m, part[pidx(c, warp) + D]);
+    for (int c = lane; c < NCk; c += 32) m = fmaxf(m, fac(warp, c));
     m = warp_max(m);
     float l = 0.f;
     for (int c = lane; c < NCk; c += 32) {
-      const float f = ex2_approx(part[pidx(c, warp) + D] - m);
-      if (slice < o_slices) fac[warp][c] = f;
-      l = fmaf(part[pidx(c, warp) + D + 1], f, l);
+      const float f = ex2_approx(fac(warp, c) - m);
+      fac(warp, c) = f;
+      l = fmaf(csum(warp, c), f, l);
     }
     l = warp_sum(l);
     if (lane == 0) {
@@ -669,7 +663,9 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
   __syncthreads();
   if (slice < o_slices) {  // O: this CTA's share of the G*D outputs, tpo lanes
                           // per output (chunks strided over them, then a
-                          // fixed butterfly sum)
+                          // fixed butterfly sum); up to kO outputs per thread
+                          // at once, each with kB chunks of loads in flight
+    constexpr int kO = 4, kB = 8;
     T* out = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.Hkv * G + g * G) * D;
     const int GD = G * D;
     const int per = (GD + o_slices - 1) / o_slices;
@@ -677,42 +673,117 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
     int tpo = 1;
     while (tpo < 32 && 2 * tpo * per <= kThreads) tpo *= 2;
     const int cg = tid % tpo;
-    for (int base = o_begin; base < o_end; base += kThreads / tpo) {
-      const int i = base + tid / tpo;
-      const bool valid = i < o_end;
-      const int h = valid ? i / D : 0, d = valid ? i % D : 0;
-      float acc = 0.f;
-      if (valid) {
-#pragma unroll 4
-        for (int c = cg; c < NCk; c += tpo) acc = fmaf(part[pidx(c, h) + d], fac[h][c], acc);
+    const int stride = kThreads / tpo;
+    for (int base = o_begin; base < o_end; base += kO * stride) {
+      float acc[kO];
+      int hh[kO], dd[kO];
+      bool valid[kO];
+#pragma unroll
+      for (int r = 0; r < kO; ++r) {
+        const int i = base + r * stride + tid / tpo;
+        valid[r] = i < o_end;
+        hh[r] = valid[r] ? i / D : 0;
+        dd[r] = valid[r] ? i % D : 0;
+        acc[r] = 0.f;
       }
-      for (int o = tpo / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (valid && cg == 0) store(out + i, acc / lh[h]);
+      for (int c0 = cg; c0 < NCk; c0 += kB * tpo) {
+        float v[kB][kO];
+#pragma unroll
+        for (int u = 0; u < kB; ++u)
+#pragma unroll
+          for (int r = 0; r < kO; ++r) {
+            const int c = c0 + u * tpo;
+            v[u][r] = (valid[r] && c < NCk) ? part[pidx(c, hh[r]) + dd[r]] : 0.f;
+          }
+#pragma unroll
+        for (int u = 0; u < kB; ++u)
+#pragma unroll
+          for (int r = 0; r < kO; ++r) {
+            const int c = c0 + u * tpo;
+            if (valid[r] && c < NCk) acc[r] = fmaf(v[u][r], fac(hh[r], c), acc[r]);
+          }
+      }
+#pragma unroll
+      for (int r = 0; r < kO; ++r) {
+        float a = acc[r];
+        for (int o = tpo / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (valid[r] && cg == 0) store(out + base + r * stride + tid / tpo, a / lh[hh[r]]);
+      }
     }
   }
 
-  // ---- summed weights of this slice's keys: slots, then the new key at C
+  // ---- summed weights of this slice's keys (slots, then the new key at C),
+  //      with the score update and this thread's eviction candidate on the
+  //      way; every load of a thread's keys issued before any is used
   const float* lg = p.logits + static_cast<size_t>(bg) * G * (C + 1);
   float* cs = p.colsum + static_cast<size_t>(bg) * p.colsum_ld;
   const int ja = slice * kDecodeSliceKeys;
   const int jb = min(n + 1, ja + kDecodeSliceKeys);
-#pragma unroll 4
-  for (int j = ja + tid; j < jb; j += kThreads) {
-    float s = 0.f;
-    for (int h = 0; h < G; ++h) s += ex2_approx(lg[static_cast<size_t>(h) * (C + 1) + j] - lse[h]);
-    cs[j < n ? j : C] = s;
-  }
   const bool last_slice = slice == static_cast<int>(gridDim.x) - 1;
+  const bool by_score = p.policy == kPolicyH2O;
+  const int sinks = p.policy == kPolicySLR ? p.sinks : 0;
+  float* score = p.scores + static_cast<size_t>(bg) * C;
+  int* pos = p.pos + static_cast<size_t>(bg) * C;
+  const bool full = p.evict && n >= C;
+  // full: candidates.  Unprotected: position < t0 + 1 - W (and, under SLR,
+  // >= the sink count).  Key: rank value (the score as an order-preserving
+  // key, or the position) then the inverted index, so that the minimum is
+  // the lowest value with the highest index.
+  const long long limit = static_cast<long long>(p.t0) + 1 - p.W;
+  unsigned long long best = ~0ull;
+  {
+    constexpr int kK = kDecodeSliceKeys / kThreads;  // keys per thread
+    float x[kK][kDecodeMaxG], sc[kK];
+    int ps[kK];
+#pragma unroll
+    for (int u = 0; u < kK; ++u) {
+      const int j = ja + tid + u * kThreads;
+      const bool key = j < jb, slot = j < jb && j < n;
+#pragma unroll
+      for (int h = 0; h < kDecodeMaxG; ++h)
+        x[u][h] = (key && h < G) ? lg[static_cast<size_t>(h) * (C + 1) + j] : 0.f;
+      sc[u] = (slot && p.evict && by_score) ? score[j] : 0.f;
+      ps[u] = (slot && full) ? pos[j] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < kK; ++u) {
+      const int j = ja + tid + u * kThreads;
+      if (j >= jb) continue;
+      float sw = 0.f;
+#pragma unroll
+      for (int h = 0; h < kDecodeMaxG; ++h)
+        if (h < G) sw += ex2_approx(x[u][h] - lse[h]);
+      if (j == n) {
+        cs[C] = sw;
+        s_new = sw;
+        continue;
+      }
+      cs[j] = sw;
+      if (!p.evict) continue;
+      if (!full) {
+        if (by_score) score[j] = __fadd_rn(sc[u], sw);
+        continue;
+      }
+      uint32_t rank;
+      if (by_score) {
+        const float v = __fadd_rn(sc[u], sw);
+        score[j] = v;
+        rank = ordered_key(v);
+      } else {
+        rank = static_cast<uint32_t>(ps[u]);
+      }
+      if (ps[u] < limit && ps[u] >= sinks) {
+        const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - j);
+        best = key < best ? key : best;
+      }
+    }
+  }
   if (last_slice)  // empty slots received nothing
     for (int j = n + tid; j < C; j += kThreads) cs[j] = 0.f;
   if (!p.evict) return;
 
   // ---- eviction
-  __syncthreads();  // this CTA's summed weights are written
-  const bool by_score = p.policy == kPolicyH2O;
-  const int sinks = p.policy == kPolicySLR ? p.sinks : 0;
-  float* score = p.scores + static_cast<size_t>(bg) * C;
-  int* pos = p.pos + static_cast<size_t>(bg) * C;
+  __syncthreads();  // s_new
   const size_t row_bytes = static_cast<size_t>(D) * (Q8 ? 1 : sizeof(T));  // cache rows
   const size_t new_bytes = static_cast<size_t>(D) * sizeof(T);
   char* kc = static_cast<char*>(p.k_cache) + static_cast<size_t>(bg) * C * row_bytes;
@@ -738,42 +809,18 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
     p.state[0] = min(C, n + 1);
     p.state[1] = p.t0 + 1;
   }
-  const int sa = ja, sb = min(jb, n);  // this slice's valid slots
-  if (n < C) {  // room left: the new token takes slot n (key n is in the last slice)
-    if (by_score)
-      for (int s = sa + tid; s < sb; s += kThreads) score[s] = __fadd_rn(score[s], cs[s]);
+  if (!full) {  // room left: the new token takes slot n (key n is in the last slice)
     if (last_slice) {
       if (tid == 0) {
-        score[n] = by_score ? cs[C] : 0.f;
+        score[n] = by_score ? s_new : 0.f;
         pos[n] = p.t0;
       }
       if (warp == 0) place_new(n);
     }
     return;
   }
-  // full: this slice's candidate.  Unprotected: position < t0 + 1 - W (and,
-  // under SLR, >= the sink count).  Key: rank value (the score as an
-  // order-preserving key, or the position) then the inverted index, so that
-  // the minimum is the lowest value with the highest index.
-  const long long limit = static_cast<long long>(p.t0) + 1 - p.W;
-  unsigned long long best = ~0ull;
-  for (int s = sa + tid; s < sb; s += kThreads) {
-    const int ps = pos[s];
-    uint32_t rank;
-    if (by_score) {
-      const float sc = __fadd_rn(score[s], cs[s]);
-      score[s] = sc;
-      rank = ordered_key(sc);
-    } else {
-      rank = static_cast<uint32_t>(ps);
-    }
-    if (ps < limit && ps >= sinks) {
-      const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - s);
-      best = key < best ? key : best;
-    }
-  }
   if (last_slice && tid == 0 && p.t0 < limit && p.t0 >= sinks) {  // W = 0: the new token competes
-    const uint32_t rank = by_score ? ordered_key(cs[C]) : static_cast<uint32_t>(p.t0);
+    const uint32_t rank = by_score ? ordered_key(s_new) : static_cast<uint32_t>(p.t0);
     const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - C);
     best = key < best ? key : best;
   }
@@ -814,35 +861,15 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
 }
 
 // One launch per step (the merge in each unit's last CTA) or two (a merge
-// kernel over slices of the keys); with one launch, one CTA per chunk or one
-// streaming CTA per SM.
-constexpr bool kDecodeFused = true;
-constexpr bool kDecodeStream = true;
-
-template <typename T, int D, int G, bool Q8>
-cudaError_t launch_stream(const DecodeParams& p, cudaStream_t st) {
-  using L = StreamLayout<T, D, G, Q8>;
-  static int attr_bits[2] = {0, 0};
-  const void* fn = reinterpret_cast<const void*>(decode_stream<T, D, G, Q8>);
-  cudaError_t e = ensure_smem_attr(fn, L::kBytes, attr_bits);
-  if (e != cudaSuccess) return e;
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0, v = 0;
-    e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    sms = v;
-  }
-  const long long total = static_cast<long long>(p.B) * p.Hkv * p.n_chunks;
-  const int grid = static_cast<int>(total < sms ? total : sms);
-  decode_stream<T, D, G, Q8><<<grid, kThreads, L::kBytes, st>>>(p);
-  return cudaGetLastError();
-}
+// kernel over slices of the keys).  Measured on one Qwen-shaped cache (C 8192,
+// 8 KV heads): 47.1 us with one launch against 31.7 us with two -- one CTA per
+// (cache, KV head) merging 8193 keys is slower than 72 CTAs behind a
+// programmatic dependent launch -- and 1719 against 1680 us on 144 caches;
+// so two.
+constexpr bool kDecodeFused = false;
 
 template <typename T, int D, int G, bool Q8>
 cudaError_t launch_partial(const DecodeParams& p, cudaStream_t st) {
-  if (kDecodeFused && kDecodeStream) return launch_stream<T, D, G, Q8>(p, st);
   using L = PartialLayout<T, D, G, Q8>;
   static int attr_bits[2] = {0, 0};
   const void* fn = reinterpret_cast<const void*>(decode_partial<T, D, G, Q8, kDecodeFused>);
@@ -864,10 +891,14 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess || kDecodeFused) return e;
+  static int attr_bits[2] = {0, 0};
+  e = ensure_smem_attr(reinterpret_cast<const void*>(decode_finish<T, D, Q8>),
+                       2 * kDecodeMaxG * kMaxChunks * 4, attr_bits);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.n_slices, p.B * p.Hkv);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = 2 * p.G * p.n_chunks * 4;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -146,6 +146,7 @@ __device__ __forceinline__ void place_rows(const EvictParams& e, int b, int g, i
 }
 
 constexpr int kLoadBatch = 8;  // global loads in flight per thread in the first pass
+constexpr int kVecBatch = 2;   // 16-byte loads per array in flight per thread (four slots each)
 constexpr int kBins = 256;     // radix passes of 8 bits, most significant first
 
 // What the selection of one (cache, KV head) needs to know.
@@ -333,7 +334,48 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
   //    count (for the shortcut below).
   uint32_t old_min = 0xFFFFFFFFu, new_max = 0u;
   int n_prot = 0;
-  for (int x0 = tid; x0 < n; x0 += kLoadBatch * NT) {
+  // the old slots four at a time (16-byte loads and stores) when the unit's
+  // scores, summed weights and positions are 16-byte aligned; the rest below
+  const bool vec = ((reinterpret_cast<uintptr_t>(score) | reinterpret_cast<uintptr_t>(cs) |
+                     reinterpret_cast<uintptr_t>(pos)) & 15) == 0;
+  const int n_vec = vec ? (n & ~3) : 0;
+  for (int v0 = tid; 4 * v0 < n_vec; v0 += kVecBatch * NT) {
+    float4 sc[kVecBatch], cv[kVecBatch];
+    int4 ps[kVecBatch];
+#pragma unroll
+    for (int k = 0; k < kVecBatch; ++k) {
+      const int v = v0 + k * NT;
+      sc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      cv[k] = sc[k];
+      ps[k] = make_int4(-1, -1, -1, -1);
+      if (4 * v < n_vec) {
+        if (by_score) {
+          sc[k] = reinterpret_cast<const float4*>(score)[v];
+          cv[k] = reinterpret_cast<const float4*>(cs)[v];
+        }
+        if (need_pos) ps[k] = reinterpret_cast<const int4*>(pos)[v];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kVecBatch; ++k) {
+      const int v = v0 + k * NT;
+      if (4 * v >= n_vec) continue;
+      const float s4[4] = {sc[k].x + cv[k].x, sc[k].y + cv[k].y, sc[k].z + cv[k].z,
+                           sc[k].w + cv[k].w};
+      const int p4[4] = {ps[k].x, ps[k].y, ps[k].z, ps[k].w};
+      uint32_t key4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool prot = old_protectable && (p4[e] >= limit || p4[e] < sinks);
+        const uint32_t key = by_score ? score_key(s4[e]) : static_cast<uint32_t>(p4[e]);
+        key4[e] = prot ? kProtectedKey : key;
+        if (prot) ++n_prot; else old_min = min(old_min, key);
+      }
+      if (by_score) reinterpret_cast<float4*>(score)[v] = make_float4(s4[0], s4[1], s4[2], s4[3]);
+      reinterpret_cast<uint4*>(keys)[v] = make_uint4(key4[0], key4[1], key4[2], key4[3]);
+    }
+  }
+  for (int x0 = n_vec + tid; x0 < n; x0 += kLoadBatch * NT) {
     float sc[kLoadBatch], cv[kLoadBatch];
     int ps[kLoadBatch];
 #pragma unroll

@@ -45,7 +45,7 @@ struct h2o_cache {
   float* dec_logits = nullptr;  // decode: [B*Hkv, G, C + 1]
   float* dec_part = nullptr;    // decode: [B*Hkv, dec_part_ld, G, d + 2]
   int dec_part_ld = 0;
-  float* dsum = nullptr;  // backward: D_i = <dO_i, O_i>, [B, Hq, nq_pad]
+  float* dsum = nullptr;  // backward: -scale * D_i, D_i = <dO_i, O_i>, [B, Hq, nq_pad]
   int fwd_nq = 0;         // n_q of the last attention whose row statistics are
   int fwd_n = -1;         // in the workspace, and the valid slots it saw
   unsigned long long* dec_best = nullptr;  // decode: [B*Hkv, dec_slices_ld]

@@ -64,8 +64,8 @@ def test_policy_step_matches_oracle(case):
         launches0 = gpu.info()["kernel_launches"]
         O = gpu.step(q.cuda(), kn.cuda(), vn.cuda())
         # no summed weights asked for: the column-sum kernel is skipped (a
-        # decode step is one launch either way)
-        assert gpu.info()["kernel_launches"] - launches0 == (1 if nq == 1 else 2)
+        # decode step is two launches either way)
+        assert gpu.info()["kernel_launches"] - launches0 == 2
         O_ref, _ = ref.step(gh.np64(q), gh.np64(kn), gh.np64(vn))
         assert float(np.max(np.abs(gh.np64(O) - O_ref))) <= gh.O_TOL
         gh.assert_state_equal(gpu.read(), ref, shape.dtype, f"{case} step {step}")
