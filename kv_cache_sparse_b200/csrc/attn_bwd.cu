@@ -91,13 +91,13 @@ constexpr int kBwdThreads = 64 + 2 * 128;
 // in nds, either per column (kCol: 32 floats each in shared memory, read 16
 // bytes at a time) or one value for the whole row (nls[0], nds[0]).  Pairs
 // of columns go through packed f32x2 arithmetic.
-template <bool kMask, bool kCol>
-__device__ __forceinline__ void p_ds_32(const uint32_t (&s)[32], const uint32_t (&dp)[32],
-                                        const float* nls, const float* nds, float c, float scale,
-                                        int first_valid, int last_valid, uint32_t (&pp)[16],
-                                        uint32_t (&dd)[16]) {
+template <int NV, bool kMask, bool kCol>
+__device__ __forceinline__ void p_ds(const uint32_t (&s)[NV], const uint32_t (&dp)[NV],
+                                     const float* nls, const float* nds, float c, float scale,
+                                     int first_valid, int last_valid, uint32_t (&pp)[NV / 2],
+                                     uint32_t (&dd)[NV / 2]) {
 #pragma unroll
-  for (int k = 0; k < 32; k += 4) {
+  for (int k = 0; k < NV; k += 4) {
     float4 nl, nd;
     if (kCol) {
       nl = *reinterpret_cast<const float4*>(nls + k);
@@ -127,6 +127,47 @@ __device__ __forceinline__ void p_ds_32(const uint32_t (&s)[32], const uint32_t 
     pp[(k >> 1) + 1] = pack_bf16x2(p2, p3);
     dd[k >> 1] = pack_bf16x2(d0, d1);
     dd[(k >> 1) + 1] = pack_bf16x2(d2, d3);
+  }
+}
+
+// The row work of one half (64 columns) of a unit's S and dP in TMEM (S at
+// s_col, dP at s_col + 128, the half's columns starting at c0): four
+// sub-blocks of 16 columns, the TMEM loads of the next issued before the
+// arithmetic of the current one, so that they overlap it; the bf16 pairs of
+// sub-block k go over columns [c0 + 8k, +8) of S (P) and of dP (scale dS)
+// -- or, kDsOverS, scale dS over S and P nowhere -- which hold values
+// already read.  Column statistics at nls / nds (per column, kCol) or the
+// row's own (nls[0], nds[0]); masking as in p_ds.
+template <bool kCol, bool kDsOverS>
+__device__ __forceinline__ void half_rows(uint32_t s_col, int c0, const float* nls,
+                                          const float* nds, float c, float scale, bool masked,
+                                          int first_valid, int last_valid) {
+  uint32_t sv[2][16], dp[2][16];
+  tmem_ld16(s_col + c0, sv[0]);
+  tmem_ld16(s_col + 128 + c0, dp[0]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int cur = k & 1;
+    if (k < 3) {
+      tmem_ld16(s_col + c0 + 16 * (k + 1), sv[cur ^ 1]);
+      tmem_ld16(s_col + 128 + c0 + 16 * (k + 1), dp[cur ^ 1]);
+    }
+    uint32_t pp[8], dd[8];
+    const float* nl = kCol ? nls + 16 * k : nls;
+    const float* nd = kCol ? nds + 16 * k : nds;
+    if (masked)
+      p_ds<16, true, kCol>(sv[cur], dp[cur], nl, nd, c, scale, first_valid - 16 * k,
+                           last_valid - 16 * k, pp, dd);
+    else
+      p_ds<16, false, kCol>(sv[cur], dp[cur], nl, nd, c, scale, 0, 0, pp, dd);
+    if (kDsOverS) {
+      tmem_st8(s_col + c0 + 8 * k, dd);
+    } else {
+      tmem_st8(s_col + c0 + 8 * k, pp);
+      tmem_st8(s_col + 128 + c0 + 8 * k, dd);
+    }
+    if (k < 3) tmem_wait_ld();
   }
 }
 
@@ -330,23 +371,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float* nds = nls + 128;
       const int qt = qt_min + u % span;
       const bool diag = is_chunk && qt == kt;  // query col sees key row iff row <= col
-#pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
-        const int q32 = 2 * hf + q2;
-        uint32_t sv[32], dp[32], pp[16], dd[16];
-        tmem_ld32(lane_base + 32 * q32, sv);
-        tmem_ld32(lane_base + 128 + 32 * q32, dp);
-        tmem_wait_ld();
-        if (diag)
-          p_ds_32<true, true>(sv, dp, nls + 32 * q32, nds + 32 * q32, c, scale, row - 32 * q32,
-                              1 << 30, pp, dd);
-        else
-          p_ds_32<false, true>(sv, dp, nls + 32 * q32, nds + 32 * q32, c, scale, 0, 0, pp, dd);
-        // bf16 pairs over the half's first columns: queries [32 q32, +32) ->
-        // columns [64 hf + 16 q2, +16)
-        tmem_st16(lane_base + 64 * hf + 16 * q2, pp);
-        tmem_st16(lane_base + 128 + 64 * hf + 16 * q2, dd);
-      }
+      // queries [64 hf, +64); bf16 pairs over the half's first 32 columns
+      half_rows<true, false>(lane_base, 64 * hf, nls + 64 * hf, nds + 64 * hf, c, scale, diag,
+                      row - 64 * hf, 1 << 30);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p0 + 8 * hf);
@@ -602,20 +629,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         masked = true;
         last = row;
       }
-#pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
-        const int q32 = 2 * hf + q2;
-        uint32_t sv[32], dp[32], pp[16], dd[16];
-        tmem_ld32(lane_base + 32 * q32, sv);
-        tmem_ld32(lane_base + 128 + 32 * q32, dp);
-        tmem_wait_ld();
-        if (masked)
-          p_ds_32<true, false>(sv, dp, nls, nds, c, scale, 0, last - 32 * q32, pp, dd);
-        else
-          p_ds_32<false, false>(sv, dp, nls, nds, c, scale, 0, 0, pp, dd);
-        // scale*dS over S: keys [32 q32, +32) -> columns [64 hf + 16 q2, +16)
-        tmem_st16(lane_base + 64 * hf + 16 * q2, dd);
-      }
+      // keys [64 hf, +64); scale*dS over S's half (P over dP's, unused)
+      half_rows<false, true>(lane_base, 64 * hf, nls, nds, c, scale, masked, 0, last - 64 * hf);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p0 + 8 * hf);
