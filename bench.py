@@ -91,6 +91,12 @@ def recorded_traffic(kernel: str, workload: str):
         return None
 
 
+def workload_of(args):
+    """The named workload, with --caches caches when given."""
+    wl = WORKLOADS[args.workload]
+    return wl.scaled(batch=args.caches) if args.caches > 0 else wl
+
+
 def attention_flops(wl, n, nq):
     """Algorithmic FLOPs of one step's attention: QK^T and PV over the
     visible (query, key) pairs, 2*d each, for every query head and cache."""
@@ -319,7 +325,7 @@ def run_ours(args, world, rank, local):
     barrier(world)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    wl = WORKLOADS[args.workload]
+    wl = workload_of(args)
     shape = binding.CacheShape(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim,
                                wl.capacity, wl.max_chunk, wl.window, wl.cache_dtype(), 0.0,
                                wl.policy, wl.sinks)
@@ -583,7 +589,7 @@ def run_reference(args, world, rank):
     independent KV groups as fit a ~120 s budget for the whole run."""
     if rank != 0:
         return None
-    wl = WORKLOADS[args.workload]
+    wl = workload_of(args)
     t1, _ = oracle_sample(wl, 1, seed=100, groups=1)       # one group, to size the sample
     budget = 120.0 / max(1, args.steps + args.warmup)
     groups = int(max(1, min(wl.n_kv_heads, budget // max(t1, 1e-3))))
@@ -623,6 +629,9 @@ def main():
     ap.add_argument("--cpu-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WL.name, choices=list(WORKLOADS))
+    ap.add_argument("--caches", type=int, default=0,
+                    help="run the workload with this many caches instead of its own count "
+                         "(a smaller case of the same kernels, for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")

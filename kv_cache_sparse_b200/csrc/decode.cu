@@ -612,8 +612,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_partial(const DecodeParams
 
 template <typename T, int D, bool Q8>
 __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) {
-  // [G][n_chunks] each: chunk max, then 2^(chunk max - head max); chunk sums
-  extern __shared__ float fin_smem[];
+  __shared__ float fac[kDecodeMaxG][kMaxChunks];  // 2^(chunk max - head max)
   __shared__ float lse[kDecodeMaxG], lh[kDecodeMaxG];
   __shared__ unsigned long long wmin[kWarps];
   __shared__ int is_last;
@@ -631,28 +630,16 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
   const float* part = p.part + static_cast<size_t>(bg) * p.part_ld * G * (D + 2);
   auto pidx = [&](int c, int h) { return (static_cast<size_t>(c) * G + h) * (D + 2); };
 
-  // ---- per-head log-sum-exp over the chunks: the chunk statistics into
-  //      shared memory (every load in flight at once), then one warp per head
-  __shared__ float s_new;  // the new token's summed weight (its slice)
-  float* fac_ = fin_smem;
-  float* csum_ = fin_smem + G * NCk;
-  auto fac = [&](int h, int c) -> float& { return fac_[h * NCk + c]; };
-  auto csum = [&](int h, int c) -> float& { return csum_[h * NCk + c]; };
-  for (int i = tid; i < G * NCk; i += kThreads) {
-    const int h = i / NCk, c = i % NCk;
-    fac(h, c) = part[pidx(c, h) + D];
-    csum(h, c) = part[pidx(c, h) + D + 1];
-  }
-  __syncthreads();
+  // ---- per-head log-sum-exp over the chunks (one warp per head)
   if (warp < G) {
     float m = -INFINITY;
-    for (int c = lane; c < NCk; c += 32) m = fmaxf(m, fac(warp, c));
+    for (int c = lane; c < NCk; c += 32) m = fmaxf(m, part[pidx(c, warp) + D]);
     m = warp_max(m);
     float l = 0.f;
     for (int c = lane; c < NCk; c += 32) {
-      const float f = ex2_approx(fac(warp, c) - m);
-      fac(warp, c) = f;
-      l = fmaf(csum(warp, c), f, l);
+      const float f = ex2_approx(part[pidx(c, warp) + D] - m);
+      if (slice < o_slices) fac[warp][c] = f;
+      l = fmaf(part[pidx(c, warp) + D + 1], f, l);
     }
     l = warp_sum(l);
     if (lane == 0) {
@@ -663,9 +650,7 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
   __syncthreads();
   if (slice < o_slices) {  // O: this CTA's share of the G*D outputs, tpo lanes
                           // per output (chunks strided over them, then a
-                          // fixed butterfly sum); up to kO outputs per thread
-                          // at once, each with kB chunks of loads in flight
-    constexpr int kO = 4, kB = 8;
+                          // fixed butterfly sum)
     T* out = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.Hkv * G + g * G) * D;
     const int GD = G * D;
     const int per = (GD + o_slices - 1) / o_slices;
@@ -673,117 +658,42 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
     int tpo = 1;
     while (tpo < 32 && 2 * tpo * per <= kThreads) tpo *= 2;
     const int cg = tid % tpo;
-    const int stride = kThreads / tpo;
-    for (int base = o_begin; base < o_end; base += kO * stride) {
-      float acc[kO];
-      int hh[kO], dd[kO];
-      bool valid[kO];
-#pragma unroll
-      for (int r = 0; r < kO; ++r) {
-        const int i = base + r * stride + tid / tpo;
-        valid[r] = i < o_end;
-        hh[r] = valid[r] ? i / D : 0;
-        dd[r] = valid[r] ? i % D : 0;
-        acc[r] = 0.f;
+    for (int base = o_begin; base < o_end; base += kThreads / tpo) {
+      const int i = base + tid / tpo;
+      const bool valid = i < o_end;
+      const int h = valid ? i / D : 0, d = valid ? i % D : 0;
+      float acc = 0.f;
+      if (valid) {
+#pragma unroll 4
+        for (int c = cg; c < NCk; c += tpo) acc = fmaf(part[pidx(c, h) + d], fac[h][c], acc);
       }
-      for (int c0 = cg; c0 < NCk; c0 += kB * tpo) {
-        float v[kB][kO];
-#pragma unroll
-        for (int u = 0; u < kB; ++u)
-#pragma unroll
-          for (int r = 0; r < kO; ++r) {
-            const int c = c0 + u * tpo;
-            v[u][r] = (valid[r] && c < NCk) ? part[pidx(c, hh[r]) + dd[r]] : 0.f;
-          }
-#pragma unroll
-        for (int u = 0; u < kB; ++u)
-#pragma unroll
-          for (int r = 0; r < kO; ++r) {
-            const int c = c0 + u * tpo;
-            if (valid[r] && c < NCk) acc[r] = fmaf(v[u][r], fac(hh[r], c), acc[r]);
-          }
-      }
-#pragma unroll
-      for (int r = 0; r < kO; ++r) {
-        float a = acc[r];
-        for (int o = tpo / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (valid[r] && cg == 0) store(out + base + r * stride + tid / tpo, a / lh[hh[r]]);
-      }
+      for (int o = tpo / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (valid && cg == 0) store(out + i, acc / lh[h]);
     }
   }
 
-  // ---- summed weights of this slice's keys (slots, then the new key at C),
-  //      with the score update and this thread's eviction candidate on the
-  //      way; every load of a thread's keys issued before any is used
+  // ---- summed weights of this slice's keys: slots, then the new key at C
   const float* lg = p.logits + static_cast<size_t>(bg) * G * (C + 1);
   float* cs = p.colsum + static_cast<size_t>(bg) * p.colsum_ld;
   const int ja = slice * kDecodeSliceKeys;
   const int jb = min(n + 1, ja + kDecodeSliceKeys);
-  const bool last_slice = slice == static_cast<int>(gridDim.x) - 1;
-  const bool by_score = p.policy == kPolicyH2O;
-  const int sinks = p.policy == kPolicySLR ? p.sinks : 0;
-  float* score = p.scores + static_cast<size_t>(bg) * C;
-  int* pos = p.pos + static_cast<size_t>(bg) * C;
-  const bool full = p.evict && n >= C;
-  // full: candidates.  Unprotected: position < t0 + 1 - W (and, under SLR,
-  // >= the sink count).  Key: rank value (the score as an order-preserving
-  // key, or the position) then the inverted index, so that the minimum is
-  // the lowest value with the highest index.
-  const long long limit = static_cast<long long>(p.t0) + 1 - p.W;
-  unsigned long long best = ~0ull;
-  {
-    constexpr int kK = kDecodeSliceKeys / kThreads;  // keys per thread
-    float x[kK][kDecodeMaxG], sc[kK];
-    int ps[kK];
-#pragma unroll
-    for (int u = 0; u < kK; ++u) {
-      const int j = ja + tid + u * kThreads;
-      const bool key = j < jb, slot = j < jb && j < n;
-#pragma unroll
-      for (int h = 0; h < kDecodeMaxG; ++h)
-        x[u][h] = (key && h < G) ? lg[static_cast<size_t>(h) * (C + 1) + j] : 0.f;
-      sc[u] = (slot && p.evict && by_score) ? score[j] : 0.f;
-      ps[u] = (slot && full) ? pos[j] : 0;
-    }
-#pragma unroll
-    for (int u = 0; u < kK; ++u) {
-      const int j = ja + tid + u * kThreads;
-      if (j >= jb) continue;
-      float sw = 0.f;
-#pragma unroll
-      for (int h = 0; h < kDecodeMaxG; ++h)
-        if (h < G) sw += ex2_approx(x[u][h] - lse[h]);
-      if (j == n) {
-        cs[C] = sw;
-        s_new = sw;
-        continue;
-      }
-      cs[j] = sw;
-      if (!p.evict) continue;
-      if (!full) {
-        if (by_score) score[j] = __fadd_rn(sc[u], sw);
-        continue;
-      }
-      uint32_t rank;
-      if (by_score) {
-        const float v = __fadd_rn(sc[u], sw);
-        score[j] = v;
-        rank = ordered_key(v);
-      } else {
-        rank = static_cast<uint32_t>(ps[u]);
-      }
-      if (ps[u] < limit && ps[u] >= sinks) {
-        const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - j);
-        best = key < best ? key : best;
-      }
-    }
+#pragma unroll 4
+  for (int j = ja + tid; j < jb; j += kThreads) {
+    float s = 0.f;
+    for (int h = 0; h < G; ++h) s += ex2_approx(lg[static_cast<size_t>(h) * (C + 1) + j] - lse[h]);
+    cs[j < n ? j : C] = s;
   }
+  const bool last_slice = slice == static_cast<int>(gridDim.x) - 1;
   if (last_slice)  // empty slots received nothing
     for (int j = n + tid; j < C; j += kThreads) cs[j] = 0.f;
   if (!p.evict) return;
 
   // ---- eviction
-  __syncthreads();  // s_new
+  __syncthreads();  // this CTA's summed weights are written
+  const bool by_score = p.policy == kPolicyH2O;
+  const int sinks = p.policy == kPolicySLR ? p.sinks : 0;
+  float* score = p.scores + static_cast<size_t>(bg) * C;
+  int* pos = p.pos + static_cast<size_t>(bg) * C;
   const size_t row_bytes = static_cast<size_t>(D) * (Q8 ? 1 : sizeof(T));  // cache rows
   const size_t new_bytes = static_cast<size_t>(D) * sizeof(T);
   char* kc = static_cast<char*>(p.k_cache) + static_cast<size_t>(bg) * C * row_bytes;
@@ -809,18 +719,42 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
     p.state[0] = min(C, n + 1);
     p.state[1] = p.t0 + 1;
   }
-  if (!full) {  // room left: the new token takes slot n (key n is in the last slice)
+  const int sa = ja, sb = min(jb, n);  // this slice's valid slots
+  if (n < C) {  // room left: the new token takes slot n (key n is in the last slice)
+    if (by_score)
+      for (int s = sa + tid; s < sb; s += kThreads) score[s] = __fadd_rn(score[s], cs[s]);
     if (last_slice) {
       if (tid == 0) {
-        score[n] = by_score ? s_new : 0.f;
+        score[n] = by_score ? cs[C] : 0.f;
         pos[n] = p.t0;
       }
       if (warp == 0) place_new(n);
     }
     return;
   }
+  // full: this slice's candidate.  Unprotected: position < t0 + 1 - W (and,
+  // under SLR, >= the sink count).  Key: rank value (the score as an
+  // order-preserving key, or the position) then the inverted index, so that
+  // the minimum is the lowest value with the highest index.
+  const long long limit = static_cast<long long>(p.t0) + 1 - p.W;
+  unsigned long long best = ~0ull;
+  for (int s = sa + tid; s < sb; s += kThreads) {
+    const int ps = pos[s];
+    uint32_t rank;
+    if (by_score) {
+      const float sc = __fadd_rn(score[s], cs[s]);
+      score[s] = sc;
+      rank = ordered_key(sc);
+    } else {
+      rank = static_cast<uint32_t>(ps);
+    }
+    if (ps < limit && ps >= sinks) {
+      const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - s);
+      best = key < best ? key : best;
+    }
+  }
   if (last_slice && tid == 0 && p.t0 < limit && p.t0 >= sinks) {  // W = 0: the new token competes
-    const uint32_t rank = by_score ? ordered_key(s_new) : static_cast<uint32_t>(p.t0);
+    const uint32_t rank = by_score ? ordered_key(cs[C]) : static_cast<uint32_t>(p.t0);
     const unsigned long long key = (static_cast<unsigned long long>(rank) << 32) | (0xffffffffu - C);
     best = key < best ? key : best;
   }
@@ -891,14 +825,10 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess || kDecodeFused) return e;
-  static int attr_bits[2] = {0, 0};
-  e = ensure_smem_attr(reinterpret_cast<const void*>(decode_finish<T, D, Q8>),
-                       2 * kDecodeMaxG * kMaxChunks * 4, attr_bits);
-  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.n_slices, p.B * p.Hkv);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = 2 * p.G * p.n_chunks * 4;
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -290,6 +290,58 @@ __device__ __forceinline__ void find_bin_block(const int* hist, int nbins, int k
   }
 }
 
+// Step 1 for the old slots [0, n_vec), four at a time (16-byte loads and
+// stores): accumulates their scores, writes their keys, and tracks the lowest
+// unprotected key and the protected count.  kB 16-byte loads per array in
+// flight per thread; kPos: the positions are needed (the score-free
+// policies, or a window or sinks that can protect an old slot).
+template <int NT, int kB, bool kPos>
+__device__ __forceinline__ void vec_pass(float* __restrict__ score, const float* __restrict__ cs,
+                                         const int* __restrict__ pos, uint32_t* keys, int n_vec,
+                                         bool by_score, bool old_protectable, long long limit,
+                                         int sinks, uint32_t& old_min, int& n_prot) {
+  const int tid = threadIdx.x;
+  for (int v0 = tid; 4 * v0 < n_vec; v0 += kB * NT) {
+    float4 sc[kB], cv[kB];
+    int4 ps[kPos ? kB : 1];
+#pragma unroll
+    for (int k = 0; k < kB; ++k) {
+      const int v = v0 + k * NT;
+      sc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      cv[k] = sc[k];
+      if (kPos) ps[k] = make_int4(-1, -1, -1, -1);
+      if (4 * v < n_vec) {
+        if (by_score) {
+          sc[k] = reinterpret_cast<const float4*>(score)[v];
+          cv[k] = reinterpret_cast<const float4*>(cs)[v];
+        }
+        if (kPos) ps[k] = reinterpret_cast<const int4*>(pos)[v];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kB; ++k) {
+      const int v = v0 + k * NT;
+      if (4 * v >= n_vec) continue;
+      const float s4[4] = {sc[k].x + cv[k].x, sc[k].y + cv[k].y, sc[k].z + cv[k].z,
+                           sc[k].w + cv[k].w};
+      int p4[4] = {-1, -1, -1, -1};
+      if (kPos) {
+        p4[0] = ps[k].x; p4[1] = ps[k].y; p4[2] = ps[k].z; p4[3] = ps[k].w;
+      }
+      uint32_t key4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool prot = kPos && old_protectable && (p4[e] >= limit || p4[e] < sinks);
+        const uint32_t key = by_score ? score_key(s4[e]) : static_cast<uint32_t>(p4[e]);
+        key4[e] = prot ? kProtectedKey : key;
+        if (prot) ++n_prot; else old_min = min(old_min, key);
+      }
+      if (by_score) reinterpret_cast<float4*>(score)[v] = make_float4(s4[0], s4[1], s4[2], s4[3]);
+      reinterpret_cast<uint4*>(keys)[v] = make_uint4(key4[0], key4[1], key4[2], key4[3]);
+    }
+  }
+}
+
 template <int NT>
 __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
     h2o_select(const EvictParams e, int plan_smem) {
@@ -339,42 +391,12 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
   const bool vec = ((reinterpret_cast<uintptr_t>(score) | reinterpret_cast<uintptr_t>(cs) |
                      reinterpret_cast<uintptr_t>(pos)) & 15) == 0;
   const int n_vec = vec ? (n & ~3) : 0;
-  for (int v0 = tid; 4 * v0 < n_vec; v0 += kVecBatch * NT) {
-    float4 sc[kVecBatch], cv[kVecBatch];
-    int4 ps[kVecBatch];
-#pragma unroll
-    for (int k = 0; k < kVecBatch; ++k) {
-      const int v = v0 + k * NT;
-      sc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-      cv[k] = sc[k];
-      ps[k] = make_int4(-1, -1, -1, -1);
-      if (4 * v < n_vec) {
-        if (by_score) {
-          sc[k] = reinterpret_cast<const float4*>(score)[v];
-          cv[k] = reinterpret_cast<const float4*>(cs)[v];
-        }
-        if (need_pos) ps[k] = reinterpret_cast<const int4*>(pos)[v];
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < kVecBatch; ++k) {
-      const int v = v0 + k * NT;
-      if (4 * v >= n_vec) continue;
-      const float s4[4] = {sc[k].x + cv[k].x, sc[k].y + cv[k].y, sc[k].z + cv[k].z,
-                           sc[k].w + cv[k].w};
-      const int p4[4] = {ps[k].x, ps[k].y, ps[k].z, ps[k].w};
-      uint32_t key4[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const bool prot = old_protectable && (p4[e] >= limit || p4[e] < sinks);
-        const uint32_t key = by_score ? score_key(s4[e]) : static_cast<uint32_t>(p4[e]);
-        key4[e] = prot ? kProtectedKey : key;
-        if (prot) ++n_prot; else old_min = min(old_min, key);
-      }
-      if (by_score) reinterpret_cast<float4*>(score)[v] = make_float4(s4[0], s4[1], s4[2], s4[3]);
-      reinterpret_cast<uint4*>(keys)[v] = make_uint4(key4[0], key4[1], key4[2], key4[3]);
-    }
-  }
+  if (need_pos)
+    vec_pass<NT, kVecBatch, true>(score, cs, pos, keys, n_vec, by_score, old_protectable, limit,
+                                  sinks, old_min, n_prot);
+  else
+    vec_pass<NT, 2 * kVecBatch, false>(score, cs, pos, keys, n_vec, by_score, old_protectable,
+                                       limit, sinks, old_min, n_prot);
   for (int x0 = n_vec + tid; x0 < n; x0 += kLoadBatch * NT) {
     float sc[kLoadBatch], cv[kLoadBatch];
     int ps[kLoadBatch];
