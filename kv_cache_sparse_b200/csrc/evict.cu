@@ -147,6 +147,7 @@ __device__ __forceinline__ void place_rows(const EvictParams& e, int b, int g, i
 
 constexpr int kLoadBatch = 8;  // global loads in flight per thread in the first pass
 constexpr int kVecBatch = 2;   // 16-byte loads per array in flight per thread (four slots each)
+constexpr int kNewPre = 4;     // new tokens' summed weights loaded per thread before the old slots
 constexpr int kBins = 256;     // radix passes of 8 bits, most significant first
 
 // What the selection of one (cache, KV head) needs to know.
@@ -391,6 +392,14 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
   const bool vec = ((reinterpret_cast<uintptr_t>(score) | reinterpret_cast<uintptr_t>(cs) |
                      reinterpret_cast<uintptr_t>(pos)) & 15) == 0;
   const int n_vec = vec ? (n & ~3) : 0;
+  // the new tokens' summed weights (the first kNewPre per thread) are loaded
+  // now, so that their latency overlaps the old slots' pass
+  float cv_pre[kNewPre];
+#pragma unroll
+  for (int k = 0; k < kNewPre; ++k) {
+    const int i = tid + k * NT;
+    cv_pre[k] = (by_score && i < nq) ? cs[C + i] : 0.f;
+  }
   if (need_pos)
     vec_pass<NT, kVecBatch, true>(score, cs, pos, keys, n_vec, by_score, old_protectable, limit,
                                   sinks, old_min, n_prot);
@@ -432,7 +441,18 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? 4 : 1))
       }
     }
   }
-  for (int i0 = tid; i0 < nq; i0 += kLoadBatch * NT) {
+#pragma unroll
+  for (int k = 0; k < kNewPre; ++k) {
+    const int i = tid + k * NT;
+    if (i < nq) {
+      const long long p = static_cast<long long>(e.t0) + i;
+      const bool prot = evict && (p >= limit || p < sinks);
+      const uint32_t key = by_score ? score_key(cv_pre[k]) : static_cast<uint32_t>(p);
+      keys[n + i] = prot ? kProtectedKey : key;
+      if (prot) ++n_prot; else new_max = max(new_max, key);
+    }
+  }
+  for (int i0 = kNewPre * NT + tid; i0 < nq; i0 += kLoadBatch * NT) {
     float cv[kLoadBatch];
 #pragma unroll
     for (int k = 0; k < kLoadBatch; ++k) {
