@@ -119,6 +119,41 @@ __device__ __forceinline__ void sum_tile(const uint32_t (&v0)[32], const uint32_
   }
 }
 
+// 32 columns: the same arithmetic as sum_tile on one 32-column piece.
+template <bool kDiag>
+__device__ __forceinline__ void sum_piece(const uint32_t (&v)[32], const float4* nlse4, float c,
+                                          int first_col, float (&part)[4]) {
+#pragma unroll
+  for (int q4 = 0; q4 < 8; ++q4) {
+    const float4 nl = nlse4[q4];
+    const int col = q4 * 4;
+    float x0, x1, x2, x3;
+    ffma2(x0, x1, __uint_as_float(v[col]), __uint_as_float(v[col + 1]), c, c, nl.x, nl.y);
+    ffma2(x2, x3, __uint_as_float(v[col + 2]), __uint_as_float(v[col + 3]), c, c, nl.z, nl.w);
+    float p0, p1, p2, p3;
+    if (((2 * q4) & 7) < kEmuPairsOf8) {
+      exp2_fma2(p0, p1, x0, x1);
+    } else {
+      p0 = ex2_approx(x0);
+      p1 = ex2_approx(x1);
+    }
+    if (((2 * q4 + 1) & 7) < kEmuPairsOf8) {
+      exp2_fma2(p2, p3, x2, x3);
+    } else {
+      p2 = ex2_approx(x2);
+      p3 = ex2_approx(x3);
+    }
+    if (kDiag) {
+      p0 = (col >= first_col) ? p0 : 0.f;
+      p1 = (col + 1 >= first_col) ? p1 : 0.f;
+      p2 = (col + 2 >= first_col) ? p2 : 0.f;
+      p3 = (col + 3 >= first_col) ? p3 : 0.f;
+    }
+    fadd2(part[0], part[1], part[0], part[1], p0, p1);
+    fadd2(part[2], part[3], part[2], part[3], p2, p3);
+  }
+}
+
 template <int D, bool Q8>
 __global__ void __launch_bounds__(64 + 128 * ColLayout<D>::kGroups, 1)
     attn_colsum_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -397,16 +432,20 @@ __global__ void __launch_bounds__(64 + 128 * ColLayout<D>::kGroups, 1)
 // the current item is summed, so no SM waits for a CTA to start up or drain
 // between items.  Group 0 copies key tiles into TMEM (when the tile has
 // landed and its TMEM buffer is free, checked before each of its row tiles).
-// Row tile v of an item's sweep goes to S buffer and summing group v mod 3,
-// the sweep starting at the same tile as in the one-CTA-per-tile kernel, so
-// every key's sum is formed in the same order as there, whatever the grid.
-// Each group writes its partial sums of an item into shared memory and the
-// last of the three groups to do so for a key adds the partials in group
-// order and writes the summed weight.
-// Summing warpgroups 4-15 with 152 registers reading a whole S tile at once
-// (warps 0-3 hand theirs over) or warps 2-13 reading it in two halves.
-// Measured on the C 8192 cache: 106.5 against 105.5 us; the halves stay.
-constexpr bool kColsumWide = false;
+// Row tile v of an item's sweep goes to S buffer v mod 3 and its summing
+// warpgroups (one per buffer, as in the one-CTA-per-tile kernel, or two,
+// each taking 64 of the tile's columns), so every key's sum is formed in an
+// order fixed by its item, whatever the grid.  Each warpgroup writes its
+// partial sums of an item into shared memory and the last to do so for a
+// key adds the partials in warpgroup order and writes the summed weight.
+// Summing warpgroups per S buffer: 1 (each reads its tile in two halves of
+// 64 columns) or 2 (each takes 64 of the tile's columns, twice as many warps
+// sharing each SM sub-partition's exponentials, 72 registers a thread).
+// Measured on the C 8192 cache: 100.4 us with one, 118.8 with two; on the
+// 144-cache stack 17.0 against 20.3 ms.  Also measured and not kept: one
+// summing warpgroup per buffer reading the whole tile at once with 152
+// registers (warps 0-3 handing theirs over), 106.5 against 105.5 us.
+constexpr int kColsumSplit = 1;
 
 template <int D, bool Q8>
 struct PColLayout {
@@ -417,13 +456,15 @@ struct PColLayout {
   static constexpr int kQStages = 4;
   static constexpr int kLseStages = 16;
   static constexpr int kSBufs = kGroups;
+  static constexpr int kSplit = kColsumSplit;      // summing warpgroups per S buffer
+  static constexpr int kParts = kGroups * kSplit;  // summing warpgroups
   static constexpr int kRedSets = 8;  // items whose partials may be pending at once
   static constexpr int kKOff = 0;                               // bf16 key tile staging
   static constexpr int kCodeOff = kKOff + kTileBytes;           // Q8 codes staging
   static constexpr int kQOff = kCodeOff + kCodeBytes;
   static constexpr int kLseOff = kQOff + kQStages * kTileBytes;
-  static constexpr int kRedOff = kLseOff + kLseStages * 512;    // [sets][groups][128] float
-  static constexpr int kCntOff = kRedOff + kRedSets * kGroups * 128 * 4;  // [sets][128] int
+  static constexpr int kRedOff = kLseOff + kLseStages * 512;    // [sets][parts][128] float
+  static constexpr int kCntOff = kRedOff + kRedSets * kParts * 128 * 4;   // [sets][128] int
   static constexpr int kDoneOff = kCntOff + kRedSets * 128 * 4;            // [sets][128] int
   static constexpr int kBarOff = kDoneOff + kRedSets * 128 * 4;
   // k_full, k_free, ktm[2], ktm_free[2], q_full[QS], q_empty[QS], l_full[LS],
@@ -436,15 +477,7 @@ struct PColLayout {
   static constexpr int kTmemCols = 512;
   static constexpr int kKCol = 128 * kSBufs;                    // two key buffers of D/2 columns
   static_assert(kKCol + D <= kTmemCols, "TMEM layout");
-  // kWide: warps 0-3 (producer, MMA, two idle) hand registers to the summing
-  // warpgroups (4-15), which then read a whole S tile (128 columns) at once
-  // and free its buffer before summing; else warps 2-13 sum, a tile in two
-  // halves of 64 columns.
-  static constexpr bool kWide = kColsumWide;
-  static constexpr int kSumWarp0 = kWide ? 4 : 2;
-  static constexpr int kThreads = 32 * kSumWarp0 + 128 * kGroups;
-  static constexpr uint32_t kLowRegs = 56, kSumRegs = 152;
-  static_assert(!kWide || 128 * kLowRegs + 128 * kGroups * kSumRegs <= 65536, "register split");
+  static constexpr int kThreads = 64 + 128 * kParts;
 };
 
 // Work item i of the list: key tile `kt` (< NCT: cache keys, else chunk key
@@ -530,11 +563,11 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
     }
     for (int s = 0; s < L::kLseStages; ++s) {
       mbar_init(bar_l_full0 + 8 * s, 1);
-      mbar_init(bar_l_empty0 + 8 * s, 128);
+      mbar_init(bar_l_empty0 + 8 * s, 128 * L::kSplit);
     }
     for (int s = 0; s < L::kSBufs; ++s) {
       mbar_init(bar_s_full0 + 8 * s, 1);
-      mbar_init(bar_s_empty0 + 8 * s, 128);
+      mbar_init(bar_s_empty0 + 8 * s, 128 * L::kSplit);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -553,8 +586,6 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < L::kSumWarp0) {
-  if (L::kWide) warpgroup_reg_dec<L::kLowRegs>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -659,12 +690,12 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
       mma_commit(bar_drain);
       mbar_wait_drain(bar_drain, 0, p.err);
     }
-  }
   } else {
     // ------------------------------------------------------------ summing groups
-    if (L::kWide) warpgroup_reg_inc<L::kSumRegs>();
     const int quad = warp & 3;
-    const int grp = (warp - L::kSumWarp0) >> 2;  // row tiles u of an item with u % kGroups == grp
+    const int part_id = (warp - 2) >> 2;       // summing warpgroup
+    const int grp = part_id / L::kSplit;       // row tiles u of an item with u % kGroups == grp
+    const int hc = part_id % L::kSplit;        // kSplit 2: its 64 of the buffer's columns
     const int row = quad * 32 + lane;  // key j0 + row of the current item
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float c = p.scale_log2;
@@ -687,34 +718,37 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
       ready = __all_sync(0xffffffffu, ready);
       if (!ready) return false;
       tc_fence_after();
-      uint32_t w[D / 2];
-      if (Q8 && !it.is_chunk) {
-        const float sc = it.j0 + row < p.n
-                             ? p.k_scale[static_cast<size_t>(it.bg) * p.C + it.j0 + row] : 0.f;
+      const float sc = (Q8 && !it.is_chunk && it.j0 + row < p.n)
+                           ? p.k_scale[static_cast<size_t>(it.bg) * p.C + it.j0 + row] : 0.f;
+      // 32 TMEM columns (64 elements) at a time
 #pragma unroll
-        for (int i = 0; i < D / 16; ++i) {
-          uint32_t piece[8];
-          q8_dequant16(*reinterpret_cast<const uint4*>(smem + L::kCodeOff + row * D + 16 * i), sc,
-                       piece);
+      for (int c0 = 0; c0 < D / 2; c0 += 32) {
+        uint32_t w[32];
+        if (Q8 && !it.is_chunk) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) w[8 * i + j] = piece[j];
+          for (int i = 0; i < 4; ++i) {
+            uint32_t piece[8];
+            q8_dequant16(*reinterpret_cast<const uint4*>(smem + L::kCodeOff + row * D + 2 * c0 +
+                                                         16 * i),
+                         sc, piece);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) w[8 * i + j] = piece[j];
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int c16 = c0 / 4 + q;
+            const uint4 v = *reinterpret_cast<const uint4*>(
+                smem + L::kKOff + (c16 / 8) * 16384 + row * 128 + (((c16 % 8) ^ (row & 7)) * 16));
+            w[4 * q] = v.x;
+            w[4 * q + 1] = v.y;
+            w[4 * q + 2] = v.z;
+            w[4 * q + 3] = v.w;
+          }
         }
-      } else {
-#pragma unroll
-        for (int c16 = 0; c16 < D / 8; ++c16) {
-          const uint4 v = *reinterpret_cast<const uint4*>(
-              smem + L::kKOff + (c16 / 8) * 16384 + row * 128 + (((c16 % 8) ^ (row & 7)) * 16));
-          w[4 * c16] = v.x;
-          w[4 * c16 + 1] = v.y;
-          w[4 * c16 + 2] = v.z;
-          w[4 * c16 + 3] = v.w;
-        }
+        tmem_st32(lane_base + L::kKCol + kb * (D / 2) + c0, w);
       }
       mbar_arrive(bar_k_free);  // the staging may take the next key tile
-#pragma unroll
-      for (int c0 = 0; c0 < D / 2; c0 += 32)
-        tmem_st32(lane_base + L::kKCol + kb * (D / 2) + c0,
-                  *reinterpret_cast<uint32_t(*)[32]>(&w[c0]));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_ktm0 + 8 * kb);
@@ -724,7 +758,7 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
     int used = 0;        // uses of this group's S buffer so far
     for (int i = first; i < items && ok; i += stride, ++k) {
       const ColItem it = col_item(i, BG, NCT, NCTC, NQT, p.G);
-      if (grp == 0 && copied == k) {  // this item's key tile must be in TMEM first
+      if (part_id == 0 && copied == k) {  // this item's key tile must be in TMEM first
         ok = copy_key_tile(k, i, true);
         if (!ok) break;
         ++copied;
@@ -734,7 +768,7 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
       // index gu0 + u), so the order of the sums depends on the item alone
       for (int u = grp; u < it.R; u += L::kGroups, ++used) {
         const int gu = gu0 + u;
-        if (grp == 0 && copied == k + 1 && i + stride < items) {  // the next item's key tile, early
+        if (part_id == 0 && copied == k + 1 && i + stride < items) {  // the next item's key tile, early
           if (copy_key_tile(k + 1, i + stride, false)) ++copied;
         }
         const int sl = gu % L::kLseStages;
@@ -746,25 +780,28 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
         const int qt = it.qt_min + it.tile_of(u) % it.span;
         const bool diag = it.is_chunk && qt == it.kt;
         float part[4] = {0.f, 0.f, 0.f, 0.f};
-        if (L::kWide) {
-          // the whole tile into registers, then the buffer is free
-          uint32_t v[4][32];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) tmem_ld32(lane_base + sb * 128 + 32 * q, v[q]);
+        if (L::kSplit == 2) {
+          // this warpgroup's 64 columns, 32 at a time; its share of the
+          // buffer is free once the second piece is in registers
+          uint32_t v[32];
+          tmem_ld32(lane_base + sb * 128 + 64 * hc, v);
           tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(bar_s_empty0 + 8 * sb);
           ok = mbar_wait(bar_l_full0 + 8 * sl, (gl_parity(gu, L::kLseStages)), p.err, abort_flag);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
-          const float4* nlse4 = reinterpret_cast<const float4*>(smem + L::kLseOff + sl * 512);
-          if (diag) {
-            sum_tile<true>(v[0], v[1], nlse4, c, row, part);
-            sum_tile<true>(v[2], v[3], nlse4 + 16, c, row - 64, part);
-          } else {
-            sum_tile<false>(v[0], v[1], nlse4, c, 0, part);
-            sum_tile<false>(v[2], v[3], nlse4 + 16, c, 0, part);
-          }
+          const float4* nlse4 = reinterpret_cast<const float4*>(smem + L::kLseOff + sl * 512) + 16 * hc;
+          if (diag)
+            sum_piece<true>(v, nlse4, c, row - 64 * hc, part);
+          else
+            sum_piece<false>(v, nlse4, c, 0, part);
+          tmem_ld32(lane_base + sb * 128 + 64 * hc + 32, v);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar_s_empty0 + 8 * sb);
+          if (diag)
+            sum_piece<true>(v, nlse4 + 8, c, row - 64 * hc - 32, part);
+          else
+            sum_piece<false>(v, nlse4 + 8, c, 0, part);
         } else {
           uint32_t v[2][32];
           tmem_ld32(lane_base + sb * 128, v[0]);
@@ -793,8 +830,9 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
       }
       if (!ok) break;
       // this group's partial of the item (in the set of item k, once the
-      // set's previous item is combined); the third group to get here for a
-      // key adds the three in group order and writes the summed weight
+      // set's previous item is combined); the last summing warpgroup to get
+      // here for a key adds the partials in warpgroup order and writes the
+      // summed weight
       const int set = k % L::kRedSets;
       const int use = k / L::kRedSets;
       const int slot = set * 128 + row;
@@ -815,13 +853,13 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
       }
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      red[(set * L::kGroups + grp) * 128 + row] = acc;
+      red[(set * L::kParts + part_id) * 128 + row] = acc;
       __threadfence_block();
-      if (atomicAdd(&cnt[slot], 1) == L::kGroups * use + L::kGroups - 1) {
+      if (atomicAdd(&cnt[slot], 1) == L::kParts * use + L::kParts - 1) {
         __threadfence_block();
         float total = 0.f;
 #pragma unroll
-        for (int gr = 0; gr < L::kGroups; ++gr) total += red[(set * L::kGroups + gr) * 128 + row];
+        for (int gr = 0; gr < L::kParts; ++gr) total += red[(set * L::kParts + gr) * 128 + row];
         __threadfence_block();
         done[slot] = use + 1;
         float* out = p.colsum + static_cast<size_t>(it.bg) * p.colsum_ld;
