@@ -19,7 +19,8 @@
 //                 S_X(t) = Q_X K(t)^T  into TMEM columns [128X, 128X+128)
 //                 O_X   += P_X(t) V(t) into TMEM columns 256 + 128X, with
 //                 P_X(t) read from TMEM (bf16, written over S_X(t))
-//   warps 2..3  int8 cache only: dequantisation (below); otherwise idle
+//   warps 2..3  int8 cache only: dequantisation (below, with warps 4..7 too,
+//               the softmax warps then being 8..15); otherwise idle
 //   warps 4..7  softmax of tile A, warps 8..11 softmax of tile B: one thread
 //               per query row (TMEM lane) reads its 128 logits once, takes
 //               the row max, then P = 2^(x - m) (packed f32x2 arithmetic for
@@ -31,7 +32,7 @@
 // softmax that sees S_X(t+1) may rescale O_X and overwrite P_X.
 //
 // The int8 cache (Q8, q8.cuh): warp 0 brings a cache tile's codes of K and of
-// V into one staging buffer each (TMA, no swizzle), and warps 2 and 3
+// V into one staging buffer each (TMA, no swizzle), and warps 2 to 7
 // dequantise them into the same bf16 rings the MMA reads (128-byte swizzle),
 // with the row scales; the chunk's own tiles still arrive in bf16 by TMA.
 #include <cuda_bf16.h>
@@ -75,15 +76,18 @@ struct FwdLayout {
   static_assert(kBytes <= kMaxDynSmem, "shared-memory layout too large");
   static constexpr int kTmemCols = 512;  // S/P_A | S/P_B | O_A | O_B
   // warpgroup 0: warp 0 TMA, warp 1 MMA, warps 2-3 dequantise (Q8) or idle;
-  // warpgroups 1 and 2: the softmax of tiles A and B.  Launched with 168
-  // registers per thread (384 x 168 <= 64 K); warpgroup 0 gives registers
-  // back so that the softmax warpgroups hold kSoftmaxRegs each:
-  // 128 x kLoadRegs + 256 x kSoftmaxRegs <= 384 x 168, and per SM
-  // sub-partition (one warp of each group) kLoadRegs + 2 kSoftmaxRegs <= 512.
-  static constexpr int kThreads = 384;
-  static constexpr uint32_t kLoadRegs = 80;
+  // Q8: warpgroup 1 dequantises too (six converter warps); then two softmax
+  // warpgroups, tiles A and B.  The non-softmax warpgroups give registers
+  // back so that the softmax warpgroups hold kSoftmaxRegs each (384 threads:
+  // launched with 168 a thread; 512: with 128).
+  static constexpr int kSoftWarp0 = Q8 ? 8 : 4;      // first softmax warp
+  static constexpr int kConvThreads = 32 * (kSoftWarp0 - 2);
+  static constexpr int kThreads = 32 * kSoftWarp0 + 256;
+  static constexpr uint32_t kLoadRegs = Q8 ? 56 : 80;
   static constexpr uint32_t kSoftmaxRegs = 200;
-  static_assert(128 * kLoadRegs + 256 * kSoftmaxRegs <= 384 * 168, "register budget");
+  static_assert(32 * kSoftWarp0 * kLoadRegs + 256 * kSoftmaxRegs <=
+                    kThreads * ((65536 / kThreads) & ~7),
+                "register budget");
 };
 
 template <int D, bool Q8>
@@ -172,8 +176,8 @@ __global__ void __launch_bounds__(FwdLayout<D, Q8>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (warp < 4) {
-  // warpgroup 0 (TMA, MMA, dequantising) hands registers to the softmax groups
+  if (warp < L::kSoftWarp0) {
+  // the TMA / MMA / dequantising warpgroups hand registers to the softmax groups
   warpgroup_reg_dec<L::kLoadRegs>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -300,8 +304,8 @@ __global__ void __launch_bounds__(FwdLayout<D, Q8>::kThreads, 1)
       mma_commit(bar_drain);
       mbar_wait_drain(bar_drain, 0, p.err);
     }
-  } else if (warp < 4) {
-    // warps 2 and 3: no role without the int8 cache
+  } else {
+    // warps 2 .. kSoftWarp0-1: no role without the int8 cache
     if (Q8) {
     // ------------------------------------------------------------ dequantise (Q8)
     // cache tile t: codes (staging) -> bf16 ring slot t % 2 of K, then of V.
@@ -309,8 +313,9 @@ __global__ void __launch_bounds__(FwdLayout<D, Q8>::kThreads, 1)
     // threads on consecutive pieces); each piece becomes two 16-byte chunks of
     // its 128-byte region row, at chunk index ^ (row & 7) (the swizzle).
     constexpr int kPer = D / 16;                    // pieces per row
-    constexpr int kJobs = 128 * kPer / 64;          // pieces per thread and tile
-    const int ct = threadIdx.x - 64;                // 0 .. 63
+    constexpr int kNC = L::kConvThreads;
+    constexpr int kJobs = (128 * kPer + kNC - 1) / kNC;  // pieces per thread and tile
+    const int ct = threadIdx.x - 64;                // 0 .. kNC - 1
     bool ok = true;
     for (int t = 0; t < NCT && ok; ++t) {
       const int j0 = t * 128;
@@ -319,8 +324,8 @@ __global__ void __launch_bounds__(FwdLayout<D, Q8>::kThreads, 1)
         float sc[kJobs];
 #pragma unroll
         for (int k = 0; k < kJobs; ++k) {
-          const int r = (ct + 64 * k) / kPer;
-          sc[k] = j0 + r < p.n ? scale[j0 + r] : 0.f;
+          const int r = (ct + kNC * k) / kPer;
+          sc[k] = (ct + kNC * k < 128 * kPer && j0 + r < p.n) ? scale[j0 + r] : 0.f;
         }
         const int NS = w ? L::kVStages : L::kKStages;
         const int s = t % NS;
@@ -328,13 +333,14 @@ __global__ void __launch_bounds__(FwdLayout<D, Q8>::kThreads, 1)
         if (ok && t >= NS)
           ok = mbar_wait((w ? bar_v_empty0 : bar_k_empty0) + 8 * s, ((t / NS) + 1) & 1, p.err,
                          abort_flag);
-        ok = named_bar_and(1, 64, ok);  // every converter thread takes the same branch
+        ok = named_bar_and(1, kNC, ok);  // every converter thread takes the same branch
         if (!ok) break;
         const uint8_t* codes = smem + (w ? L::kV8Off : L::kK8Off);
         uint8_t* dst = smem + (w ? L::kVOff : L::kKOff) + s * L::kTileBytes;
 #pragma unroll 4
         for (int k = 0; k < kJobs; ++k) {
-          const int job = ct + 64 * k;
+          const int job = ct + kNC * k;
+          if (job >= 128 * kPer) break;
           const int r = job / kPer, i = job % kPer;
           uint32_t wv[8];
           q8_dequant16(*reinterpret_cast<const uint4*>(codes + r * D + 16 * i), sc[k], wv);
@@ -346,7 +352,7 @@ __global__ void __launch_bounds__(FwdLayout<D, Q8>::kThreads, 1)
               make_uint4(wv[4], wv[5], wv[6], wv[7]);
         }
         fence_proxy_async_smem();  // the MMA reads the operand through the async proxy
-        named_bar_sync(1, 64);     // all 64 converters are done with the codes and the slot
+        named_bar_sync(1, kNC);    // all converters are done with the codes and the slot
         if (ct == 0) {
           mbar_arrive((w ? bar_v_full0 : bar_k_full0) + 8 * s);
           mbar_arrive(w ? bar_v8_empty : bar_k8_empty);
@@ -358,7 +364,7 @@ __global__ void __launch_bounds__(FwdLayout<D, Q8>::kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax rows
     warpgroup_reg_inc<L::kSoftmaxRegs>();
-    const int x = (warp - 4) >> 2;  // tile A or B
+    const int x = (warp - L::kSoftWarp0) >> 2;  // tile A or B
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const int T = x ? TB : TA;
