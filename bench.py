@@ -46,7 +46,7 @@ KERNELS = ["attn_fwd_kernel", "attn_colsum_persistent", "h2o_select", "reserved"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # fp32 FMA peak from the unit counts: 148 SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz
 F32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-# spec targets: attention + summed weights against the bf16 dense peak,
+# performance targets: attention + summed weights against the bf16 dense peak,
 # the eviction (score update, selection, scatter) against HBM bandwidth
 TARGET_ATTENTION_TC = 0.50
 TARGET_EVICT_HBM = 0.60
