@@ -587,8 +587,6 @@ __global__ void __launch_bounds__(kThreads, 3) decode_partial(const DecodeParams
   extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ __align__(8) uint64_t bars[2];
   __shared__ int abort_flag;
-  // the merge kernel may start; it waits for this grid before reading
-  griddep_launch_dependents();
   const int bg = blockIdx.y;
   const int chunk = blockIdx.x;
   const uint32_t bK = smem_u32(&bars[0]), bV = smem_u32(&bars[1]);
@@ -605,6 +603,10 @@ __global__ void __launch_bounds__(kThreads, 3) decode_partial(const DecodeParams
   chunk_partial<T, D, G, Q8>(p, bg, chunk, dsm + L::kK, dsm + L::kV, dsm + L::kN,
                              reinterpret_cast<float*>(dsm + L::kS),
                              reinterpret_cast<float*>(dsm + L::kX), bK, bV, 0u, &abort_flag, qf);
+  // the merge kernel may start now (its CTAs wait for this grid before
+  // reading; triggered at the start instead, they take SM slots from this
+  // grid's second wave: 31.7 against 29.7 us per step on one cache)
+  griddep_launch_dependents();
   if (!kFused) return;
   // the merge's scratch reuses the K and V rows (every copy has landed)
   if (last_of_unit(p, bg)) merge_unit<T, D, G, Q8>(p, bg, reinterpret_cast<float*>(dsm));
