@@ -83,7 +83,21 @@ struct DkdvLayout {
 
 // Both tensor-core kernels: warp 0 TMA, warp 1 TMEM + MMA, then two
 // warpgroups of row threads, one per half of the 128 columns of S.
-constexpr int kBwdThreads = 64 + 2 * 128;
+// Row warps per TMEM lane quadrant and half of a unit: 1 (a warp takes the
+// half's 64 columns) or 2 (32 columns each, so that one warp's TMEM loads
+// and exponentials overlap the other's).  Measured on the C 8192 cache: the
+// row work of a half drops from ~1650 to ~1270 cycles with 2, but the MMA
+// thread, sharing its SM sub-partition with twice the row warps, notices
+// the ready rows ~750 cycles late instead of ~300 (spinning or not), and the
+// backward takes 609-611 us against 595-597 with 1.
+constexpr int kRowSplit = 1;
+constexpr int kBwdThreads = 64 + 2 * 128 * kRowSplit;
+
+// TMEM column of the bf16 pairs of 16 columns ks (0..3) of half hf: each row
+// warp writes the pairs of its own columns over the first of them.
+__device__ __forceinline__ uint32_t pair_col(int hf, int ks) {
+  return kRowSplit == 2 ? 64 * hf + 32 * (ks >> 1) + 8 * (ks & 1) : 64 * hf + 8 * ks;
+}
 
 // Row arithmetic shared by the two kernels: from 32 logits s and 32 dP
 // values of one row (or one key), the bf16 pairs of P and of scale * dS =
@@ -130,26 +144,26 @@ __device__ __forceinline__ void p_ds(const uint32_t (&s)[NV], const uint32_t (&d
   }
 }
 
-// The row work of one half (64 columns) of a unit's S and dP in TMEM (S at
-// s_col, dP at s_col + 128, the half's columns starting at c0): four
-// sub-blocks of 16 columns, the TMEM loads of the next issued before the
-// arithmetic of the current one, so that they overlap it; the bf16 pairs of
-// sub-block k go over columns [c0 + 8k, +8) of S (P) and of dP (scale dS)
-// -- or, kDsOverS, scale dS over S and P nowhere -- which hold values
-// already read.  Column statistics at nls / nds (per column, kCol) or the
-// row's own (nls[0], nds[0]); masking as in p_ds.
-template <bool kCol, bool kDsOverS>
-__device__ __forceinline__ void half_rows(uint32_t s_col, int c0, const float* nls,
-                                          const float* nds, float c, float scale, bool masked,
-                                          int first_valid, int last_valid) {
+// The row work of NSUB x 16 columns of a unit's S and dP in TMEM (S at
+// s_col, dP at s_col + 128, the block's columns starting at c0): sub-blocks
+// of 16 columns whose TMEM loads are issued one ahead of the arithmetic; the
+// bf16 pairs of sub-block k go over columns [c0 + 8k, +8) of S (P) and of dP
+// (scale dS) -- or, kDsOverS, scale dS over S and P nowhere -- which hold
+// values this thread has already read.  Column statistics at nls / nds (per
+// column, kCol) or the row's own (nls[0], nds[0]); masking as in p_ds, the
+// bounds relative to column c0.
+template <bool kCol, bool kDsOverS, int NSUB>
+__device__ __forceinline__ void rows_block(uint32_t s_col, int c0, const float* nls,
+                                           const float* nds, float c, float scale, bool masked,
+                                           int first_valid, int last_valid) {
   uint32_t sv[2][16], dp[2][16];
   tmem_ld16(s_col + c0, sv[0]);
   tmem_ld16(s_col + 128 + c0, dp[0]);
   tmem_wait_ld();
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
+  for (int k = 0; k < NSUB; ++k) {
     const int cur = k & 1;
-    if (k < 3) {
+    if (k + 1 < NSUB) {
       tmem_ld16(s_col + c0 + 16 * (k + 1), sv[cur ^ 1]);
       tmem_ld16(s_col + 128 + c0 + 16 * (k + 1), dp[cur ^ 1]);
     }
@@ -167,7 +181,7 @@ __device__ __forceinline__ void half_rows(uint32_t s_col, int c0, const float* n
       tmem_st8(s_col + c0 + 8 * k, pp);
       tmem_st8(s_col + 128 + c0 + 8 * k, dd);
     }
-    if (k < 3) tmem_wait_ld();
+    if (k + 1 < NSUB) tmem_wait_ld();
   }
 }
 
@@ -221,7 +235,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(bar_s0 + 8 * h, 1);
-      mbar_init(bar_p0 + 8 * h, 128);
+      mbar_init(bar_p0 + 8 * h, 128 * kRowSplit);
     }
     mbar_init(bar_o, 1);
     mbar_init(bar_drain, 1);
@@ -308,13 +322,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t db = sbase + L::kDOOff + s * L::kTileBytes;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          mma_bf16_ts(tmem + 256, tmem + 64 * hf + 8 * ks,
+          mma_bf16_ts(tmem + 256, tmem + pair_col(hf, ks),
                       sw128_desc(db + (4 * hf + ks) * 2048, 16384, 1024), kIdescAcc,
                       (first && ks == 0) ? 0u : 1u);
         }
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          mma_bf16_ts(tmem + 384, tmem + 128 + 64 * hf + 8 * ks,
+          mma_bf16_ts(tmem + 384, tmem + 128 + pair_col(hf, ks),
                       sw128_desc(qb + (4 * hf + ks) * 2048, 16384, 1024), kIdescAcc,
                       (first && ks == 0) ? 0u : 1u);
         }
@@ -354,7 +368,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_wait_drain(bar_drain, 0, p.err);
     }
   } else {
-    const int hf = (warp - 2) >> 2;  // half of the unit's queries
+    const int rw = warp - 2;
+    const int hf = rw / (4 * kRowSplit);       // half of the unit's queries
+    const int sub = (rw >> 2) % kRowSplit;     // kRowSplit 2: its 32 of the half's columns
     const int quad = warp & 3;
     const int row = quad * 32 + lane;  // key j0 + row
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
@@ -371,9 +387,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float* nds = nls + 128;
       const int qt = qt_min + u % span;
       const bool diag = is_chunk && qt == kt;  // query col sees key row iff row <= col
-      // queries [64 hf, +64); bf16 pairs over the half's first 32 columns
-      half_rows<true, false>(lane_base, 64 * hf, nls + 64 * hf, nds + 64 * hf, c, scale, diag,
-                      row - 64 * hf, 1 << 30);
+      // queries [c0, +64 / kRowSplit); bf16 pairs over the first of them
+      const int c0 = 64 * hf + (64 / kRowSplit) * sub;
+      rows_block<true, false, 4 / kRowSplit>(lane_base, c0, nls + c0, nds + c0, c, scale, diag,
+                                            row - c0, 1 << 30);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p0 + 8 * hf);
@@ -383,7 +400,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
-      // half 0 writes dK, half 1 dV
+      // half 0 writes dK, half 1 dV (kRowSplit 2: each warp half of the columns)
       tc_fence_after();
       const int key = j0 + row;
       float* dst = nullptr;
@@ -396,8 +413,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       const bool valid = is_chunk ? key < p.nq : key < p.n;
       const uint32_t col = hf == 0 ? 384 : 256;
+      constexpr int kW = D / kRowSplit;  // columns of the row this warp writes
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = sub * kW; c0 < (sub + 1) * kW; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(lane_base + col + c0, v);
         tmem_wait_ld();
@@ -482,7 +500,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     for (int hf = 0; hf < 2; ++hf) {
       mbar_init(bar_s0 + 8 * hf, 1);
-      mbar_init(bar_p0 + 8 * hf, 128);
+      mbar_init(bar_p0 + 8 * hf, 128 * kRowSplit);
     }
     mbar_init(bar_o, 1);
     mbar_init(bar_drain, 1);
@@ -564,7 +582,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t kb = sbase + L::kKOff + s * L::kTileBytes;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          mma_bf16_ts(tmem + 256, tmem + 64 * hf + 8 * ks,
+          mma_bf16_ts(tmem + 256, tmem + pair_col(hf, ks),
                       sw128_desc(kb + (4 * hf + ks) * 2048, 16384, 1024), kIdescAcc,
                       (first && ks == 0) ? 0u : 1u);
         }
@@ -602,7 +620,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_wait_drain(bar_drain, 0, p.err);
     }
   } else {
-    const int hf = (warp - 2) >> 2;  // half of each key tile
+    const int rw = warp - 2;
+    const int hf = rw / (4 * kRowSplit);       // half of each key tile
+    const int sub = (rw >> 2) % kRowSplit;     // kRowSplit 2: its 32 of the half's columns
     const int quad = warp & 3;
     const int row = quad * 32 + lane;  // query qt*128 + row
     const int i = qt * 128 + row;
@@ -629,8 +649,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         masked = true;
         last = row;
       }
-      // keys [64 hf, +64); scale*dS over S's half (P over dP's, unused)
-      half_rows<false, true>(lane_base, 64 * hf, nls, nds, c, scale, masked, 0, last - 64 * hf);
+      // keys [c0, +64 / kRowSplit); scale*dS over S's first of them
+      const int c0 = 64 * hf + (64 / kRowSplit) * sub;
+      rows_block<false, true, 4 / kRowSplit>(lane_base, c0, nls, nds, c, scale, masked, 0,
+                                             last - c0);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p0 + 8 * hf);
@@ -640,17 +662,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
-      // each half writes D/2 of the row's dQ columns
+      // each warp writes its share of the row's dQ columns
       tc_fence_after();
       float* dqr = p.dq + ((static_cast<size_t>(b) * p.nq + i) * p.Hq + h) * D;
+      constexpr int kW = D / (2 * kRowSplit);  // 16, 32 or 64 columns
+      const int part = hf * kRowSplit + sub;
 #pragma unroll
-      for (int c0 = hf * (D / 2); c0 < (hf + 1) * (D / 2); c0 += 32) {
-        uint32_t qv[32];
-        tmem_ld32(lane_base + 256 + c0, qv);
+      for (int c0 = part * kW; c0 < (part + 1) * kW; c0 += 16) {
+        uint32_t qv[16];
+        tmem_ld16(lane_base + 256 + c0, qv);
         tmem_wait_ld();
         if (i < p.nq) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
+          for (int e = 0; e < 16; e += 4)
             *reinterpret_cast<float4*>(dqr + c0 + e) =
                 make_float4(__uint_as_float(qv[e]), __uint_as_float(qv[e + 1]),
                             __uint_as_float(qv[e + 2]), __uint_as_float(qv[e + 3]));
