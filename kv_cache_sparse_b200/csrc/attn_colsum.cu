@@ -430,7 +430,8 @@ __global__ void __launch_bounds__(64 + 128 * ColLayout<D>::kGroups, 1)
 // Q and row-statistic rings continue with a global row-tile counter, and the
 // next item's key tile is loaded and copied into a second TMEM buffer while
 // the current item is summed, so no SM waits for a CTA to start up or drain
-// between items.  Group 0 copies key tiles into TMEM (when the tile has
+// between items.  Two threads (lane 0 of warps 1 and 2) issue the MMAs, the
+// row tiles in turn.  Group 0 copies key tiles into TMEM (when the tile has
 // landed and its TMEM buffer is free, checked before each of its row tiles).
 // Row tile v of an item's sweep goes to S buffer v mod 3 and its summing
 // warpgroups (one per buffer, as in the one-CTA-per-tile kernel, or two,
@@ -446,6 +447,16 @@ __global__ void __launch_bounds__(64 + 128 * ColLayout<D>::kGroups, 1)
 // summing warpgroup per buffer reading the whole tile at once with 152
 // registers (warps 0-3 handing theirs over), 106.5 against 105.5 us.
 constexpr int kColsumSplit = 1;
+// MMA-issuing threads (lane 0 of warps 1 .. kColsumIssuers), taking the row
+// tiles in turn.  Each issue of a tile's MMAs returns about when the tensor
+// pipe has taken them, so one thread's own waits, commits and bookkeeping
+// between tiles leave the pipe idle; a second issuer fills those gaps.
+// Measured on the C 8192 cache: 102.4 against 106.5 us with one issuer; on
+// the 144-cache stack 18.1 against 18.7 ms.  With two issuers a whole-tile
+// read (warps 0-3 handing registers to the summing warpgroups, which free an
+// S buffer before summing it) is still no faster: 104.4 us at 160 registers,
+// 106.5 at 152 (spills), against 102.4.
+constexpr int kColsumIssuers = 2;
 
 template <int D, bool Q8>
 struct PColLayout {
@@ -477,8 +488,34 @@ struct PColLayout {
   static constexpr int kTmemCols = 512;
   static constexpr int kKCol = 128 * kSBufs;                    // two key buffers of D/2 columns
   static_assert(kKCol + D <= kTmemCols, "TMEM layout");
-  static constexpr int kThreads = 64 + 128 * kParts;
+  static constexpr int kIssuers = kColsumIssuers;  // MMA-issuing warps, 1 .. kIssuers
+  static constexpr int kGroupWarp0 = 1 + kIssuers;  // first summing warp
+  static constexpr int kThreads = 32 * kGroupWarp0 + 128 * kParts;
 };
+
+// Waits until *count >= target (a count that another thread of the CTA
+// raises); gives up like mbar_wait_spin.
+__device__ __forceinline__ bool wait_count(const volatile int* count, int target, int* err,
+                                           volatile int* abort) {
+  if (*count >= target) {
+    __threadfence_block();
+    return true;
+  }
+  const uint64_t start = global_timer_ns();
+  uint32_t n = 0;
+  while (*count < target) {
+    if ((++n & 255) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - start > kWaitLimitNs) {
+        *abort = 1;
+        atomicOr(err, kDevErrTimeout);
+        return false;
+      }
+    }
+  }
+  __threadfence_block();
+  return true;
+}
 
 // Work item i of the list: key tile `kt` (< NCT: cache keys, else chunk key
 // tile kt - NCT) of unit bg.
@@ -546,6 +583,7 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
   const uint32_t bar_drain = bar_s_empty0 + 8 * L::kSBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  volatile int* issued = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 8);  // row tiles issued
   float* red = reinterpret_cast<float*>(smem + L::kRedOff);
   int* cnt = reinterpret_cast<int*>(smem + L::kCntOff);     // partials arrived, per set and key
   volatile int* done = reinterpret_cast<volatile int*>(smem + L::kDoneOff);  // uses combined
@@ -555,7 +593,7 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
     mbar_init(bar_k_free, 128);
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar_ktm0 + 8 * x, 128);
-      mbar_init(bar_ktm_free0 + 8 * x, 1);
+      mbar_init(bar_ktm_free0 + 8 * x, L::kIssuers);
     }
     for (int s = 0; s < L::kQStages; ++s) {
       mbar_init(bar_q_full0 + 8 * s, 1);
@@ -569,8 +607,9 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
       mbar_init(bar_s_full0 + 8 * s, 1);
       mbar_init(bar_s_empty0 + 8 * s, 128 * L::kSplit);
     }
-    mbar_init(bar_drain, 1);
+    mbar_init(bar_drain, L::kIssuers);
     *abort_flag = 0;
+    *issued = 0;
     fence_barrier_init();
   }
   for (int i = threadIdx.x; i < L::kRedSets * 128; i += blockDim.x) {
@@ -651,8 +690,16 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
       for (int u = max(0, gl - L::kLseStages); u < gl; ++u)
         mbar_wait_drain(bar_l_full0 + 8 * (u % L::kLseStages), (u / L::kLseStages) & 1, p.err);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp <= L::kIssuers) {
+    // ------------------------------------------------------------ MMA issuers
+    // Issuer `me` takes the row tiles gu with gu % kIssuers == me (a Q stage
+    // always with the same issuer) and issues tile gu once tile gu - 1 is
+    // issued, so the tiles reach the pipe in order.  That order also makes the
+    // parity test of an S buffer's release sound: the buffer's previous use
+    // was issued, by either issuer, after the use before it was released.
+    // Both issuers commit each key buffer's release.
+    static_assert(L::kQStages % L::kIssuers == 0, "a Q stage belongs to one issuer");
+    const int me = warp - 1;
     if (lane == 0) {
       constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, false, false);
       const uint64_t q_desc0 = sw128_desc(sbase + L::kQOff, 16, 1024);
@@ -664,10 +711,12 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
         const int kb = n_items & 1;
         ok = mbar_wait_spin(bar_ktm0 + 8 * kb, (n_items >> 1) & 1, p.err, abort_flag);
         for (int u = 0; u < it.R && ok; ++u, ++gu) {
+          if (L::kIssuers > 1 && gu % L::kIssuers != me) continue;
           const int s = gu % L::kQStages;
           const int sb = u % L::kSBufs;  // row tile u of an item: S buffer and group u % 3
           const int j = (sb == 0 ? used0 : sb == 1 ? used1 : used2) + u / L::kSBufs;
           ok = mbar_wait_spin(bar_q_full0 + 8 * s, (gu / L::kQStages) & 1, p.err, abort_flag);
+          if (ok && L::kIssuers > 1 && gu > 0) ok = wait_count(issued, gu, p.err, abort_flag);
           if (ok && j >= 1)
             ok = mbar_wait_spin(bar_s_empty0 + 8 * sb, (j - 1) & 1, p.err, abort_flag);
           if (!ok) break;
@@ -678,6 +727,10 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
             const uint32_t off = ((ks >> 2) * 16384 + (ks & 3) * 32) >> 4;
             mma_bf16_ts(tmem + sb * 128, tmem + L::kKCol + kb * (D / 2) + 8 * ks, qd + off,
                         kIdesc, ks > 0 ? 1u : 0u);
+          }
+          if (L::kIssuers > 1) {
+            __threadfence_block();
+            *issued = gu + 1;
           }
           mma_commit(bar_s_full0 + 8 * sb);
           mma_commit(bar_q_empty0 + 8 * s);
@@ -693,7 +746,7 @@ __global__ void __launch_bounds__(PColLayout<D, Q8>::kThreads, 1)
   } else {
     // ------------------------------------------------------------ summing groups
     const int quad = warp & 3;
-    const int part_id = (warp - 2) >> 2;       // summing warpgroup
+    const int part_id = (warp - L::kGroupWarp0) >> 2;  // summing warpgroup
     const int grp = part_id / L::kSplit;       // row tiles u of an item with u % kGroups == grp
     const int hc = part_id % L::kSplit;        // kSplit 2: its 64 of the buffer's columns
     const int row = quad * 32 + lane;  // key j0 + row of the current item
