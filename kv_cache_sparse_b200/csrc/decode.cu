@@ -37,7 +37,12 @@
 //                   its slots' scores and finds its eviction candidate; the
 //                   last CTA of the (cache, KV head) to finish (atomic ticket)
 //                   takes the minimum over the slices and places the new
-//                   token.  The rule is the top-C rule of the chunk step with
+//                   token.  Each pass needs data from HBM or L2, so every
+//                   load is issued up front: the slots' scores and positions
+//                   and the new token's rows before the wait for the
+//                   split-KV grid, the chunk statistics, partial outputs and
+//                   logits together right after it.  The rule is the top-C
+//                   rule of the chunk step with
 //                   N_q = 1: the unprotected candidate last in (score desc,
 //                   index asc) order leaves -- the lowest score, the highest
 //                   index among equal scores (for the score-free policies the
@@ -612,35 +617,122 @@ __global__ void __launch_bounds__(kThreads, 3) decode_partial(const DecodeParams
   if (last_of_unit(p, bg)) merge_unit<T, D, G, Q8>(p, bg, reinterpret_cast<float*>(dsm));
 }
 
-template <typename T, int D, bool Q8>
+template <typename T, int D, int G, bool Q8>
 __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) {
-  __shared__ float fac[kDecodeMaxG][kMaxChunks];  // 2^(chunk max - head max)
-  __shared__ float lse[kDecodeMaxG], lh[kDecodeMaxG];
+  constexpr int kPer = kDecodeSliceKeys / kThreads;  // keys of the slice per thread
+  constexpr int kStatB = 4;  // chunk statistics per lane read at once (128 chunks a warp)
+  constexpr int kOB = 24;    // partial outputs per thread read at once
+  static_assert(kDecodeSliceKeys % kThreads == 0, "slice keys per thread");
+  __shared__ float fac[G][kMaxChunks];  // 2^(chunk max - head max)
+  __shared__ float lse[G], lh[G];
   __shared__ unsigned long long wmin[kWarps];
   __shared__ int is_last;
-  const int G = p.G;
   const int slice = blockIdx.x;
   const int bg = blockIdx.y;
   const int b = bg / p.Hkv, g = bg % p.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int NCk = p.n_chunks;
   const int C = p.C, n = p.n;
-  // the CTAs that merge O: all slices when there are few (cache, KV head)
-  // units (latency), else the first only (less repeated work)
-  const int o_slices = p.spread_o ? static_cast<int>(gridDim.x) : 1;
-  griddep_wait();  // the partials come from the preceding kernel
+  const int ja = slice * kDecodeSliceKeys;      // this slice's keys [ja, jb): thread tid
+  const int jb = min(n + 1, ja + kDecodeSliceKeys);  // takes ja + tid + r * kThreads
+  const int sb = min(jb, n);                     // of them cache slots: [ja, sb)
+  const bool by_score = p.policy == kPolicyH2O;
+  const bool last_slice = slice == static_cast<int>(gridDim.x) - 1;
+  // Every pass below needs data from HBM or L2, so the loads are issued up
+  // front, all at once: a dependent round trip per pass made the kernel
+  // latency bound.  First what the split-KV kernel does not write, read
+  // while it still runs: this thread's slots' scores and positions, and the
+  // new token's rows (warp 0, 16 bytes a lane; the int8 cache quantises them
+  // from global memory instead).
+  float sc_old[kPer];
+  int ps_old[kPer];
+  uint4 k_row = make_uint4(0, 0, 0, 0), v_row = make_uint4(0, 0, 0, 0);
+  constexpr int kNewBytes = D * static_cast<int>(sizeof(T));
+  static_assert(kNewBytes <= 32 * 16, "a new row is at most 16 bytes a lane");
+  if (p.evict) {
+    const float* score = p.scores + static_cast<size_t>(bg) * C;
+    const int* pos = p.pos + static_cast<size_t>(bg) * C;
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      const int s = ja + tid + r * kThreads;
+      sc_old[r] = (by_score && s < sb) ? score[s] : 0.f;
+      ps_old[r] = (n >= C && s < sb) ? pos[s] : 0;
+    }
+    if (!Q8 && warp == 0 && lane * 16 < kNewBytes) {
+      k_row = *reinterpret_cast<const uint4*>(static_cast<const char*>(p.k_new) +
+                                              static_cast<size_t>(bg) * kNewBytes + lane * 16);
+      v_row = *reinterpret_cast<const uint4*>(static_cast<const char*>(p.v_new) +
+                                              static_cast<size_t>(bg) * kNewBytes + lane * 16);
+    }
+  }
+  griddep_wait();  // the partials and logits come from the preceding kernel
   const float* part = p.part + static_cast<size_t>(bg) * p.part_ld * G * (D + 2);
   auto pidx = [&](int c, int h) { return (static_cast<size_t>(c) * G + h) * (D + 2); };
+
+  // ---- then the split-KV kernel's outputs, together: (a) the chunk
+  // statistics of head `warp` (warps < G); (b) the first partial outputs of
+  // this thread's share of O; (c) the logits of this thread's keys
+  float cm[kStatB], cl[kStatB];
+#pragma unroll
+  for (int t = 0; t < kStatB; ++t) {
+    const int c = lane + 32 * t;
+    const bool v = warp < G && c < NCk;
+    cm[t] = v ? part[pidx(c, warp) + D] : -INFINITY;
+    cl[t] = v ? part[pidx(c, warp) + D + 1] : 0.f;
+  }
+  // O: the CTAs that merge it are all slices when there are few (cache, KV
+  // head) units (latency), else the first only (less repeated work); tpo
+  // lanes per output, each summing chunks cg, cg + tpo, ... in order, then a
+  // fixed butterfly over the tpo lanes
+  const int o_slices = p.spread_o ? static_cast<int>(gridDim.x) : 1;
+  const bool do_o = slice < o_slices;
+  const int GD = G * D;
+  const int per = (GD + o_slices - 1) / o_slices;
+  const int o_begin = slice * per, o_end = min(GD, o_begin + per);
+  int tpo = 1;
+  while (tpo < 32 && 2 * tpo * per <= kThreads) tpo *= 2;
+  const int cg = tid % tpo;
+  const int o_stride = kThreads / tpo;  // outputs per pass
+  float ov[kOB];
+  auto load_o = [&](int i, int c0) {  // output i (if valid), chunks c0, c0 + tpo, ...
+    const bool valid = do_o && i < o_end;
+    const int h = valid ? i / D : 0, d = valid ? i % D : 0;
+#pragma unroll
+    for (int u = 0; u < kOB; ++u) {
+      const int c = c0 + u * tpo;
+      ov[u] = (valid && c < NCk) ? part[pidx(c, h) + d] : 0.f;
+    }
+  };
+  load_o(o_begin + tid / tpo, cg);
+  const float* lg = p.logits + static_cast<size_t>(bg) * G * (C + 1);
+  float lv[kPer][G];
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    const int j = ja + tid + r * kThreads;
+#pragma unroll
+    for (int h = 0; h < G; ++h) lv[r][h] = j < jb ? lg[static_cast<size_t>(h) * (C + 1) + j] : 0.f;
+  }
 
   // ---- per-head log-sum-exp over the chunks (one warp per head)
   if (warp < G) {
     float m = -INFINITY;
-    for (int c = lane; c < NCk; c += 32) m = fmaxf(m, part[pidx(c, warp) + D]);
+#pragma unroll
+    for (int t = 0; t < kStatB; ++t) m = fmaxf(m, cm[t]);
+    for (int c = lane + 32 * kStatB; c < NCk; c += 32) m = fmaxf(m, part[pidx(c, warp) + D]);
     m = warp_max(m);
     float l = 0.f;
-    for (int c = lane; c < NCk; c += 32) {
+#pragma unroll
+    for (int t = 0; t < kStatB; ++t) {
+      const int c = lane + 32 * t;
+      if (c < NCk) {
+        const float f = ex2_approx(cm[t] - m);
+        if (do_o) fac[warp][c] = f;
+        l = fmaf(cl[t], f, l);
+      }
+    }
+    for (int c = lane + 32 * kStatB; c < NCk; c += 32) {
       const float f = ex2_approx(part[pidx(c, warp) + D] - m);
-      if (slice < o_slices) fac[warp][c] = f;
+      if (do_o) fac[warp][c] = f;
       l = fmaf(part[pidx(c, warp) + D + 1], f, l);
     }
     l = warp_sum(l);
@@ -650,24 +742,23 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
     }
   }
   __syncthreads();
-  if (slice < o_slices) {  // O: this CTA's share of the G*D outputs, tpo lanes
-                          // per output (chunks strided over them, then a
-                          // fixed butterfly sum)
+  if (do_o) {
     T* out = static_cast<T*>(p.out) + (static_cast<size_t>(b) * p.Hkv * G + g * G) * D;
-    const int GD = G * D;
-    const int per = (GD + o_slices - 1) / o_slices;
-    const int o_begin = slice * per, o_end = min(GD, o_begin + per);
-    int tpo = 1;
-    while (tpo < 32 && 2 * tpo * per <= kThreads) tpo *= 2;
-    const int cg = tid % tpo;
-    for (int base = o_begin; base < o_end; base += kThreads / tpo) {
+    for (int base = o_begin; base < o_end; base += o_stride) {
       const int i = base + tid / tpo;
       const bool valid = i < o_end;
-      const int h = valid ? i / D : 0, d = valid ? i % D : 0;
+      const int h = valid ? i / D : 0;
+      if (base != o_begin) load_o(i, cg);
       float acc = 0.f;
-      if (valid) {
-#pragma unroll 4
-        for (int c = cg; c < NCk; c += tpo) acc = fmaf(part[pidx(c, h) + d], fac[h][c], acc);
+      for (int c0 = cg;;) {
+#pragma unroll
+        for (int u = 0; u < kOB; ++u) {
+          const int c = c0 + u * tpo;
+          if (valid && c < NCk) acc = fmaf(ov[u], fac[h][c], acc);
+        }
+        c0 += kOB * tpo;
+        if (c0 >= NCk) break;
+        load_o(i, c0);
       }
       for (int o = tpo / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (valid && cg == 0) store(out + i, acc / lh[h]);
@@ -675,56 +766,60 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
   }
 
   // ---- summed weights of this slice's keys: slots, then the new key at C
-  const float* lg = p.logits + static_cast<size_t>(bg) * G * (C + 1);
   float* cs = p.colsum + static_cast<size_t>(bg) * p.colsum_ld;
-  const int ja = slice * kDecodeSliceKeys;
-  const int jb = min(n + 1, ja + kDecodeSliceKeys);
-#pragma unroll 4
-  for (int j = ja + tid; j < jb; j += kThreads) {
+  float csv[kPer];
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    const int j = ja + tid + r * kThreads;
     float s = 0.f;
-    for (int h = 0; h < G; ++h) s += ex2_approx(lg[static_cast<size_t>(h) * (C + 1) + j] - lse[h]);
-    cs[j < n ? j : C] = s;
+#pragma unroll
+    for (int h = 0; h < G; ++h) s += ex2_approx(lv[r][h] - lse[h]);
+    csv[r] = s;
+    if (j < jb) cs[j < n ? j : C] = s;
   }
-  const bool last_slice = slice == static_cast<int>(gridDim.x) - 1;
   if (last_slice)  // empty slots received nothing
     for (int j = n + tid; j < C; j += kThreads) cs[j] = 0.f;
   if (!p.evict) return;
 
   // ---- eviction
   __syncthreads();  // this CTA's summed weights are written
-  const bool by_score = p.policy == kPolicyH2O;
   const int sinks = p.policy == kPolicySLR ? p.sinks : 0;
   float* score = p.scores + static_cast<size_t>(bg) * C;
   int* pos = p.pos + static_cast<size_t>(bg) * C;
   const size_t row_bytes = static_cast<size_t>(D) * (Q8 ? 1 : sizeof(T));  // cache rows
-  const size_t new_bytes = static_cast<size_t>(D) * sizeof(T);
   char* kc = static_cast<char*>(p.k_cache) + static_cast<size_t>(bg) * C * row_bytes;
   char* vc = static_cast<char*>(p.v_cache) + static_cast<size_t>(bg) * C * row_bytes;
-  const char* kn = static_cast<const char*>(p.k_new) + static_cast<size_t>(bg) * new_bytes;
-  const char* vn = static_cast<const char*>(p.v_new) + static_cast<size_t>(bg) * new_bytes;
-  // the new token's rows into slot `slot`: copied, or quantised (Q8); one warp
+  // the new token's rows into slot `slot`: stored from registers, or
+  // quantised (Q8); warp 0
   auto place_new = [&](int slot) {
     if (!H2O_IN_BOUNDS(slot >= 0 && slot < C, p.state + 2)) return;
     if (Q8) {
-      q8_quantize_row_warp<D>(reinterpret_cast<const __nv_bfloat16*>(kn),
-                              reinterpret_cast<int8_t*>(kc + static_cast<size_t>(slot) * row_bytes),
-                              p.k_scale + static_cast<size_t>(bg) * C + slot, lane);
-      q8_quantize_row_warp<D>(reinterpret_cast<const __nv_bfloat16*>(vn),
-                              reinterpret_cast<int8_t*>(vc + static_cast<size_t>(slot) * row_bytes),
-                              p.v_scale + static_cast<size_t>(bg) * C + slot, lane);
-    } else {
-      copy_row(kc + static_cast<size_t>(slot) * row_bytes, kn, static_cast<int>(row_bytes), lane);
-      copy_row(vc + static_cast<size_t>(slot) * row_bytes, vn, static_cast<int>(row_bytes), lane);
+      const size_t new_off = static_cast<size_t>(bg) * kNewBytes;
+      q8_quantize_row_warp<D>(
+          reinterpret_cast<const __nv_bfloat16*>(static_cast<const char*>(p.k_new) + new_off),
+          reinterpret_cast<int8_t*>(kc + static_cast<size_t>(slot) * row_bytes),
+          p.k_scale + static_cast<size_t>(bg) * C + slot, lane);
+      q8_quantize_row_warp<D>(
+          reinterpret_cast<const __nv_bfloat16*>(static_cast<const char*>(p.v_new) + new_off),
+          reinterpret_cast<int8_t*>(vc + static_cast<size_t>(slot) * row_bytes),
+          p.v_scale + static_cast<size_t>(bg) * C + slot, lane);
+    } else if (lane * 16 < kNewBytes) {
+      *reinterpret_cast<uint4*>(kc + static_cast<size_t>(slot) * row_bytes + lane * 16) = k_row;
+      *reinterpret_cast<uint4*>(vc + static_cast<size_t>(slot) * row_bytes + lane * 16) = v_row;
     }
   };
   if (bg == 0 && slice == 0 && tid == 0) {
     p.state[0] = min(C, n + 1);
     p.state[1] = p.t0 + 1;
   }
-  const int sa = ja, sb = min(jb, n);  // this slice's valid slots
   if (n < C) {  // room left: the new token takes slot n (key n is in the last slice)
-    if (by_score)
-      for (int s = sa + tid; s < sb; s += kThreads) score[s] = __fadd_rn(score[s], cs[s]);
+    if (by_score) {
+#pragma unroll
+      for (int r = 0; r < kPer; ++r) {
+        const int s = ja + tid + r * kThreads;
+        if (s < sb) score[s] = __fadd_rn(sc_old[r], csv[r]);
+      }
+    }
     if (last_slice) {
       if (tid == 0) {
         score[n] = by_score ? cs[C] : 0.f;
@@ -740,11 +835,14 @@ __global__ void __launch_bounds__(kThreads) decode_finish(const DecodeParams p) 
   // the minimum is the lowest value with the highest index.
   const long long limit = static_cast<long long>(p.t0) + 1 - p.W;
   unsigned long long best = ~0ull;
-  for (int s = sa + tid; s < sb; s += kThreads) {
-    const int ps = pos[s];
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    const int s = ja + tid + r * kThreads;
+    if (s >= sb) continue;
+    const int ps = ps_old[r];
     uint32_t rank;
     if (by_score) {
-      const float sc = __fadd_rn(score[s], cs[s]);
+      const float sc = __fadd_rn(sc_old[r], csv[r]);
       score[s] = sc;
       rank = ordered_key(sc);
     } else {
@@ -816,17 +914,8 @@ cudaError_t launch_partial(const DecodeParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <typename T, int D, bool Q8 = false>
-cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
-  cudaError_t e;
-  switch (p.G) {
-    case 1: e = launch_partial<T, D, 1, Q8>(p, st); break;
-    case 2: e = launch_partial<T, D, 2, Q8>(p, st); break;
-    case 4: e = launch_partial<T, D, 4, Q8>(p, st); break;
-    case 8: e = launch_partial<T, D, 8, Q8>(p, st); break;
-    default: return cudaErrorInvalidValue;
-  }
-  if (e != cudaSuccess || kDecodeFused) return e;
+template <typename T, int D, int G, bool Q8>
+cudaError_t launch_finish(const DecodeParams& p, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.n_slices, p.B * p.Hkv);
   cfg.blockDim = dim3(kThreads);
@@ -837,7 +926,25 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_finish<T, D, Q8>, p);
+  return cudaLaunchKernelEx(&cfg, decode_finish<T, D, G, Q8>, p);
+}
+
+template <typename T, int D, int G, bool Q8>
+cudaError_t launch_group(const DecodeParams& p, cudaStream_t st) {
+  const cudaError_t e = launch_partial<T, D, G, Q8>(p, st);
+  if (e != cudaSuccess || kDecodeFused) return e;
+  return launch_finish<T, D, G, Q8>(p, st);
+}
+
+template <typename T, int D, bool Q8 = false>
+cudaError_t launch(const DecodeParams& p, cudaStream_t st) {
+  switch (p.G) {
+    case 1: return launch_group<T, D, 1, Q8>(p, st);
+    case 2: return launch_group<T, D, 2, Q8>(p, st);
+    case 4: return launch_group<T, D, 4, Q8>(p, st);
+    case 8: return launch_group<T, D, 8, Q8>(p, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
