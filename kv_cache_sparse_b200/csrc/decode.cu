@@ -151,8 +151,9 @@ struct PartialLayout {
   static constexpr int kK = 0;                          // [KC][D] cache rows of K; after the
                                                         // logits: [warps][G][D] float sums of P V
   static constexpr int kV = kK + KC * kRow;             // [KC][D] of V
-  static constexpr int kX = kV + KC * kRow;             // [G][KC] float: logits, then P
-  static constexpr int kS = kX + G * KC * 4;            // Q8: [2][KC] float scales of K, V
+  static constexpr int kX = kV + KC * kRow;             // [G][KC] float logits, then
+                                                        // [KC][G] float P (key-major)
+  static constexpr int kS = kX + 2 * G * KC * 4;        // Q8: [2][KC] float scales of K, V
   static constexpr int kN = kS + (Q8 ? 2 * KC * 4 : 0);  // Q8: the new token's K, V rows (T)
   static constexpr int kBytes = kN + (Q8 ? 2 * D * static_cast<int>(sizeof(T)) : 0);
   static_assert(kWarps * G * D * 4 <= KC * kRow, "the P V sums must fit over the K rows");
@@ -468,7 +469,9 @@ __device__ __forceinline__ bool chunk_partial(const DecodeParams& p, int bg, int
     }
   }
   __syncthreads();
-  // ---- chunk max and sum per head (one warp per head), P into xs
+  // ---- chunk max and sum per head (one warp per head), P key-major into
+  // pk, so that P V reads a key's G weights at once
+  float* pk = xs + G * KC;
   if (ok && warp < G) {
     float m = -INFINITY;
     for (int k = lane; k < nkc; k += 32) m = fmaxf(m, xs[warp * KC + k]);
@@ -476,7 +479,7 @@ __device__ __forceinline__ bool chunk_partial(const DecodeParams& p, int bg, int
     float l = 0.f;
     for (int k = lane; k < nkc; k += 32) {
       const float pw = ex2_approx(xs[warp * KC + k] - m);
-      xs[warp * KC + k] = pw;
+      pk[k * G + warp] = pw;
       l += pw;
     }
     l = warp_sum(l);
@@ -495,15 +498,33 @@ __device__ __forceinline__ bool chunk_partial(const DecodeParams& p, int bg, int
 #pragma unroll
     for (int e = 0; e < E; ++e) o[h][e] = 0.f;
   if (ok) {
+#pragma unroll 2
     for (int k = warp; k < nkc; k += kWarps) {
       float vf[E];
       kv_row(k, true, vf);
+      float pw[G];
+      if constexpr (G % 4 == 0) {
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float pw = xs[h * KC + k];
-#pragma unroll
-        for (int e = 0; e < E; ++e) o[h][e] = fmaf(pw, vf[e], o[h][e]);
+        for (int h = 0; h < G; h += 4) {
+          const float4 w = *reinterpret_cast<const float4*>(pk + k * G + h);
+          pw[h] = w.x;
+          pw[h + 1] = w.y;
+          pw[h + 2] = w.z;
+          pw[h + 3] = w.w;
+        }
+      } else if constexpr (G == 2) {
+        const float2 w = *reinterpret_cast<const float2*>(pk + k * G);
+        pw[0] = w.x;
+        pw[1] = w.y;
+      } else {
+        pw[0] = pk[k];
       }
+      // o += P V two elements at a time (the same fused multiply-adds)
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int e = 0; e < E; e += 2)
+          ffma2(o[h][e], o[h][e + 1], pw[h], pw[h], vf[e], vf[e + 1], o[h][e], o[h][e + 1]);
     }
   }
   if (!ok && tid == 0 && rows > 0) {  // a wait gave up: the copies land before their
