@@ -17,6 +17,8 @@ def test_evict_pin(pin):
     dict(seed=10, C=12, W=2, chunk_sizes=(5, 5, 3, 6, 4, 5)),
     dict(seed=11, C=7, W=0, chunk_sizes=(4, 4, 4, 1, 3)),            # partial fill, N_q = 1
     dict(seed=12, C=9, W=6, chunk_sizes=(3, 3, 3, 3, 3)),            # window wider than chunk
+    dict(seed=13, C=6, W=2, chunk_sizes=(6, 1, 1, 1, 1, 1, 1, 1)),   # decode steps on a full cache
+    dict(seed=14, C=5, W=0, chunk_sizes=(5, 1, 1, 1, 1, 1)),         # decode, the new token competes
 ])
 def test_trajectory_token_centric(args):
     pins.check_trajectory(**args)
